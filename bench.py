@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Decode-step throughput of libhata on synthetic HATA workloads.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one hata_decode_step call over one layer's inputs: encode the
+queries, encode + append the new key, Hamming scan with the GQA sum, top-k,
+gather + sparse flash-decode.  Steps cycle over R layer buffers whose touched
+bytes exceed 4x the L2 size, so every step reads its codes and K/V rows from
+HBM.  The K timed steps are CUDA-graph replays bracketed by CUDA events on the
+launching stream, with a device synchronize (and a barrier across ranks) on
+both sides; the time is the max over ranks.
+
+Prints one JSON line.  --impl reference times the CPU oracle on this host
+(rank 0 only) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hata_inputs import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "HATA decode-attn steps/s at 32K-128K ctx; achieved HBM GB/s vs peak"
+DEFAULT_WORKLOAD = "llama8b_128k"
+FALLBACK_HBM_GBS = 6650.0
+GRAPH_CHUNK = 1000  # steps per captured graph
+
+
+# ----------------------------------------------------------------------------
+# byte accounting (algorithmic: r/8 per cached token per KV head, 2*k*d*e of
+# gathered K/V per KV head, plus q and the output)
+# ----------------------------------------------------------------------------
+
+def algorithmic_bytes(wl, seq_lens) -> int:
+    e = wl.elem_bytes
+    total = 0
+    for Lb in seq_lens:
+        Lb = int(Lb)
+        total += wl.n_kv_heads * (Lb * wl.hash_bits // 8 + 2 * min(wl.k, Lb) * wl.head_dim * e)
+    total += 2 * wl.batch * wl.n_q_heads * wl.head_dim * e
+    return total
+
+
+def peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML, the same counters nvidia-smi reads)
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _sample(self):
+        nv = self._nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+        try:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            self.reasons |= nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+            if not self.samples:
+                self._sample()
+
+    def summary(self):
+        if not self._ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing (replicas: no data-path collective)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_config(wl, seq_lens, l2_note):
+    return {
+        "workload": wl.name,
+        "batch": wl.batch,
+        "n_q_heads": wl.n_q_heads,
+        "n_kv_heads": wl.n_kv_heads,
+        "head_dim": wl.head_dim,
+        "seq_len": int(wl.max_seq) if wl.seq_len_range is None else f"ragged {wl.seq_len_range}",
+        "total_cached_tokens": int(np.sum(seq_lens)),
+        "hash_bits": wl.hash_bits,
+        "top_k": wl.k,
+        "kv_dtype": wl.dtype,
+        "l2": l2_note,
+        "parallelism": "replicas",
+    }
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the CPU oracle on this host
+# ----------------------------------------------------------------------------
+
+def oracle_unit_runner(wl, inp):
+    """Returns (run(unit), n_units): run one (batch, KV head) unit of the decode step through the oracle."""
+    import oracle
+
+    G = wl.group
+    units = [(b, g) for b in range(wl.batch) for g in range(wl.n_kv_heads)]
+    prepared = {}
+
+    def prep(u):
+        b, g = units[u % len(units)]
+        if (b, g) not in prepared:
+            Lb = int(inp["seq_lens"][b])
+            K = inp["K"][b:b + 1, g:g + 1]
+            codes, _ = oracle.encode_cache(K, inp["W_H"][g:g + 1], np.array([Lb]))
+            prepared[(b, g)] = (inp["q"][b:b + 1, g * G:(g + 1) * G], K, inp["V"][b:b + 1, g:g + 1],
+                                inp["W_H"][g:g + 1], codes, np.array([Lb]))
+        return prepared[(b, g)]
+
+    def run(u):
+        q, K, V, W, codes, lens = prep(u)
+        t0 = time.perf_counter()
+        oracle.decode_step(q, K, V, W, codes, lens, wl.k)
+        return time.perf_counter() - t0
+
+    return run, prep, len(units)
+
+
+def cpu_baseline(wl, inp, budget_s=15.0, max_units=None):
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(1):
+        run, prep, n_units = oracle_unit_runner(wl, inp)
+        elapsed, done = 0.0, 0
+        limit = n_units if max_units is None else min(max_units, n_units)
+        while done < limit and (elapsed < budget_s or done == 0):
+            prep(done)
+            elapsed += run(done)
+            done += 1
+    steps_per_s = (done / n_units) / elapsed
+    return {
+        "value": steps_per_s,
+        "unit": "steps/s",
+        "cores": 1,
+        "kind": "oracle",
+        "sample": f"{done} of {n_units} (batch, KV head) units of one decode step, float64 numpy, 1 thread",
+    }
+
+
+def run_reference(args, wl):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = make_inputs(wl, seed=args.seed)
+    from threadpoolctl import threadpool_limits
+
+    with threadpool_limits(1):
+        run, prep, n_units = oracle_unit_runner(wl, inp)
+        for u in range(args.warmup):
+            prep(u)
+            run(u)
+        times = []
+        for u in range(args.steps):
+            prep(u)
+            times.append(run(u))
+    total = sum(times)
+    value = (args.steps / n_units) / total
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "steps/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": 1e3 / value,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(wl, inp["seq_lens"], "host CPU"),
+        "cpu_baseline": {
+            "value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"each step = one of {n_units} (batch, KV head) units of one decode step; "
+                      "value scaled to whole steps",
+        },
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+def run_gpu(args, wl):
+    import torch
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    import hash_aware_top_b200 as H
+
+    dev = torch.device("cuda", local)
+    inp = make_inputs(wl, seed=args.seed)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    dims = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.hash_bits, wl.max_seq, wl.dtype)
+    step_bytes = algorithmic_bytes(wl, inp["seq_lens"])
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(4 * l2 / step_bytes)) if args.layers is None else args.layers
+
+    def to_dev(a):
+        return torch.from_numpy(a).to(dev).to(tdt)
+
+    base = {
+        "q": to_dev(inp["q"]), "K": to_dev(inp["K"]), "V": to_dev(inp["V"]),
+        "W": torch.from_numpy(inp["W_H"]).to(dev),
+        "lens": torch.from_numpy(inp["seq_lens"]).to(dev),
+    }
+    ws = torch.empty(H.hata_workspace_size(dims, wl.k), dtype=torch.uint8, device=dev)
+    H.hata_workspace_init(ws)
+    # prefill: encode every cached key through the library
+    codes0 = torch.zeros((wl.batch, wl.n_kv_heads, wl.max_seq, wl.words), dtype=torch.int32, device=dev)
+    H.hata_encode_append(dims, base["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, base["lens"], base["W"], codes0,
+                         wl.max_seq)
+    layers = []
+    for i in range(R):
+        lay = {n: (t if i == 0 else t.clone()) for n, t in base.items()}
+        lay["codes"] = codes0 if i == 0 else codes0.clone()
+        lay["out"] = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=tdt, device=dev)
+        layers.append(lay)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i):
+        L = layers[i % R]
+        H.hata_decode_step(dims, L["q"], L["K"], L["V"], L["W"], L["codes"], L["lens"], wl.k, 0.0, L["out"], None,
+                           None, ws, stream)
+
+    def capture(n, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(first + i)
+        return g
+
+    with torch.cuda.stream(stream):
+        for i in range(3):  # eager calls before capture (first-launch setup)
+            step(i)
+    torch.cuda.synchronize()
+    chunk = min(args.steps, GRAPH_CHUNK)
+    g_chunk = capture(chunk, 0)
+    rem = args.steps % chunk
+    g_rem = capture(rem, 0) if rem else None
+    g_warm = capture(args.warmup, 0) if args.warmup else None
+    torch.cuda.synchronize()
+
+    if g_warm is not None:
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        ev0.record(stream)
+        for _ in range(args.steps // chunk):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if dist:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    status = H.hata_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {H.hata_status_string(status)}")
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # end to end through the public call: pinned host inputs in, output read back, every step
+    e2e_steps = min(args.steps, 300)
+    L0 = layers[0]
+    q_host = L0["q"].cpu().pin_memory()
+    kv_host = torch.stack([torch.stack([L0["K"][b, :, int(inp["seq_lens"][b]) - 1] for b in range(wl.batch)]),
+                           torch.stack([L0["V"][b, :, int(inp["seq_lens"][b]) - 1] for b in range(wl.batch)])]
+                          ).cpu().pin_memory()
+    out_host = torch.empty_like(L0["out"], device="cpu").pin_memory()
+    h2d = q_host.numel() * q_host.element_size() + kv_host.numel() * kv_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for i in range(e2e_steps):
+            L = layers[i % R]
+            L["q"].copy_(q_host, non_blocking=True)
+            for b in range(wl.batch):
+                pos = int(inp["seq_lens"][b]) - 1
+                L["K"][b, :, pos].copy_(kv_host[0, b], non_blocking=True)
+                L["V"][b, :, pos].copy_(kv_host[1, b], non_blocking=True)
+            step(i)
+            out_host.copy_(L["out"], non_blocking=True)
+            stream.synchronize()
+    e2e_s = time.perf_counter() - t0
+    if dist:
+        t = torch.tensor([e2e_s], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_s = float(t.item())
+    e2e_value = world * e2e_steps / e2e_s
+
+    peak, peak_kind = peak_hbm()
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.dtype,
+        "data": "synthetic",
+        "config": workload_config(
+            wl, inp["seq_lens"],
+            f"inputs larger than L2: steps rotate over {R} layer buffers, {R * step_bytes / 1e6:.0f} MB touched "
+            f"per rotation vs {l2 / 1e6:.0f} MB L2"),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "hata_decode_step (whole step)",
+            "achieved": achieved,
+            "peak": peak,
+            "peak_kind": peak_kind,
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": None,
+            "algorithmic_bytes_per_step": step_bytes,
+        },
+        "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, inp)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="hata", choices=["hata", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=None, help="layer buffers to rotate over (default: > 4x L2)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

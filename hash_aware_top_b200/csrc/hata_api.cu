@@ -1,0 +1,172 @@
+// extern "C" entry points of libhata: argument validation, workspace carving,
+// launches.  Nothing here allocates device memory or synchronises (except
+// hata_read_device_status).
+#include <cmath>
+#include <cstdio>
+
+#include "hata_kernels.cuh"
+
+using namespace hata;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+hata_status_t check_dims(const hata_dims_t* d) {
+  if (!d) return HATA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->max_seq < 1 || d->head_dim < 1 ||
+      d->hash_bits < 1)
+    return HATA_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads) return HATA_ERR_INVALID_ARG;
+  if (d->dtype != HATA_F32 && d->dtype != HATA_BF16) return HATA_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return HATA_ERR_UNSUPPORTED;
+  if (d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
+    return HATA_ERR_UNSUPPORTED;
+  const long long G = d->n_q_heads / d->n_kv_heads;
+  if (G > 16 || G * d->hash_bits + 1 > kMaxBins) return HATA_ERR_UNSUPPORTED;
+  return HATA_OK;
+}
+
+hata_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return HATA_OK;
+  return HATA_ERR_CUDA;
+}
+
+WsLayout layout_for(const hata_dims_t& d, int k) { return make_layout(d, k, fused_step_ws_bytes(d, k)); }
+
+hata_status_t check_ws(const hata_dims_t& d, int k, const void* ws, size_t bytes, WsLayout* L) {
+  *L = layout_for(d, k);
+  if (!ws || !aligned16(ws)) return HATA_ERR_WORKSPACE;
+  if (bytes < L->total) return HATA_ERR_WORKSPACE;
+  return HATA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int hata_version(void) { return 100; }
+
+const char* hata_status_string(hata_status_t s) {
+  switch (s) {
+    case HATA_OK: return "ok";
+    case HATA_ERR_INVALID_ARG: return "invalid argument";
+    case HATA_ERR_UNSUPPORTED: return "unsupported shape or type";
+    case HATA_ERR_CUDA: return "CUDA error";
+    case HATA_ERR_TIMEOUT: return "device-side wait timed out";
+    case HATA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+hata_status_t hata_workspace_size(const hata_dims_t* dims, int k, size_t* bytes) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (k < 1 || !bytes) return HATA_ERR_INVALID_ARG;
+  *bytes = layout_for(*dims, k).total;
+  return HATA_OK;
+}
+
+hata_status_t hata_workspace_init(void* ws, size_t bytes, void* stream) {
+  if (!ws || bytes == 0) return HATA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_heads, int x_len, int n_tok,
+                                 const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,
+                                 void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!x || !W_H || !codes || !aligned16(x) || !aligned16(W_H) || !aligned16(codes)) return HATA_ERR_INVALID_ARG;
+  if (x_heads < 1 || x_heads % dims->n_kv_heads || x_len < 1 || codes_len < 1 || n_tok < 0)
+    return HATA_ERR_INVALID_ARG;
+  if (n_tok == 0) return HATA_OK;
+  return cuda_status(launch_encode(*dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_hamming_scores(const hata_dims_t* dims, const uint32_t* qcode, const uint32_t* codes,
+                                  const int32_t* seq_lens, int32_t* scores, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!qcode || !codes || !seq_lens || !scores || !aligned16(codes)) return HATA_ERR_INVALID_ARG;
+  return cuda_status(launch_hamming(*dims, qcode, codes, seq_lens, scores, static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_topk(const hata_dims_t* dims, const int32_t* scores, const int32_t* seq_lens, int k,
+                        int32_t* idx, int32_t* n_sel, void* workspace, size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!scores || !seq_lens || !idx || k < 1) return HATA_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = check_ws(*dims, k, workspace, workspace_bytes, &L)) != HATA_OK) return s;
+  return cuda_status(launch_topk(*dims, L, scores, seq_lens, k, idx, n_sel, static_cast<char*>(workspace),
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_sparse_decode(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                 const int32_t* idx, int k, float scale, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!q || !K || !V || !idx || !out || k < 1) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HATA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return HATA_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = check_ws(*dims, k, workspace, workspace_bytes, &L)) != HATA_OK) return s;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)dims->head_dim);
+  return cuda_status(launch_sparse_decode(*dims, L, q, K, V, idx, k, scale, out, static_cast<char*>(workspace),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                               const float* W_H, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
+                               void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!q || !K || !V || !W_H || !codes || !seq_lens || !out || k < 1) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(W_H) || !aligned16(codes) || !aligned16(out))
+    return HATA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return HATA_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = check_ws(*dims, k, workspace, workspace_bytes, &L)) != HATA_OK) return s;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)dims->head_dim);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+
+  cudaError_t e = launch_fused_step(*dims, L, q, K, V, W_H, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws, st);
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+
+  // Chain of the granular kernels (shapes the fused kernel does not cover).
+  const hata_dims_t& d = *dims;
+  uint32_t* qc = qcode_out ? qcode_out : reinterpret_cast<uint32_t*>(ws + L.qcode);
+  int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  int32_t* sc = reinterpret_cast<int32_t*>(ws + L.scores);
+  if ((e = launch_encode(d, q, d.n_q_heads, 1, 1, nullptr, W_H, qc, 1, st)) != cudaSuccess) return cuda_status(e);
+  if ((e = launch_encode(d, K, d.n_kv_heads, d.max_seq, 1, seq_lens, W_H, codes, d.max_seq, st)) != cudaSuccess)
+    return cuda_status(e);
+  if ((e = launch_hamming(d, qc, codes, seq_lens, sc, st)) != cudaSuccess) return cuda_status(e);
+  if ((e = launch_topk(d, L, sc, seq_lens, k, ix, nullptr, ws, st)) != cudaSuccess) return cuda_status(e);
+  return cuda_status(launch_sparse_decode(d, L, q, K, V, ix, k, scale, out, ws, st));
+}
+
+int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {
+  if (check_dims(dims) != HATA_OK || k < 1) return -1;
+  return fused_step_applies(*dims, k) ? 1 : 6;
+}
+
+hata_status_t hata_read_device_status(void* workspace, void* stream, int* device_status) {
+  if (!workspace || !device_status) return HATA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return HATA_ERR_CUDA;
+  *device_status = (int)v;
+  return HATA_OK;
+}
+
+}  // extern "C"

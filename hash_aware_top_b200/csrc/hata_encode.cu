@@ -1,0 +1,100 @@
+// HashEncode + cache update: y = x . W_H (fp32), bit = [y > 0], LSB-first pack,
+// written straight into the code cache.  One kernel for queries, the appended
+// key and prefill ("HATA" paper notes, 硬件高效优化: projection -> sign ->
+// bitpack -> cache update fused in one kernel).
+//
+// Each CTA owns one (batch, KV group) and a tile of 32 rows of that group (a
+// row is one (head, token) pair; the G query heads of a group share W_H[g]).
+// The tile is staged in shared memory as fp32; thread (slice s, column j)
+// accumulates y_j for rows s, s + NS, ... with exact fp32 FMAs in ascending i,
+// reading W_H[g][i][j] coalesced along j.  The sign bits of 32 consecutive
+// columns are one warp ballot, i.e. one packed word.
+#include "hata_kernels.cuh"
+
+namespace hata {
+
+namespace {
+
+constexpr int kEncThreads = 256;
+constexpr int kEncRows = 32;
+
+template <typename T, int R>
+__global__ void __launch_bounds__(kEncThreads)
+    encode_kernel(const T* __restrict__ x, int x_heads, int x_len, int n_tok, const int32_t* __restrict__ seq_end,
+                  const float* __restrict__ W, uint32_t* __restrict__ codes, int codes_len, int hpg) {
+  constexpr int D = kHeadDim;
+  constexpr int NS = kEncThreads / R;  // row slices
+  constexpr int RPT = kEncRows / NS;   // rows per thread
+  constexpr int NW = R / 32;
+  __shared__ float xs[kEncRows][D];
+
+  const int b = blockIdx.z, g = blockIdx.y;
+  const int rows_total = hpg * n_tok;
+  const int row0 = blockIdx.x * kEncRows;
+  const int end = seq_end ? seq_end[b] : x_len;
+  const int t_lo = end - n_tok;
+  const int lim = min(x_len, codes_len);
+
+  for (int e = threadIdx.x; e < kEncRows * D; e += kEncThreads) {
+    const int rr = e / D, i = e % D, rho = row0 + rr;
+    float v = 0.f;
+    if (rho < rows_total) {
+      const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
+      if (t >= 0 && t < lim) v = to_f32(x[(((size_t)b * x_heads + h) * x_len + t) * D + i]);
+    }
+    xs[rr][i] = v;
+  }
+  __syncthreads();
+
+  const int j = threadIdx.x % R, s = threadIdx.x / R;
+  float acc[RPT];
+#pragma unroll
+  for (int q = 0; q < RPT; ++q) acc[q] = 0.f;
+  const float* Wg = W + (size_t)g * D * R + j;
+#pragma unroll 4
+  for (int i = 0; i < D; ++i) {
+    const float w = __ldg(Wg + (size_t)i * R);
+#pragma unroll
+    for (int q = 0; q < RPT; ++q) acc[q] = fmaf(xs[s + q * NS][i], w, acc[q]);
+  }
+
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < RPT; ++q) {
+    const unsigned word = __ballot_sync(0xffffffffu, acc[q] > 0.f);
+    const int rho = row0 + s + q * NS;
+    if (lane == 0 && rho < rows_total) {
+      const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
+      if (t >= 0 && t < lim) codes[(((size_t)b * x_heads + h) * codes_len + t) * NW + j / 32] = word;
+    }
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok, const int32_t* seq_end,
+                     const float* W, uint32_t* codes, int codes_len, cudaStream_t st) {
+  const int hpg = x_heads / d.n_kv_heads;
+  const long long rows = (long long)hpg * n_tok;
+  dim3 grid((unsigned)((rows + kEncRows - 1) / kEncRows), d.n_kv_heads, d.batch);
+  const T* xp = static_cast<const T*>(x);
+  switch (d.hash_bits) {
+    case 32: encode_kernel<T, 32><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 64: encode_kernel<T, 64><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 128: encode_kernel<T, 128><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 256: encode_kernel<T, 256><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
+                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                          cudaStream_t stream) {
+  if (d.dtype == HATA_BF16)
+    return launch_t<__nv_bfloat16>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, stream);
+  return launch_t<float>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, stream);
+}
+
+}  // namespace hata

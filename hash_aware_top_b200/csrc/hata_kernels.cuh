@@ -1,0 +1,33 @@
+// Internal launchers of libhata's kernels (host side).  Arguments are already
+// validated by hata_api.cu; every launcher returns cudaGetLastError().
+#pragma once
+
+#include "hata_common.cuh"
+
+namespace hata {
+
+cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
+                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                          cudaStream_t stream);
+
+cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,
+                           const int32_t* seq_lens, int32_t* scores, cudaStream_t stream);
+
+cudaError_t launch_topk(const hata_dims_t& d, const WsLayout& L, const int32_t* scores, const int32_t* seq_lens,
+                        int k, int32_t* idx, int32_t* n_sel, char* ws, cudaStream_t stream);
+
+cudaError_t launch_sparse_decode(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K,
+                                 const void* V, const int32_t* idx, int k, float scale, void* out, char* ws,
+                                 cudaStream_t stream);
+
+// Whether the fused decode-step kernel covers these dims and budget.
+bool fused_step_applies(const hata_dims_t& d, int k);
+// Fused decode step: bytes of workspace its plan needs (0 if it does not apply)
+size_t fused_step_ws_bytes(const hata_dims_t& d, int k);
+// Returns cudaErrorNotSupported when the fused kernel does not apply to these dims.
+cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K,
+                              const void* V, const float* W, uint32_t* codes, const int32_t* seq_lens, int k,
+                              float scale, void* out, uint32_t* qcode_out, int32_t* idx_out, char* ws,
+                              cudaStream_t stream);
+
+}  // namespace hata

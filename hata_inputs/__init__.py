@@ -40,6 +40,8 @@ __all__ = [
     "bf16_bits",
     "make_inputs",
     "random_codes",
+    "random_scores",
+    "random_indices",
 ]
 
 N_STREAMS = 8
@@ -172,3 +174,23 @@ def random_codes(shape, hash_bits: int, seed: int = 0) -> np.ndarray:
     """Uniformly random packed codes: uint32 array of shape (*shape, hash_bits // 32)."""
     rng = _streams(seed)[S_CODES]
     return rng.integers(0, 2**32, size=tuple(shape) + (hash_bits // 32,), dtype=np.uint64).astype(np.uint32)
+
+
+def random_scores(shape, max_value: int, seed: int = 0, n_distinct: Optional[int] = None) -> np.ndarray:
+    """Integer scores in [0, max_value] (int32); with n_distinct, drawn from that many values (heavy ties)."""
+    rng = _streams(seed)[S_CODES]
+    if n_distinct is None:
+        return rng.integers(0, max_value, size=shape, endpoint=True).astype(np.int32)
+    vals = rng.choice(max_value + 1, size=min(n_distinct, max_value + 1), replace=False)
+    return vals[rng.integers(0, len(vals), size=shape)].astype(np.int32)
+
+
+def random_indices(n_units: int, L: np.ndarray, k: int, seed: int = 0) -> np.ndarray:
+    """Per unit, min(k, L_u) distinct ascending indices below L_u, -1 padded to k (int32 [n_units][k])."""
+    rng = _streams(seed)[S_CODES]
+    out = np.full((n_units, k), -1, dtype=np.int32)
+    for u in range(n_units):
+        n = min(k, int(L[u]))
+        if n > 0:
+            out[u, :n] = np.sort(rng.choice(int(L[u]), size=n, replace=False))
+    return out

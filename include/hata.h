@@ -1,0 +1,190 @@
+/*
+ * hata.h -- C ABI of libhata, the B200 (sm_100a) decode-step hot path of HATA,
+ * Hash-Aware Top-k Attention.
+ *
+ * Method source: "HATA: Trainable and Hardware-Efficient Hash-Aware Top-k
+ * Attention for Scalable Large Model Inference" (paper notes, ACL 2025).
+ *   - section 方法详解 > 关键设计: the hash h(x) = 2*Sigmoid(sigma * x W_H) - 1 with
+ *     one trainable W_H per attention head; its sign is the code.
+ *   - section 方法详解 > Decode 阶段算法: per decode step, HashEncode the new query
+ *     and key (matrix multiply + Sign + BitPack), append the key code to the
+ *     hash-code cache, Hamming distance bitcount(xor(Q_H, K_H_cache)) against all
+ *     cached codes, aggregate the scores of the query heads that share a KV
+ *     cache (GQA), select top-k, gather those K/V rows and run exact attention.
+ *   - section 硬件高效优化: projection + sign + bitpack + cache update fused in one
+ *     kernel; XOR + popc Hamming operator with coalesced access; gather fused
+ *     into the flash-attention kernel.
+ *
+ * Readings this library fixes where the pages are silent:
+ *   - bit j of a code is [y_j > 0] with y = x . W_H computed in fp32; bit j sits
+ *     in 32-bit word j / 32 at position j % 32 (least significant first);
+ *   - W_H is one [d][r] fp32 matrix per KV head, shared by the G = Hq / Hkv
+ *     query heads of that group and by its keys; query head h is in group h / G;
+ *   - the GQA aggregate is the sum of the G per-head distances, so a score lies
+ *     in [0, G * r]; lower is more similar;
+ *   - top-k keeps the min(k, L_b) tokens with the smallest score; ties go to the
+ *     lower token index; indices are reported in ascending order;
+ *   - attention is softmax(scale * q . K_t) V_t over the selected rows only, fp32
+ *     accumulation, one rounding to the output type; scale <= 0 means 1/sqrt(d);
+ *   - an empty selection (L_b <= 0) gives an all-zero output row.
+ *
+ * Conventions for every call:
+ *   - All tensor arguments are DEVICE pointers owned by the caller.  The library
+ *     allocates no device memory and keeps no global mutable state; scratch
+ *     space is a caller-provided workspace (hata_workspace_size).
+ *   - Every call only enqueues work on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and never synchronises, except
+ *     hata_read_device_status.
+ *   - Host-visible argument errors are reported before anything is launched
+ *     (HATA_ERR_INVALID_ARG / HATA_ERR_UNSUPPORTED); a failed launch reports
+ *     HATA_ERR_CUDA.  Errors that only the device can see (a sequence length
+ *     beyond max_seq, an index outside the cache, a bounded wait that ran out)
+ *     are recorded in the workspace's status word, read with
+ *     hata_read_device_status.  No kernel traps or asserts.
+ *   - Layouts are C-contiguous:
+ *       q, out      [B][Hq][d]            (dtype)
+ *       K, V        [B][Hkv][max_seq][d]  (dtype), one contiguous row per token
+ *       W_H         [Hkv][d][r]           fp32, used as x . W_H
+ *       codes       [B][Hkv][max_seq][r/32] uint32 (the hash-code cache)
+ *       qcode       [B][Hq][r/32]         uint32
+ *       seq_lens    [B]                   int32, cached length incl. the new token
+ *       scores      [B][Hkv][max_seq]     int32
+ *       idx         [B][Hkv][k]           int32, ascending, -1 padded
+ *       n_sel       [B]                   int32, min(k, L_b)
+ *   - Pointers must be 16-byte aligned.
+ */
+#ifndef HATA_H_
+#define HATA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HATA_API __attribute__((visibility("default")))
+#else
+#define HATA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HATA_OK = 0,
+  HATA_ERR_INVALID_ARG = 1, /* bad pointer, size or shape */
+  HATA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim != 128) */
+  HATA_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+  HATA_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up */
+  HATA_ERR_WORKSPACE = 5    /* workspace missing or smaller than hata_workspace_size */
+} hata_status_t;
+
+typedef enum { HATA_F32 = 0, HATA_BF16 = 1 } hata_dtype_t;
+
+/* Problem shape, shared by every call. */
+typedef struct {
+  int batch;      /* B >= 1 */
+  int n_q_heads;  /* Hq >= 1, a multiple of n_kv_heads */
+  int n_kv_heads; /* Hkv >= 1 */
+  int head_dim;   /* d; this version supports 128 */
+  int hash_bits;  /* r in {32, 64, 128, 256} */
+  int max_seq;    /* token capacity of each (b, kv head) cache slab, >= 1 */
+  int dtype;      /* hata_dtype_t of q, K, V and out */
+} hata_dims_t;
+
+/* Bytes of workspace that every call below needs for these dims and budget k
+ * (one size serves all calls).  Returns HATA_OK and writes *bytes. */
+HATA_API hata_status_t hata_workspace_size(const hata_dims_t* dims, int k, size_t* bytes);
+
+/* Zero a workspace before its first use (enqueued memset).  Every call leaves
+ * the workspace's counters back at zero, so this is needed once, and again
+ * only after a call reported HATA_ERR_TIMEOUT. */
+HATA_API hata_status_t hata_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * HashEncode + cache update (Decode 阶段算法, first two steps; 硬件高效优化,
+ * fused projection -> sign -> bitpack -> cache update).  For every batch b,
+ * head h < x_heads and token t in [end_b - n_tok, end_b) that also lies in
+ * [0, min(x_len, codes_len)):
+ *     codes[b][h][t][:] = pack(x[b][h][t][:] . W_H[h / (x_heads / Hkv)] > 0)
+ * with end_b = seq_end[b] if seq_end is not NULL, else x_len.
+ *   x         device [B][x_heads][x_len][d], dims->dtype
+ *   x_heads   Hq to encode queries, Hkv to encode keys (a multiple of Hkv)
+ *   seq_end   device [B] int32 or NULL
+ *   codes     device [B][x_heads][codes_len][r/32] uint32
+ * Typical uses: query codes (x = q, x_heads = Hq, x_len = codes_len = 1,
+ * n_tok = 1, seq_end = NULL); appending the new key (x = K, x_heads = Hkv,
+ * x_len = codes_len = max_seq, n_tok = 1, seq_end = seq_lens); prefill
+ * (same with n_tok = max_seq).  The projection is fp32 (tensor cores with a
+ * three-way bf16 split of W_H for large n_tok, exact fp32 FMA otherwise).
+ */
+HATA_API hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_heads, int x_len, int n_tok,
+                                 const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,
+                                 void* stream);
+
+/*
+ * Hamming scan with the GQA sum (Decode 阶段算法, Hamming and GQA steps;
+ * 硬件高效优化, XOR + popc operator):
+ *     scores[b][g][t] = sum over h in group g of popcount(qcode[b][h] ^ codes[b][g][t])
+ * for t < L_b = min(seq_lens[b], max_seq); entries t >= L_b are not written.
+ */
+HATA_API hata_status_t hata_hamming_scores(const hata_dims_t* dims, const uint32_t* qcode, const uint32_t* codes,
+                                  const int32_t* seq_lens, int32_t* scores, void* stream);
+
+/*
+ * Top-k select (Decode 阶段算法, top-k step): for each (b, g), the min(k, L_b)
+ * tokens t < L_b with the smallest scores[b][g][t], ties to the lower t, written
+ * in ascending t to idx[b][g][0 .. n-1]; idx[b][g][n .. k-1] = -1.  n_sel[b]
+ * (nullable) receives n.  Scores must lie in [0, G * r] (values outside are
+ * clamped and flagged in the workspace status word).
+ */
+HATA_API hata_status_t hata_topk(const hata_dims_t* dims, const int32_t* scores, const int32_t* seq_lens, int k,
+                        int32_t* idx, int32_t* n_sel, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Gather-fused sparse flash-decode (Decode 阶段算法, gather + sparse attention;
+ * 硬件高效优化, gather fused into flash attention): for each b and query head h
+ * in group g,
+ *     out[b][h] = sum_j softmax_j(scale * q[b][h] . K[b][g][t_j]) V[b][g][t_j]
+ * over the entries t_j = idx[b][g][j], j < k, with t_j >= 0 (negative entries
+ * are padding).  Entries >= max_seq are skipped and flagged in the workspace
+ * status word.  scale <= 0 selects 1/sqrt(d).
+ */
+HATA_API hata_status_t hata_sparse_decode(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                 const int32_t* idx, int k, float scale, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * The whole decode step in one call (Decode 阶段算法 end to end, with the
+ * fusions of 硬件高效优化): encode the queries; encode the new key K[b][g][L_b-1]
+ * and write its code to codes[b][g][L_b-1]; Hamming scan with the GQA sum over
+ * t < L_b; top-k; gather + attention into out.  The new token is a candidate
+ * like any other.  Results equal the chain hata_encode_append ->
+ * hata_hamming_scores -> hata_topk -> hata_sparse_decode bit for bit in codes
+ * and indices.  qcode_out ([B][Hq][r/32]) and idx_out ([B][Hkv][k]) are
+ * optional copies of the intermediates (NULL to skip).
+ */
+HATA_API hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                               const float* W_H, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
+                               void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* Number of kernels one hata_decode_step call with these dims and k enqueues
+ * (1 when the fused persistent kernel applies), or -1 for invalid dims. */
+HATA_API int hata_decode_step_kernel_count(const hata_dims_t* dims, int k);
+
+/* Wait for `stream`, then return the workspace's device status word (a
+ * hata_status_t recorded by a kernel, HATA_OK if none) in *device_status and
+ * clear it.  The only call that synchronises. */
+HATA_API hata_status_t hata_read_device_status(void* workspace, void* stream, int* device_status);
+
+/* Static description of a status code. */
+HATA_API const char* hata_status_string(hata_status_t status);
+
+/* Library version as 10000 * major + 100 * minor + patch. */
+HATA_API int hata_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HATA_H_ */
