@@ -44,6 +44,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhata.so"
 
 HATA_OK, HATA_ERR_INVALID_ARG, HATA_ERR_UNSUPPORTED, HATA_ERR_CUDA, HATA_ERR_TIMEOUT, HATA_ERR_WORKSPACE = range(6)
 HATA_F32, HATA_BF16 = 0, 1
+HATA_FLAG_EARLY_PREFETCH = 1
 
 EXPORTED_SYMBOLS = (
     "hata_workspace_size",
@@ -75,6 +76,7 @@ class Dims(ctypes.Structure):
         ("hash_bits", ctypes.c_int),
         ("max_seq", ctypes.c_int),
         ("dtype", ctypes.c_int),
+        ("flags", ctypes.c_int),
     ]
 
     @property
@@ -127,12 +129,12 @@ def hata_version() -> int:
     return lib.hata_version()
 
 
-def dims_for(batch, n_q_heads, n_kv_heads, head_dim, hash_bits, max_seq, dtype) -> Dims:
+def dims_for(batch, n_q_heads, n_kv_heads, head_dim, hash_bits, max_seq, dtype, flags=0) -> Dims:
     if isinstance(dtype, torch.dtype):
         dtype = HATA_F32 if dtype == torch.float32 else HATA_BF16 if dtype == torch.bfloat16 else -1
     elif isinstance(dtype, str):
         dtype = {"f32": HATA_F32, "bf16": HATA_BF16}[dtype]
-    return Dims(batch, n_q_heads, n_kv_heads, head_dim, hash_bits, max_seq, dtype)
+    return Dims(batch, n_q_heads, n_kv_heads, head_dim, hash_bits, max_seq, dtype, flags)
 
 
 def _check(status: int, where: str):

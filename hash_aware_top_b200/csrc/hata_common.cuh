@@ -143,11 +143,42 @@ __device__ __forceinline__ void load_code(const uint32_t* p, uint32_t (&w)[NW]) 
   }
 }
 
-// Query-side state of one KV group for the per-token score.
-//   G % 4 == 0 : G/4 quads (2 popc per word each)
-//   G == 2     : popc(q0^q1) + 2 popc((q0^k) & (q1^k))   (1 popc per word)
-//   G == 1     : popc(q0^k)
+// Sum of popcounts of N words.  Groups of three words go through a carry-save
+// adder first (x0 + x1 + x2 = xor3 + 2 * maj3, two LOP3 each), which trades
+// one popc (16 per clock per SM) for two logic ops (64 per clock per SM); three
+// adders per eight words balance the two pipes.
+template <int N>
+__device__ __forceinline__ int popc_sum(const uint32_t (&x)[N]) {
+  if constexpr (N == 1) {
+    return __popc(x[0]);
+  } else if constexpr (N == 2) {
+    return __popc(x[0]) + __popc(x[1]);
+  } else if constexpr (N == 4) {
+    const uint32_t s = x[0] ^ x[1] ^ x[2], c = (x[0] & x[1]) | (x[2] & (x[0] ^ x[1]));
+    return __popc(s) + __popc(x[3]) + 2 * __popc(c);
+  } else if constexpr (N == 8) {
+    const uint32_t s1 = x[0] ^ x[1] ^ x[2], c1 = (x[0] & x[1]) | (x[2] & (x[0] ^ x[1]));
+    const uint32_t s2 = x[3] ^ x[4] ^ x[5], c2 = (x[3] & x[4]) | (x[5] & (x[3] ^ x[4]));
+    const uint32_t s3 = s1 ^ s2 ^ x[6], c3 = (s1 & s2) | (x[6] & (s1 ^ s2));
+    return __popc(s3) + __popc(x[7]) + 2 * (__popc(c1) + __popc(c2) + __popc(c3));
+  } else {
+    static_assert(N % 8 == 0, "popc_sum: N must be 1, 2, 4 or a multiple of 8");
+    int s = 0;
+#pragma unroll
+    for (int i = 0; i < N; i += 8) {
+      const uint32_t y[8] = {x[i], x[i + 1], x[i + 2], x[i + 3], x[i + 4], x[i + 5], x[i + 6], x[i + 7]};
+      s += popc_sum<8>(y);
+    }
+    return s;
+  }
+}
+
+// Query-side state of one KV group for the per-token score D = sum_h popc(q_h ^ k).
+//   G % 4 == 0 : G/4 quads, each 2 weight-2 words per code word (QuadWord)
+//   G == 2     : popc(q0 ^ q1) + 2 popc((q0 ^ k) & (q1 ^ k))
+//   G == 1     : popc(q0 ^ k)
 //   G == 0     : runtime group size, plain sum over heads (codes in shared memory)
+// The per-token words are summed with popc_sum (carry-save, see above).
 template <int NW, int G>
 struct GroupQuery {
   static constexpr int NQ = G >= 4 ? G / 4 : 1;
@@ -180,27 +211,71 @@ struct GroupQuery {
   }
 
   __device__ __forceinline__ int score(const uint32_t (&k)[NW], const uint32_t* qg, int g_rt) const {
-    int s = cst;
     if constexpr (G % 4 == 0 && G > 0) {
+      uint32_t x[2 * NQ * NW];
 #pragma unroll
       for (int u = 0; u < NQ; ++u)
 #pragma unroll
-        for (int w = 0; w < NW; ++w) s += quad_word_var(quad[u][w], k[w]);
+        for (int w = 0; w < NW; ++w) {
+          x[2 * (u * NW + w)] = quad[u][w].M ^ k[w];
+          x[2 * (u * NW + w) + 1] = (quad[u][w].Q ^ k[w]) & (quad[u][w].q3 ^ k[w]);
+        }
+      return cst + 2 * popc_sum<2 * NQ * NW>(x);
     } else if constexpr (G == 2) {
+      uint32_t x[NW];
 #pragma unroll
-      for (int w = 0; w < NW; ++w) s += 2 * __popc((a[w] ^ k[w]) & (c[w] ^ k[w]));
+      for (int w = 0; w < NW; ++w) x[w] = (a[w] ^ k[w]) & (c[w] ^ k[w]);
+      return cst + 2 * popc_sum<NW>(x);
     } else if constexpr (G == 1) {
+      uint32_t x[NW];
 #pragma unroll
-      for (int w = 0; w < NW; ++w) s += __popc(a[w] ^ k[w]);
+      for (int w = 0; w < NW; ++w) x[w] = a[w] ^ k[w];
+      return popc_sum<NW>(x);
     } else {
+      int s = 0;
       for (int h = 0; h < g_rt; ++h)
 #pragma unroll
         for (int w = 0; w < NW; ++w) s += __popc(qg[h * NW + w] ^ k[w]);
+      return s;
     }
-    return s;
   }
 };
 
+// y = sum_{i < 128} x[i] * w[i] computed by one warp in a fixed order: lane l
+// accumulates x[l + 32u] * w[l + 32u] for u = 0..3 with fp32 FMAs (u
+// ascending, starting from the u = 0 product), then the 32 partial sums are
+// combined by a xor butterfly over offsets 16, 8, 4, 2, 1 (every lane ends with
+// the same value, since each step adds two equal operand pairs).  Every kernel
+// that encodes a decode-time vector uses this function, so query and key codes
+// are bit-identical across the granular and the fused paths.
+__device__ __forceinline__ float warp_dot128(const float* x, const float* w, int lane) {
+  float p = x[lane] * w[lane];
+  p = fmaf(x[lane + 32], w[lane + 32], p);
+  p = fmaf(x[lane + 64], w[lane + 64], p);
+  p = fmaf(x[lane + 96], w[lane + 96], p);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+  return p;
+}
+
+// warp_dot128 for N (x, w) pairs at once: the same operations per pair, in
+// the same order, interleaved so that the shuffle chains overlap.
+template <int N>
+__device__ __forceinline__ void warp_dot128_multi(const float* const (&x)[N], const float* const (&w)[N], int lane,
+                                                  float (&y)[N]) {
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    float p = x[j][lane] * w[j][lane];
+    p = fmaf(x[j][lane + 32], w[j][lane + 32], p);
+    p = fmaf(x[j][lane + 64], w[j][lane + 64], p);
+    p = fmaf(x[j][lane + 96], w[j][lane + 96], p);
+    y[j] = p;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1)
+#pragma unroll
+    for (int j = 0; j < N; ++j) y[j] += __shfl_xor_sync(0xffffffffu, y[j], o);
+}
 
 // Block-wide exclusive prefix sum over NT threads (NT a multiple of 32).
 // `warp_sums` is shared scratch of NT / 32 ints.  Returns this thread's

@@ -1,14 +1,20 @@
 // HashEncode + cache update: y = x . W_H (fp32), bit = [y > 0], LSB-first pack,
-// written straight into the code cache.  One kernel for queries, the appended
-// key and prefill ("HATA" paper notes, 硬件高效优化: projection -> sign ->
-// bitpack -> cache update fused in one kernel).
+// written straight into the code cache ("HATA" paper notes, 硬件高效优化:
+// projection -> sign -> bitpack -> cache update fused in one kernel).
 //
-// Each CTA owns one (batch, KV group) and a tile of 32 rows of that group (a
-// row is one (head, token) pair; the G query heads of a group share W_H[g]).
-// The tile is staged in shared memory as fp32; thread (slice s, column j)
-// accumulates y_j for rows s, s + NS, ... with exact fp32 FMAs in ascending i,
-// reading W_H[g][i][j] coalesced along j.  The sign bits of 32 consecutive
-// columns are one warp ballot, i.e. one packed word.
+// Two forms, chosen by the number of tokens per sequence:
+//   * decode form (n_tok <= kDecodeTok): the few rows of a call (G query heads,
+//     or one new key per KV head) are latency-bound, so the work is spread over
+//     one CTA per (32-column word, KV group, batch).  Each CTA stages its rows
+//     and its 32 columns of W_H (transposed) in shared memory and every (row,
+//     column) projection is one warp_dot128 -- the same arithmetic as the fused
+//     decode step, so both paths produce identical codes.
+//   * prefill form: each CTA owns one (batch, KV group) and a tile of 32 rows;
+//     thread (slice s, column j) accumulates y_j for rows s, s + NS, ... with
+//     fp32 FMAs in ascending i, reading W_H[g][i][j] coalesced along j; the sign
+//     bits of 32 consecutive columns are one warp ballot, i.e. one packed word.
+// The two forms round differently, so a key encoded by both can differ only in
+// bits whose projection is within fp32 rounding of zero.
 #include "hata_kernels.cuh"
 
 namespace hata {
@@ -17,6 +23,56 @@ namespace {
 
 constexpr int kEncThreads = 256;
 constexpr int kEncRows = 32;
+constexpr int kDecodeTok = 4;     // decode form up to this many tokens per sequence
+constexpr int kDecRows = 16;      // rows per decode-form CTA
+
+template <typename T>
+__global__ void __launch_bounds__(kEncThreads)
+    encode_decode_kernel(const T* __restrict__ x, int x_heads, int x_len, int n_tok,
+                         const int32_t* __restrict__ seq_end, const float* __restrict__ W,
+                         uint32_t* __restrict__ codes, int codes_len, int hpg, int R) {
+  constexpr int D = kHeadDim;
+  __shared__ float xs[kDecRows][D];
+  __shared__ float ws[32][D];
+  __shared__ uint32_t words[kDecRows];
+  const int w = blockIdx.x, g = blockIdx.y;
+  const int b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nbz = (hpg * n_tok + kDecRows - 1) / kDecRows;
+  const int bb = b / nbz, row0 = (b % nbz) * kDecRows;
+  const int rows_total = hpg * n_tok;
+  const int end = seq_end ? seq_end[bb] : x_len;
+  const int t_lo = end - n_tok;
+  const int lim = min(x_len, codes_len);
+  for (int e = tid; e < kDecRows * D; e += kEncThreads) {
+    const int rr = e / D, i = e % D, rho = row0 + rr;
+    float v = 0.f;
+    if (rho < rows_total) {
+      const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
+      if (t >= 0 && t < lim) v = to_f32(x[(((size_t)bb * x_heads + h) * x_len + t) * D + i]);
+    }
+    xs[rr][i] = v;
+  }
+  const float* Wg = W + (size_t)g * D * R + 32 * w;
+  for (int e = tid; e < 32 * D; e += kEncThreads) {
+    const int i = e / 32, c = e % 32;
+    ws[c][i] = __ldg(Wg + (size_t)i * R + c);
+  }
+  if (tid < kDecRows) words[tid] = 0u;
+  __syncthreads();
+  const int nrows = min(kDecRows, rows_total - row0);
+  for (int pr = warp; pr < nrows * 32; pr += kEncThreads / 32) {
+    const int rr = pr / 32, c = pr % 32;
+    const float y = warp_dot128(xs[rr], ws[c], lane);
+    if (lane == 0 && y > 0.f) atomicOr(&words[rr], 1u << c);
+  }
+  __syncthreads();
+  if (tid < nrows) {
+    const int rho = row0 + tid;
+    const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
+    if (t >= 0 && t < lim) codes[(((size_t)bb * x_heads + h) * codes_len + t) * (R / 32) + w] = words[tid];
+  }
+}
 
 template <typename T, int R>
 __global__ void __launch_bounds__(kEncThreads)
@@ -74,6 +130,13 @@ template <typename T>
 cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok, const int32_t* seq_end,
                      const float* W, uint32_t* codes, int codes_len, cudaStream_t st) {
   const int hpg = x_heads / d.n_kv_heads;
+  if (n_tok <= kDecodeTok) {
+    const int nbz = (hpg * n_tok + kDecRows - 1) / kDecRows;
+    dim3 grid(d.hash_bits / 32, d.n_kv_heads, d.batch * nbz);
+    encode_decode_kernel<T><<<grid, kEncThreads, 0, st>>>(static_cast<const T*>(x), x_heads, x_len, n_tok, seq_end,
+                                                          W, codes, codes_len, hpg, d.hash_bits);
+    return cudaGetLastError();
+  }
   const long long rows = (long long)hpg * n_tok;
   dim3 grid((unsigned)((rows + kEncRows - 1) / kEncRows), d.n_kv_heads, d.batch);
   const T* xp = static_cast<const T*>(x);

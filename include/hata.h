@@ -89,7 +89,19 @@ typedef struct {
   int hash_bits;  /* r in {32, 64, 128, 256} */
   int max_seq;    /* token capacity of each (b, kv head) cache slab, >= 1 */
   int dtype;      /* hata_dtype_t of q, K, V and out */
+  int flags;      /* HATA_FLAG_* bits, 0 for none */
 } hata_dims_t;
+
+/* hata_decode_step is launched with programmatic dependent launch: it waits for
+ * the kernel before it on the stream to finish before reading anything.  With
+ * HATA_FLAG_EARLY_PREFETCH it instead starts reading seq_lens, W_H and the
+ * cached codes of slots [0, L_b - 1) while that kernel is still running, and
+ * waits only before it reads q, the new K/V row or writes anything.  Set the
+ * flag only when the preceding kernel writes none of seq_lens, W_H and those
+ * code slots -- e.g. when it is the projection that produces q and the new
+ * K/V row.  It must not be set when the preceding kernel is a decode step or an
+ * encode of the same cache. */
+#define HATA_FLAG_EARLY_PREFETCH 1
 
 /* Bytes of workspace that every call below needs for these dims and budget k
  * (one size serves all calls).  Returns HATA_OK and writes *bytes. */

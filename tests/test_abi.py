@@ -57,7 +57,7 @@ def test_version_and_status_strings(H):
     ],
 )
 def test_workspace_size_validates_dims(H, dims, status):
-    d = H.Dims(*dims)
+    d = H.Dims(*dims, 0)
     n = ctypes.c_size_t(0)
     assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == status
     if status == 0:
@@ -107,3 +107,11 @@ def test_binding_refuses_cpu_tensors(H):
     with pytest.raises(ValueError, match="CUDA tensor"):
         H.hata_hamming_scores(d, torch.zeros(1, 4, 4, dtype=torch.int32), torch.zeros(1, 1, 64, 4, dtype=torch.int32),
                               torch.zeros(1, dtype=torch.int32), torch.zeros(1, 1, 64, dtype=torch.int32))
+
+
+def test_unknown_flags_rejected(H):
+    n = ctypes.c_size_t(0)
+    d = H.dims_for(1, 32, 8, 128, 128, 1024, "bf16", flags=H.HATA_FLAG_EARLY_PREFETCH)
+    assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 0
+    d.flags = 6
+    assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 1

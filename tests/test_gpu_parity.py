@@ -232,7 +232,18 @@ STEP_CASES = {
     "tiny_f32_4k": Workload("tiny_f32_4k", 1, 1, 1, 128, 4096, 128, 256, "f32", n_planted=40),
     "llama_shape_9k": Workload("llama_shape_9k", 1, 32, 8, 128, 9000, 128, 512, "bf16"),
     "ragged_b3": Workload("ragged_b3", 3, 8, 2, 128, 12000, 128, 1024, "bf16", seq_len_range=(300, 12000)),
-    "narrow32": Workload("narrow32", 2, 8, 2, 128, 8192, 32, 256, "bf16"),
+    "narrow32": Workload("narrow32", 2, 8, 2, 128, 8192, 32, 256, "bf16", seq_len_range=(5000, 8192)),
+    "g3_chain": Workload("g3_chain", 2, 6, 2, 128, 3000, 128, 100, "bf16", seq_len_range=(1500, 3000)),
+    "short_lens": Workload("short_lens", 6, 8, 2, 128, 64, 128, 16, "bf16", seq_len_range=(1, 64), n_planted=2),
+    "budget_gt_slice": Workload("budget_gt_slice", 1, 8, 2, 128, 3000, 128, 2048, "f32"),
+    "r32_g8_f32": Workload("r32_g8_f32", 2, 16, 2, 128, 6000, 32, 300, "f32", seq_len_range=(3001, 6000)),
+    # many units -> small clusters with more than 8192 tokens per CTA (multi-pass selection)
+    "many_units_fallback": Workload("many_units_fallback", 16, 8, 2, 128, 40000, 128, 600, "bf16",
+                                    seq_len_range=(20000, 40000)),
+    "many_units_covered": Workload("many_units_covered", 16, 8, 2, 128, 40000, 128, 40, "bf16",
+                                   seq_len_range=(20000, 40000)),
+    "narrow_many_units": Workload("narrow_many_units", 8, 16, 4, 128, 30000, 32, 900, "bf16",
+                                  seq_len_range=(15001, 30000)),
     "r64_g2": Workload("r64_g2", 2, 4, 2, 128, 5000, 64, 300, "f32"),
     "r256_g8": Workload("r256_g8", 1, 8, 1, 128, 5000, 256, 128, "bf16"),
 }
@@ -345,3 +356,8 @@ def test_decode_step_flags_length_beyond_cache(H):
     codes0 = random_codes((1, 1, 256), 128, seed=2)
     got = run_step(H, wl, inp, codes0)
     assert H.hata_read_device_status(got["ws"]) == H.HATA_ERR_INVALID_ARG
+
+
+def test_kernel_count_reports_fused_and_chain(H):
+    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 1
+    assert H.hata_decode_step_kernel_count(H.dims_for(1, 6, 2, 128, 128, 3000, "bf16"), 100) == 6
