@@ -29,6 +29,7 @@ __all__ = [
     "hata_encode_append",
     "hata_hamming_scores",
     "hata_topk",
+    "hata_topk_noalloc",
     "hata_sparse_decode",
     "hata_decode_step",
     "hata_read_device_status",
@@ -58,6 +59,7 @@ EXPORTED_SYMBOLS = (
     "hata_status_string",
     "hata_version",
     "hata_decode_step_kernel_count",
+    "hata_topk_noalloc",
 )
 
 
@@ -110,6 +112,7 @@ def _load():
         "hata_status_string": (ctypes.c_char_p, [I]),
         "hata_version": (I, []),
         "hata_decode_step_kernel_count": (I, [DP, I]),
+        "hata_topk_noalloc": (I, [DP, P, P, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -227,6 +230,23 @@ def hata_topk(dims: Dims, scores, seq_lens, k, idx, n_sel, ws, stream=None):
             _ptr(n_sel, "n_sel", (d.batch,), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_topk")
+
+
+def hata_topk_noalloc(dims: Dims, scores, seq_lens, k, idx, n_sel, stream=None):
+    """hata_topk with the library's built-in scratch instead of a workspace: nothing is allocated.
+
+    For callers that cannot allocate device memory.  Calls on one device share the scratch, so they must not
+    overlap on the GPU; the first call on a device should come before any stream capture.
+    """
+    d = dims
+    _check(
+        lib.hata_topk_noalloc(
+            ctypes.byref(d),
+            _ptr(scores, "scores", (d.batch, d.n_kv_heads, d.max_seq), torch.int32),
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k),
+            _ptr(idx, "idx", (d.batch, d.n_kv_heads, k), torch.int32),
+            _ptr(n_sel, "n_sel", (d.batch,), torch.int32, optional=True), _stream(stream)),
+        "hata_topk_noalloc")
 
 
 def hata_sparse_decode(dims: Dims, q, K, V, idx, k, scale, out, ws, stream=None):

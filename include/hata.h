@@ -180,6 +180,21 @@ HATA_API hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, 
                                void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/*
+ * hata_topk without a workspace, for callers that cannot allocate device memory
+ * (no counterpart on the pages: it only changes where scratch lives).  Same
+ * inputs, outputs and results as hata_topk.  Its scratch is one 8 MiB array of
+ * device memory owned by the library, present on every GPU that loads it until
+ * the process exits.  Problems whose scratch would exceed it return
+ * HATA_ERR_WORKSPACE before any launch.  The first call on a device looks up
+ * the array's address (that device current): make it before any stream
+ * capture.  All calls on a device share the array, so calls whose work
+ * overlaps on the GPU race; each call clears the counters it needs.  Device-side
+ * argument errors of this call are not reported.  Allocates nothing.
+ */
+HATA_API hata_status_t hata_topk_noalloc(const hata_dims_t* dims, const int32_t* scores, const int32_t* seq_lens,
+                                         int k, int32_t* idx, int32_t* n_sel, void* stream);
+
 /* Number of kernels one hata_decode_step call with these dims and k enqueues
  * (1 when the fused persistent kernel applies), or -1 for invalid dims. */
 HATA_API int hata_decode_step_kernel_count(const hata_dims_t* dims, int k);
