@@ -2,26 +2,26 @@
 // (batch, KV head) unit ("HATA" paper notes, Decode 阶段算法 end to end, with the
 // fusions of 硬件高效优化).
 //
-// A unit's L cached tokens are split evenly over the CS CTAs of its cluster
-// (CS = 16 for a single long sequence).  Each CTA:
-//   1. streams its slice of the code cache into a 4-stage shared-memory ring with
-//      bulk (TMA) copies, evict-first in L2, issued before anything else;
-//   2. meanwhile encodes the G queries and the new key for its r / CS columns of
-//      W_H (warp_dot128: the same arithmetic as hata_encode_append's decode
-//      form) and stores its code bits into a per-source slot of every CTA of the
-//      cluster; after a cluster barrier each CTA ORs the slots locally, and the
-//      CTA owning slot L - 1 appends the key code to the cache;
+// A unit's L cached tokens are split evenly over the CS CTAs of its cluster.
+// Each CTA:
+//   1. streams its slice of the code cache into a 4-8 stage shared-memory ring
+//      with bulk (TMA) copies, evict-first in L2, issued as soon as L is known;
+//   2. encodes the G queries and the new key for its slice of the W_H columns
+//      (warp_dot128: the same arithmetic as hata_encode_append's decode form),
+//      stores its code bits into a per-source slot of every CTA of the cluster;
+//      after a cluster barrier each CTA ORs the slots locally, and the CTA
+//      owning slot L - 1 appends the key code to the cache;
 //   3. scores every token of its slice (xor + popc with the GQA sum folded into
 //      per-word constants and a carry-save popc sum), keeping the u16 scores and
 //      their histogram in shared memory; warps release ring stages on their own;
-//   4. guesses its own share of the selection from the local histogram and
+//   4. turns the histogram into a cumulative one and stores it (u16) into its
+//      slot of every CTA; guesses its own share of the selection from it and
 //      starts gathering those candidate K/V rows (cp.async) right away;
-//   5. finds the unit's threshold T (the smallest score with at least
-//      n = min(k, L) tokens at or below it), the tie quota m, and the counts of
-//      earlier CTAs, in two rounds of stores into every CTA's slots: coarse
-//      histograms (bins of 16 scores), then the 16 fine bins of the coarse bin
-//      holding the threshold.  Ties go to the lower token index exactly as in a
-//      global sort;
+//   5. after a cluster barrier, every CTA sums the CS cumulative histograms
+//      (one bin per thread) to find the unit's threshold T (the smallest score
+//      with at least n = min(k, L) tokens at or below it), the tie quota m and
+//      the counts of earlier CTAs, so ties go to the lower token index exactly
+//      as in a global sort;
 //   6. computes the flash-decode partial (max, sum, weighted V) of each of the G
 //      query heads over its selected rows (falling back to a second gather when
 //      the guess missed), and stores each partial's column slice into the CTA
@@ -46,14 +46,14 @@ namespace {
 
 constexpr int kFThreads = 512;
 constexpr int kNWarp = kFThreads / 32;
-constexpr int kMaxStages = 8;        // ring stages (16 KB each), 4..8 depending on shared memory left
-constexpr int kMinStages = 4;
-constexpr int kStageBytes = 16384;
-constexpr int kRingBytes = kMinStages * kStageBytes;  // ring part reused for gathered rows
-constexpr int kTokCap = 65536;        // max tokens per CTA (u16 score array)
+constexpr int kMaxStages = 6;        // ring stages (32 KB each), 2..6 depending on shared memory left
+constexpr int kMinStages = 2;
+constexpr int kStageBytes = 32768;
+constexpr int kTokCap = 65520;       // max tokens per CTA: u16 scores and u16 cumulative counts
+constexpr int kWCols = 32;           // W_H columns staged per encode batch
+constexpr int kMaxCS = 16;           // largest cluster
+constexpr int kMaxGB = 256;          // largest gather batch (rows)
 constexpr int kOneCtaSmem = 116 * 1024;  // dynamic shared memory that keeps one CTA per SM
-constexpr int kWCols = 32;            // W_H columns staged per encode batch
-constexpr int kCoarse = 16;           // scores per coarse histogram bin
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct FusedParams {
@@ -72,8 +72,8 @@ struct FusedParams {
 };
 
 struct SmemLayout {
-  uint32_t ring, D, hist, xs, wsl, enc, qslot, sel, lg, part, cslot, fslot, mslot, stat, mbar, total;
-  int ncb, mcols;
+  uint32_t ring, D, hist, hslot, xs, wsl, enc, qslot, sel, lg, part, mslot, stat, mbar, total;
+  int nbp, mcols, gb;
 };
 
 struct Bump {
@@ -86,8 +86,6 @@ struct Bump {
   }
 };
 
-__host__ __device__ inline int gather_rows(int esize) { return kRingBytes / (2 * kHeadDim * esize); }
-
 // W_H columns encoded by each CTA of a cluster of CS: ceil(r / CS) rounded up to
 // a multiple of 4 (the last ranks may get fewer, or none).
 __host__ __device__ inline int enc_cols_per_cta(int R, int CS) { return ((R + CS - 1) / CS + 3) / 4 * 4; }
@@ -99,28 +97,29 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int 
                                                   int wcols, int CS, int stages) {
   SmemLayout s;
   Bump b;
-  s.ncb = (nbins + kCoarse - 1) / kCoarse;
+  s.nbp = (nbins + 7) / 8 * 8;  // histogram bins padded to whole 16-byte groups of u16
   s.mcols = merge_cols(G, CS);
+  s.gb = stages * kStageBytes / (2 * kHeadDim * esize);
+  if (s.gb > kMaxGB) s.gb = kMaxGB;
   s.ring = b.take(stages * kStageBytes, 128);
   s.D = b.take(tok_cap * 2, 16);
-  s.hist = b.take(s.ncb * kCoarse * 4, 16);           // local counts, padded to whole coarse bins
+  s.hist = b.take(s.nbp * 4, 16);                     // local counts, then cumulative, then unit totals
+  s.hslot = b.take(CS * s.nbp * 2, 16);               // u16 cumulative histograms from every CTA
   s.xs = b.take((G + 1) * kHeadDim * 4, 16);          // G queries + new key, fp32
   s.wsl = b.take(wcols * kHeadDim * 4, 16);           // W_H column slice, transposed
   s.enc = b.take((G + 1) * NW * 4, 16);               // this CTA's code bits
   s.qslot = b.take(CS * (G + 1) * NW * 4, 16);        // code bits from every CTA
   s.sel = b.take(sel_cap * 4, 16);                    // selected rows (fallback path)
-  s.lg = b.take(G * gather_rows(esize) * 4, 16);      // logits / probabilities
-  s.part = b.take(G * (kHeadDim + 2) * 4, 16);        // running (max, sum) per head
-  s.cslot = b.take(CS * s.ncb * 4, 16);               // coarse histograms from every CTA
-  s.fslot = b.take(CS * kCoarse * 4, 16);             // fine bins of the threshold bin
+  s.lg = b.take(G * s.gb * 4, 16);                    // logits / probabilities
+  s.part = b.take(G * 4 * 4, 16);                     // running (max, sum, alpha) per head
   s.mslot = b.take(CS * (s.mcols + 2 * G) * 4, 16);   // partials for this CTA's output columns
   s.stat = b.take(16 * 4, 16);
-  s.mbar = b.take(kMaxStages * 8, 8);
+  s.mbar = b.take((kMaxStages + 1) * 8, 8);  // ring stages + the row-gather barrier
   s.total = b.take(0, 128);
   return s;
 }
 
-enum { ST_T = 0, ST_M, ST_LESS_BEFORE, ST_EQ_BEFORE, ST_SPEC, ST_ABORT, ST_J, ST_BELOWJ, ST_LESSJ, ST_MYLESS, ST_TMP_EQ };
+enum { ST_T = 0, ST_M, ST_LESS_BEFORE, ST_EQ_BEFORE, ST_SPEC, ST_ABORT, ST_MYLESS, ST_MYEQ, ST_NBELOW };
 
 template <typename T>
 struct Vec16;  // 16-byte vector of T as fp32
@@ -128,6 +127,15 @@ template <>
 struct Vec16<__nv_bfloat16> {
   __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&o)[8]) {
     const uint4 v = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(h[j]);
+      o[2 * j] = f.x;
+      o[2 * j + 1] = f.y;
+    }
+  }
+  __device__ __forceinline__ static void convert(const uint4& v, float (&o)[8]) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -146,6 +154,12 @@ struct Vec16<float> {
     o[2] = v.z;
     o[3] = v.w;
   }
+  __device__ __forceinline__ static void convert(const uint4& v, float (&o)[4]) {
+    o[0] = __uint_as_float(v.x);
+    o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z);
+    o[3] = __uint_as_float(v.w);
+  }
 };
 
 template <typename T, int NW, int G>
@@ -154,23 +168,26 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   constexpr int D = kHeadDim;
   constexpr int ESZ = (int)sizeof(T);
   constexpr int ST = kStageBytes / (4 * NW);      // tokens per ring stage
-  constexpr int GB = kRingBytes / (2 * D * ESZ);  // gathered rows per batch (K and V)
-  constexpr int CPR = D * ESZ / 16;               // 16-byte chunks per row
   constexpr int NV = G + 1;                       // encoded vectors: G queries + new key
   constexpr int BULK_Q = NW >= 4 ? 1 : 4 / NW;    // tokens per 16 bytes
   constexpr int XV = NV * D * ESZ / 16;           // 16-byte vectors of q + new key
+  constexpr int QV = G * D * ESZ / 16;            // ... of which the queries
   constexpr int EPV = 16 / ESZ;                   // elements per 16-byte vector
-  constexpr int SEGT = 8;                         // threads per row in the logits
-  constexpr int SEGE = D / SEGT;                  // elements per thread in the logits
+  constexpr int LT = 16;                          // threads per row in the logits
+  constexpr int LE = D / LT;                      // elements per thread in the logits (8)
+  constexpr int PVG = kFThreads / (D / 2);        // row groups in P.V (8): thread = (column pair, row group)
+  static_assert(XV <= kFThreads, "one vector of q / new key per thread");
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int CS = (int)ptx::cluster_nctarank();
   const int rank = (int)ptx::cluster_ctarank();
   const int kStages = p.stages;
   const SmemLayout S = smem_layout(G, NW, ESZ, p.tok_cap, p.sel_cap, p.nbins, p.wcols, CS, kStages);
+  const int GB = S.gb, nbp = S.nbp;
   unsigned char* ring = smem + S.ring;
   uint16_t* Ds = reinterpret_cast<uint16_t*>(smem + S.D);
   int* hist = reinterpret_cast<int*>(smem + S.hist);
+  uint16_t* hslot = reinterpret_cast<uint16_t*>(smem + S.hslot);
   float* xs = reinterpret_cast<float*>(smem + S.xs);
   float* wsl = reinterpret_cast<float*>(smem + S.wsl);
   uint32_t* enc = reinterpret_cast<uint32_t*>(smem + S.enc);
@@ -178,43 +195,42 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   int* sel = reinterpret_cast<int*>(smem + S.sel);
   float* lg = reinterpret_cast<float*>(smem + S.lg);
   float* part = reinterpret_cast<float*>(smem + S.part);
-  int* cslot = reinterpret_cast<int*>(smem + S.cslot);
-  int* fslot = reinterpret_cast<int*>(smem + S.fslot);
   float* mslot = reinterpret_cast<float*>(smem + S.mslot);
   int* stat = reinterpret_cast<int*>(smem + S.stat);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + S.mbar);
   __shared__ int warp_sums[kNWarp];
   __shared__ int done[kMaxStages];
-  __shared__ int cand[GB];
-  __shared__ uint8_t candf[GB];
+  __shared__ int cand[kMaxGB];
+  __shared__ uint8_t candf[kMaxGB];
   __shared__ uint32_t qc[NV * NW];
 
   const int u = blockIdx.x / CS;
   const int b = u / p.Hkv, g = u % p.Hkv;
   const bool early = (p.flags & HATA_FLAG_EARLY_PREFETCH) != 0;
-  const int ncb = S.ncb;
 
   ptx::cluster_arrive_relaxed();  // completed by the wait before the first remote store
   if (!early) ptx::pdl_wait();
   ptx::pdl_launch_dependents();
 
-  // W_H slice loads go out first: they depend on nothing
+  // ---- 1. first wave of loads: W_H slice, seq_lens; then the codes stream -----
   const int R = NW * 32;
   const int cpr = enc_cols_per_cta(R, CS);  // a multiple of 4: 16-byte aligned W_H slices
   const int j0 = rank * cpr;
   const int ncols = max(0, min(cpr, R - j0));  // the last ranks may get fewer (or no) columns
   const uint64_t pol_keep = ptx::policy_evict_last();
   const float* Wg = p.W + (size_t)g * D * R + j0;
-  const int nc0 = min(p.wcols, ncols);
-  const bool wvec = nc0 % 4 == 0;
+  const int nc0 = min(p.wcols, ncols);  // a multiple of 4
   float4 wv[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int e = tid + q * kFThreads;
     wv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (wvec && e < D * nc0 / 4) wv[q] = ptx::ld_f4_policy(Wg + (size_t)(e / (nc0 / 4)) * R + (e % (nc0 / 4)) * 4, pol_keep);
+    if (e < D * nc0 / 4) wv[q] = ptx::ld_f4_policy(Wg + (size_t)(e / (nc0 / 4)) * R + (e % (nc0 / 4)) * 4, pol_keep);
   }
-
+  // query vectors do not depend on L: load them now unless they may still be being written
+  const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+  if (!early && tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
   const int L = clamp_len(p.seq_lens, b, p.max_seq, p.status);
   int C = (L + CS - 1) / CS;
   C = (C + 15) & ~15;
@@ -222,10 +238,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int nmine = t1 - t0;
   const int nst = (nmine + ST - 1) / ST;
   uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;
-
-  // ---- 1. stream this CTA's codes into the ring (bulk copies) ----------------
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) ptx::mbar_init(&mbar[s], 1);
+    ptx::mbar_init(&mbar[kMaxStages], 1);
     ptx::fence_mbarrier_init();
   }
   if (tid < kStages) done[tid] = 0;
@@ -244,10 +259,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     for (int s = 0; s < min(nst, kStages); ++s) issue(s);
 
   // ---- 2. encode the G queries and the new key, this CTA's column slice --------
+  if (early) {
+    ptx::pdl_wait();  // q and the new key row come from the preceding kernel
+    if (tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
+  }
+  {
+    const T* kn = static_cast<const T*>(p.K) + (((size_t)u * p.max_seq) + (L > 0 ? L - 1 : 0)) * D;
+    if (tid >= QV && tid < XV && L > 0) xv = reinterpret_cast<const uint4*>(kn)[tid - QV];
+  }
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const int e = tid + q * kFThreads;
-    if (wvec && e < D * nc0 / 4) {
+    if (e < D * nc0 / 4) {
       const int i = e / (nc0 / 4), c4 = (e % (nc0 / 4)) * 4;
       wsl[(c4 + 0) * D + i] = wv[q].x;
       wsl[(c4 + 1) * D + i] = wv[q].y;
@@ -255,23 +278,17 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       wsl[(c4 + 3) * D + i] = wv[q].w;
     }
   }
-  if (early) ptx::pdl_wait();  // q and the new key row come from the preceding kernel
-  const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
-  const T* kn = static_cast<const T*>(p.K) + (((size_t)u * p.max_seq) + (L > 0 ? L - 1 : 0)) * D;
   if (tid < XV) {
-    const int e = tid * EPV, v = e / D, i = e % D;
     float xe[EPV];
+    Vec16<T>::convert(xv, xe);
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) xe[j] = 0.f;
-    if (v < G || L > 0) Vec16<T>::load(v < G ? qg + (size_t)v * D + i : kn + i, xe);
-#pragma unroll
-    for (int j = 0; j < EPV; ++j) xs[e + j] = xe[j];
+    for (int j = 0; j < EPV; ++j) xs[tid * EPV + j] = xe[j];
   }
   if (tid < NV * NW) enc[tid] = 0u;
-  for (int v = tid; v < ncb * kCoarse; v += kFThreads) hist[v] = 0;
+  for (int v = tid; v < nbp; v += kFThreads) hist[v] = 0;
   for (int cb = 0; cb < ncols; cb += p.wcols) {
     const int nc = min(p.wcols, ncols - cb);
-    if (cb > 0 || !wvec) {  // further column batches (small clusters) or unaligned slices: scalar staging
+    if (cb > 0) {  // further column batches (small clusters): scalar staging
       __syncthreads();
       for (int e = tid; e < D * nc; e += kFThreads) {
         const int i = e / nc, c = e % nc;
@@ -292,8 +309,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       }
       float y[4];
       warp_dot128_multi<4>(xp, wp, lane, y);
-      if (lane < nd && y[lane & 3] > 0.f) {
-        // lane j (< nd) publishes pair j's bit
+      float yl = y[0];
+#pragma unroll
+      for (int j = 1; j < 4; ++j) yl = lane == j ? y[j] : yl;
+      if (lane < nd && yl > 0.f) {  // lane j (< nd) publishes pair j's bit
         const int dj = d0 + lane, col = j0 + cb + dj % nc;
         atomicOr(&enc[(dj / nc) * NW + (col >> 5)], 1u << (col & 31));
       }
@@ -301,8 +320,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   __syncthreads();
   ptx::cluster_wait();  // every CTA of the cluster has started
-  // store this CTA's bits into slot `rank` of every CTA
-  for (int e = tid; e < NV * NW * CS; e += kFThreads) {
+  for (int e = tid; e < NV * NW * CS; e += kFThreads) {  // this CTA's bits into slot `rank` of every CTA
     const int w = e % (NV * NW), c = e / (NV * NW);
     ptx::st_dsmem_u32(ptx::dsmem_addr(&qslot[rank * NV * NW + w], c), enc[w]);
   }
@@ -323,116 +341,145 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     uint32_t keyc[NW];
 #pragma unroll
     for (int w = 0; w < NW; ++w) keyc[w] = qc[G * NW + w];
+    // Each thread scores TPS tokens of a stage (all loads first, then the
+    // arithmetic, for ILP).  Warps release stages on their own: lane 0 adds to the
+    // stage's counter and checks the returned count one stage later, so no lane
+    // waits on the atomic; the warp that completed a stage refills it.
+    constexpr int TPS = ST / kFThreads;
+    int rel_old = -1, rel_s = -1;  // lane 0: ticket of the previous stage's release
     for (int s = 0; s < nst; ++s) {
-      if (!ptx::mbar_wait_bounded(&mbar[s % kStages], (uint32_t)(s / kStages) & 1u, kWaitTries)) {
+      if (!ptx::mbar_wait_spin(&mbar[s % kStages], (uint32_t)(s / kStages) & 1u, kWaitTries)) {
         set_status(p.status, HATA_ERR_TIMEOUT);
         stat[ST_ABORT] = 1;
       }
       const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
       const int nb = nt / BULK_Q * BULK_Q;
       const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + (s % kStages) * kStageBytes);
-      for (int i = tid; i < nt; i += kFThreads) {
-        uint32_t kw[NW];
+      uint32_t kw[TPS][NW];
+#pragma unroll
+      for (int j = 0; j < TPS; ++j) {
+        const int i = tid + j * kFThreads;
         if (i < nb) {
           if constexpr (NW >= 4) {
 #pragma unroll
             for (int w4 = 0; w4 < NW / 4; ++w4) {
               const uint4 v4 = reinterpret_cast<const uint4*>(buf + (size_t)i * NW)[w4];
-              kw[4 * w4] = v4.x;
-              kw[4 * w4 + 1] = v4.y;
-              kw[4 * w4 + 2] = v4.z;
-              kw[4 * w4 + 3] = v4.w;
+              kw[j][4 * w4] = v4.x;
+              kw[j][4 * w4 + 1] = v4.y;
+              kw[j][4 * w4 + 2] = v4.z;
+              kw[j][4 * w4 + 3] = v4.w;
             }
+          } else if constexpr (NW == 2) {
+            const uint2 v2 = reinterpret_cast<const uint2*>(buf + (size_t)i * NW)[0];
+            kw[j][0] = v2.x;
+            kw[j][1] = v2.y;
           } else {
-#pragma unroll
-            for (int w = 0; w < NW; ++w) kw[w] = buf[(size_t)i * NW + w];
+            kw[j][0] = buf[i];
           }
-        } else {
+        } else if (i < nt) {
 #pragma unroll
-          for (int w = 0; w < NW; ++w) kw[w] = cu[(size_t)(ts + i) * NW + w];
+          for (int w = 0; w < NW; ++w) kw[j][w] = cu[(size_t)(ts + i) * NW + w];
         }
-        if (ts + i == L - 1) {
+      }
 #pragma unroll
-          for (int w = 0; w < NW; ++w) kw[w] = keyc[w];
+      for (int j = 0; j < TPS; ++j) {
+        const int i = tid + j * kFThreads;
+        if (i < nt) {
+          const int dv = gq.score(kw[j], qc, G);  // <= G * r by construction
+          Ds[ts + i - t0] = (uint16_t)dv;
+          atomicAdd(&hist[dv], 1);
         }
-        const int dv = min(gq.score(kw, qc, G), p.nbins - 1);
-        Ds[ts + i - t0] = (uint16_t)dv;
-        atomicAdd(&hist[dv], 1);
       }
       __syncwarp();
       if (lane == 0) {
-        // the last warp to finish this stage refills its buffer (counters never reset:
-        // the k-th use of buffer s % kStages ends when the count reaches k * kNWarp)
-        const int old = atomicAdd(&done[s % kStages], 1);
-        if (old == ((s / kStages) + 1) * kNWarp - 1 && s + kStages < nst) {
+        // counters never reset: the k-th use of buffer s % kStages ends at count k * kNWarp
+        if (rel_s >= 0 && rel_old == ((rel_s / kStages) + 1) * kNWarp - 1 && rel_s + kStages < nst) {
           ptx::fence_proxy_async_smem();
-          issue(s + kStages);
+          issue(rel_s + kStages);
         }
+        rel_old = atomicAdd(&done[s % kStages], 1);
+        rel_s = s;
       }
-    }
-  }
-  __syncthreads();
-
-  // ---- 4. local guess of this CTA's share of the selection ---------------------
-  const int n = min(p.k, L);
-  {
-    // coarse counts of this CTA (one thread per coarse bin) and the local guess:
-    // enough rows for twice this CTA's fair share of the budget
-    int* ccl = reinterpret_cast<int*>(lg);  // [ncb] scratch (lg is unused until the logits)
-    for (int j = tid; j < ncb; j += kFThreads) {
-      int c = 0;
-#pragma unroll
-      for (int i = 0; i < kCoarse; ++i) c += hist[j * kCoarse + i];
-      ccl[j] = c;
     }
     __syncthreads();
-    // coarse histograms to every CTA (slot `rank`)
-    for (int e = tid; e < ncb * CS; e += kFThreads) {
-      const int j = e % ncb, c = e / ncb;
-      ptx::st_dsmem_u32(ptx::dsmem_addr(&cslot[rank * ncb + j], c), (uint32_t)ccl[j]);
-    }
-    if (warp == 0) {
-      const int want = min(nmine, min(GB / 2, 2 * ((n + CS - 1) / CS) + 8));
-      int run = 0, spec = p.nbins;
-      // walk the coarse bins 32 at a time, then the fine bins of the crossing one
-      for (int j0c = 0; j0c < ncb && spec == p.nbins && want > 0; j0c += 32) {
-        const int j = j0c + lane;
-        const int c = j < ncb ? ccl[j] : 0;
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const unsigned hit = __ballot_sync(0xffffffffu, run + incl >= want);
-        if (hit) {
-          const int jl = __ffs(hit) - 1;
-          const int before = run + __shfl_sync(0xffffffffu, incl - c, jl);
-          const int jj = j0c + jl;
-          // fine bins of coarse bin jj (16 lanes)
-          const int f = lane < kCoarse ? hist[jj * kCoarse + lane] : 0;
-          int fi = f;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, fi, o);
-            if (lane >= o) fi += y;
-          }
-          const unsigned fh = __ballot_sync(0xffffffffu, lane < kCoarse && before + fi >= want);
-          spec = jj * kCoarse + (__ffs(fh) - 1);
-        }
-        run += __shfl_sync(0xffffffffu, incl, 31);
+    // the ring (or global memory) may have held the old code of slot L - 1: rescore it
+    // with the appended key code and move its histogram count
+    if (own_last && tid == 0) {
+      const int d_new = gq.score(keyc, qc, G), d_old = Ds[L - 1 - t0];
+      if (d_new != d_old) {
+        Ds[L - 1 - t0] = (uint16_t)d_new;
+        hist[d_old] -= 1;
+        hist[d_new] += 1;
       }
-      if (lane == 0) stat[ST_SPEC] = spec;
     }
   }
   __syncthreads();
+
+  // ---- 4. cumulative histogram -> every CTA; local guess; speculative gather ---
+  const int n = min(p.k, L);
+  {
+    // inclusive cumulative counts in place (each thread a contiguous span of bins)
+    const int span = (nbp + kFThreads - 1) / kFThreads;
+    const int v0 = min(nbp, tid * span), v1 = min(nbp, v0 + span);
+    int local = 0;
+    for (int v = v0; v < v1; ++v) local += hist[v];
+    int total;
+    int run = block_exclusive_scan<kFThreads>(local, warp_sums, &total);
+    // guess: enough local rows for about 1.5x this CTA's fair share of the budget
+    const int want = min(nmine, min(GB, 5 * ((n + CS - 1) / CS) / 4 + 8));
+    if (tid == 0) stat[ST_SPEC] = want > 0 ? INT_MAX : -1;
+    __syncthreads();
+    for (int v = v0; v < v1; ++v) {
+      const int before = run;
+      run += hist[v];
+      hist[v] = run;
+      if (want > 0 && before < want && run >= want) stat[ST_SPEC] = v;
+    }
+  }
+  __syncthreads();
+  // u16 cumulative histogram into slot `rank` of every CTA (8 bins per 16-byte store)
+  for (int e = tid; e < (nbp / 8) * CS; e += kFThreads) {
+    const int v8 = e % (nbp / 8), c = e / (nbp / 8);
+    uint4 pk;
+    const int* h = hist + v8 * 8;
+    pk.x = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+    pk.y = (uint32_t)h[2] | ((uint32_t)h[3] << 16);
+    pk.z = (uint32_t)h[4] | ((uint32_t)h[5] << 16);
+    pk.w = (uint32_t)h[6] | ((uint32_t)h[7] << 16);
+    ptx::st_dsmem_v4(ptx::dsmem_addr(&hslot[rank * nbp + v8 * 8], c), pk);
+  }
   const int Tspec = stat[ST_SPEC];
 
-  // ---- 5. speculative gather of the candidates (score <= Tspec), up to GB rows ---
   const T* Kb = static_cast<const T*>(p.K) + (size_t)u * p.max_seq * D;
   const T* Vb = static_cast<const T*>(p.V) + (size_t)u * p.max_seq * D;
   T* Kr = reinterpret_cast<T*>(ring);
   T* Vr = reinterpret_cast<T*>(ring) + (size_t)GB * D;
+  // Row gathers: one bulk copy per K row and per V row, all completing on the
+  // gather mbarrier (one phase per gather).  An index outside this CTA's slice
+  // (never expected) is flagged and replaced by row t0, so the byte count holds.
+  uint64_t* gbar = &mbar[kMaxStages];
+  uint32_t gphase = 0;
+  const uint64_t pol_rows = ptx::policy_evict_first();
+  auto gather = [&](const int* list, int nr) {
+    if (tid == 0) ptx::mbar_arrive_expect_tx(gbar, (uint32_t)(2 * nr * D * ESZ));
+    for (int e = tid; e < 2 * nr; e += kFThreads) {
+      const int r = e >> 1;
+      int t = list[r];
+      if (t < t0 || t >= t1) {
+        set_status(p.status, HATA_ERR_INVALID_ARG);
+        t = t0;
+      }
+      if (e & 1) ptx::bulk_g2s(Vr + (size_t)r * D, Vb + (size_t)t * D, D * ESZ, gbar, pol_rows);
+      else ptx::bulk_g2s(Kr + (size_t)r * D, Kb + (size_t)t * D, D * ESZ, gbar, pol_rows);
+    }
+  };
+  auto gather_wait = [&]() {
+    if (!ptx::mbar_wait_spin(gbar, gphase & 1u, kWaitTries)) {
+      set_status(p.status, HATA_ERR_TIMEOUT);
+      stat[ST_ABORT] = 1;
+    }
+    ++gphase;
+  };
   // Passes over this CTA's scores go 8192 at a time: each thread owns 16
   // consecutive scores of the pass (two 16-byte loads); scores past nmine read as 0xffff.
   constexpr int TPT = 16, CHUNK = kFThreads * TPT;
@@ -452,7 +499,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     }
   };
   int ncand = 0;
-  for (int base = 0; base < nmine; base += CHUNK) {
+  for (int base = 0; base < nmine && Tspec >= 0; base += CHUNK) {
     uint16_t dv[TPT];
     load16(base, dv);
     int mine = 0;
@@ -472,115 +519,60 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   ncand = min(ncand, GB);
   if (stat[ST_ABORT]) ncand = 0;  // a bulk copy never completed: the ring may still be written
   __syncthreads();
-  for (int e = tid; e < ncand * CPR; e += kFThreads) {
-    const int r = e / CPR, c = e % CPR;
-    const int t = cand[r];
-    if (t < t0 || t >= t1) {  // never: candidates are this CTA's own tokens
-      set_status(p.status, HATA_ERR_INVALID_ARG);
-      continue;
-    }
-    ptx::cp_async16(reinterpret_cast<char*>(Kr + (size_t)r * D) + 16 * c, reinterpret_cast<const char*>(Kb + t * D) + 16 * c);
-    ptx::cp_async16(reinterpret_cast<char*>(Vr + (size_t)r * D) + 16 * c, reinterpret_cast<const char*>(Vb + t * D) + 16 * c);
-  }
+  gather(cand, ncand);  // speculative: waited for in section 8
 
-  // ---- 6. threshold, round 1: coarse histograms of every CTA ---------------------
-  ptx::cluster_sync();  // #2
-  if (warp == 0) {
-    // coarse bin J holding the threshold, the count below it, and this CTA's share
-    // of the tokens below it in earlier CTAs
-    int run = 0, J = ncb - 1, belowJ = 0;
-    bool found = n == 0;
-    if (n == 0) J = 0;
-    for (int j0c = 0; j0c < ncb && !found; j0c += 32) {
-      const int j = j0c + lane;
-      int c = 0;
-      if (j < ncb)
-        for (int cc = 0; cc < CS; ++cc) c += cslot[cc * ncb + j];
-      int incl = c;
+  // ---- 5. unit threshold from the CS cumulative histograms -------------------
+  ptx::cluster_sync();  // #2: every CTA holds every CTA's cumulative histogram
+  {
+    // unit totals, one bin per thread; T = number of bins whose cumulative total is below n
+    int below = 0;
+    for (int v = tid; v < nbp; v += kFThreads) {
+      int cv[kMaxCS];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      const unsigned hit = __ballot_sync(0xffffffffu, j < ncb && run + incl >= n);
-      if (hit) {
-        const int jl = __ffs(hit) - 1;
-        J = j0c + jl;
-        belowJ = run + __shfl_sync(0xffffffffu, incl - c, jl);
-        found = true;
-      }
-      run += __shfl_sync(0xffffffffu, incl, 31);
-    }
-    // tokens of earlier CTAs in coarse bins below J, and of this CTA
-    int lessJ = 0, myless = 0;
-    for (int e = lane; e < J * (rank + 1); e += 32) {
-      const int cc = e / max(J, 1), j = e % max(J, 1);
-      const int v = cslot[cc * ncb + j];
-      if (cc < rank) lessJ += v;
-      else myless += v;
+      for (int c = 0; c < kMaxCS; ++c) cv[c] = c < CS ? (int)hslot[c * nbp + v] : 0;
+      int tv = 0;
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) tv += cv[c];
+      hist[v] = tv;  // the local counts are no longer needed (this CTA's are in hslot[rank])
+      below += (v < p.nbins && tv < n);
     }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      lessJ += __shfl_xor_sync(0xffffffffu, lessJ, o);
-      myless += __shfl_xor_sync(0xffffffffu, myless, o);
+    for (int o = 16; o; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+    if (lane == 0) warp_sums[warp] = below;
+    __syncthreads();
+    if (warp == 0) {
+      int Tth = lane < kNWarp ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) Tth += __shfl_xor_sync(0xffffffffu, Tth, o);
+      const int Tc = min(Tth, p.nbins - 1);
+      // per source CTA (lane c): cumulative count below T and at T
+      int cb = 0, ce = 0;
+      if (lane < CS) {
+        cb = Tc > 0 ? (int)hslot[lane * nbp + Tc - 1] : 0;
+        ce = (int)hslot[lane * nbp + Tc] - cb;
+      }
+      const int lb = __reduce_add_sync(0xffffffffu, lane < rank ? cb : 0);
+      const int eb = __reduce_add_sync(0xffffffffu, lane < rank ? ce : 0);
+      const int myl = __shfl_sync(0xffffffffu, cb, rank);
+      const int mye = __shfl_sync(0xffffffffu, ce, rank);
+      if (lane == 0) {
+        stat[ST_T] = n == 0 ? 0 : Tth;
+        stat[ST_M] = n == 0 ? 0 : n - (Tc > 0 ? hist[Tc - 1] : 0);
+        stat[ST_LESS_BEFORE] = lb;
+        stat[ST_EQ_BEFORE] = eb;
+        stat[ST_MYLESS] = myl;
+        stat[ST_MYEQ] = mye;
+      }
     }
-    if (lane == 0) {
-      stat[ST_J] = J;
-      stat[ST_BELOWJ] = belowJ;
-      stat[ST_LESSJ] = lessJ;
-      stat[ST_MYLESS] = myless;
-    }
-    __syncwarp();
-    // round 2 payload: this CTA's fine counts of coarse bin J to every CTA
-    for (int e = lane; e < kCoarse * CS; e += 32) {
-      const int i = e % kCoarse, c = e / kCoarse;
-      ptx::st_dsmem_u32(ptx::dsmem_addr(&fslot[rank * kCoarse + i], c), (uint32_t)hist[J * kCoarse + i]);
-    }
+    __syncthreads();
   }
-  ptx::cluster_sync();  // #3
-  if (warp == 0) {
-    const int J = stat[ST_J], belowJ = stat[ST_BELOWJ];
-    // lane i < 16: fine bin i of coarse bin J summed over CTAs; before / mine parts
-    int tot = 0, before = 0, mine = 0;
-    if (lane < kCoarse)
-      for (int cc = 0; cc < CS; ++cc) {
-        const int v = fslot[cc * kCoarse + lane];
-        tot += v;
-        if (cc < rank) before += v;
-        if (cc == rank) mine = v;
-      }
-    int incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const unsigned hit = __ballot_sync(0xffffffffu, lane < kCoarse && belowJ + incl >= n);
-    const int it = n == 0 ? 0 : (hit ? __ffs(hit) - 1 : kCoarse - 1);
-    const int T_ = n == 0 ? 0 : J * kCoarse + it;
-    const int m_ = n - (belowJ + __shfl_sync(0xffffffffu, incl - tot, it));
-    // earlier CTAs: below T inside bin J, and equal to T; this CTA likewise
-    const int lb = __reduce_add_sync(0xffffffffu, lane < it ? before : 0);
-    const int eb = __shfl_sync(0xffffffffu, before, it);
-    const int ml = __reduce_add_sync(0xffffffffu, lane < it ? mine : 0);
-    const int me = __shfl_sync(0xffffffffu, mine, it);
-    if (lane == 0) {
-      stat[ST_T] = T_;
-      stat[ST_M] = n == 0 ? 0 : m_;
-      stat[ST_LESS_BEFORE] = stat[ST_LESSJ] + lb;
-      stat[ST_EQ_BEFORE] = eb;
-      stat[ST_MYLESS] = stat[ST_MYLESS] + ml;
-      stat[ST_TMP_EQ] = me;
-    }
-  }
-  __syncthreads();
   const int Tt = stat[ST_T], m = stat[ST_M];
   const int less_before = stat[ST_LESS_BEFORE], eq_before = stat[ST_EQ_BEFORE];
   const int sel_before = less_before + min(eq_before, m);
-  const int ties_here = max(0, min(m - eq_before, stat[ST_TMP_EQ]));
+  const int ties_here = max(0, min(m - eq_before, stat[ST_MYEQ]));
   const int nsel_here = stat[ST_MYLESS] + ties_here;  // this CTA's share of the selection
   // the candidates cover the selection when every selected score is <= Tspec and none was cut off
-  const bool covered = !truncated && Tt <= Tspec;
+  const bool covered = nsel_here == 0 || (!truncated && Tt <= Tspec);
 
   // ---- 7. ascending indices (only when asked for) and the row list --------------
   int32_t* ix = p.idx_out ? p.idx_out + (size_t)u * p.k : nullptr;
@@ -640,65 +632,63 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
 #pragma unroll
   for (int q = 0; q < OPT; ++q) oacc[q] = 0.f;
   if (tid < G) {
-    part[tid * (D + 2)] = -INFINITY;
-    part[tid * (D + 2) + 1] = 0.f;
+    part[tid * 4] = -INFINITY;
+    part[tid * 4 + 1] = 0.f;
   }
   const int nrows_total = covered ? ncand : (stat[ST_ABORT] ? 0 : min(nsel_here, p.sel_cap));
+  gather_wait();  // the speculative rows (they were issued before the threshold was known)
   for (int r0 = 0; r0 < nrows_total; r0 += GB) {
     const int nr = min(GB, nrows_total - r0);
-    if (!covered) {
-      ptx::cp_async_wait_all();  // speculative copies land before the buffers are reused
-      __syncthreads();
-      for (int e = tid; e < nr * CPR; e += kFThreads) {
-        const int r = e / CPR, c = e % CPR;
-        const int t = sel[r0 + r];
-        if (t < t0 || t >= t1) {  // never: every listed row is one of this CTA's selected tokens
-          set_status(p.status, HATA_ERR_INVALID_ARG);
-          continue;
-        }
-        ptx::cp_async16(reinterpret_cast<char*>(Kr + (size_t)r * D) + 16 * c, reinterpret_cast<const char*>(Kb + t * D) + 16 * c);
-        ptx::cp_async16(reinterpret_cast<char*>(Vr + (size_t)r * D) + 16 * c, reinterpret_cast<const char*>(Vb + t * D) + 16 * c);
-      }
+    if (!covered) {  // the guess missed: gather the selected rows batch by batch
+      __syncthreads();  // previous batch's readers are done with the buffers
+      gather(sel + r0, nr);
+      gather_wait();
     }
-    ptx::cp_async_wait_all();
     __syncthreads();
-    // logits (exp2 domain): 8 threads per row, 16 elements each, all G heads at once
-    for (int rb = warp * (32 / SEGT); rb < nr; rb += kFThreads / SEGT) {  // warp-uniform trip count
-      const int r = rb + lane / SEGT, sgi = lane % SEGT;
-      const bool valid = r < nr;
-      float kv[SEGE];
-#pragma unroll
-      for (int v = 0; v < SEGE / EPV; ++v) {
-        float t8[EPV];
-#pragma unroll
-        for (int j = 0; j < EPV; ++j) t8[j] = 0.f;
-        if (valid) Vec16<T>::load(Kr + (size_t)r * D + sgi * SEGE + v * EPV, t8);
-#pragma unroll
-        for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
-      }
-      float acc[G];
+    // logits (exp2 domain): 16 threads per row, 8 elements each, every head at once;
+    // each thread keeps its 8-element slice of the G query vectors in registers
+    {
+      const int sgi = lane % LT;
+      float xq[G][LE];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        const float4* xq = reinterpret_cast<const float4*>(xs + h * D + sgi * SEGE);
-        float a = 0.f;
-#pragma unroll
-        for (int v = 0; v < SEGE / 4; ++v) {
-          const float4 x4 = xq[v];
-          a = fmaf(x4.x, kv[4 * v], a);
-          a = fmaf(x4.y, kv[4 * v + 1], a);
-          a = fmaf(x4.z, kv[4 * v + 2], a);
-          a = fmaf(x4.w, kv[4 * v + 3], a);
-        }
-        acc[h] = a;
+        const float4 a = reinterpret_cast<const float4*>(xs + h * D + sgi * LE)[0];
+        const float4 c = reinterpret_cast<const float4*>(xs + h * D + sgi * LE)[1];
+        xq[h][0] = a.x; xq[h][1] = a.y; xq[h][2] = a.z; xq[h][3] = a.w;
+        xq[h][4] = c.x; xq[h][5] = c.y; xq[h][6] = c.z; xq[h][7] = c.w;
       }
+      for (int rb = warp * (32 / LT); rb < nr; rb += kFThreads / LT) {  // warp-uniform trip count
+        const int r = rb + lane / LT;
+        const bool valid = r < nr;
+        float kv[LE];
 #pragma unroll
-      for (int o = 1; o < SEGT; o <<= 1)
+        for (int j = 0; j < LE; ++j) kv[j] = 0.f;
+        if (valid) {
 #pragma unroll
-        for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-      if (valid && sgi == 0) {
-        const bool use = !covered || candf[r];
+          for (int v = 0; v < LE / EPV; ++v) {
+            float t8[EPV];
+            Vec16<T>::load(Kr + (size_t)r * D + sgi * LE + v * EPV, t8);
 #pragma unroll
-        for (int h = 0; h < G; ++h) lg[h * GB + r] = use ? acc[h] * p.scale_log2 : -INFINITY;
+            for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
+          }
+        }
+        float acc[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float a = xq[h][0] * kv[0];
+#pragma unroll
+          for (int j = 1; j < LE; ++j) a = fmaf(xq[h][j], kv[j], a);
+          acc[h] = a;
+        }
+#pragma unroll
+        for (int o = 1; o < LT; o <<= 1)
+#pragma unroll
+          for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+        if (valid && sgi == 0) {
+          const bool use = !covered || candf[r];
+#pragma unroll
+          for (int h = 0; h < G; ++h) lg[h * GB + r] = use ? acc[h] * p.scale_log2 : -INFINITY;
+        }
       }
     }
     __syncthreads();
@@ -707,7 +697,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       for (int r = lane; r < nr; r += 32) mx = fmaxf(mx, lg[h * GB + r]);
 #pragma unroll
       for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = part[h * (D + 2)];
+      const float m_old = part[h * 4];
       const float m_new = fmaxf(m_old, mx);
       float ssum = 0.f;
       for (int r = lane; r < nr; r += 32) {
@@ -721,25 +711,56 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       __syncwarp();
       if (lane == 0) {
         const float alpha = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
-        part[h * (D + 2)] = m_new;
-        part[h * (D + 2) + 1] = part[h * (D + 2) + 1] * alpha + ssum;
-        part[h * (D + 2) + 2] = alpha;
+        part[h * 4] = m_new;
+        part[h * 4 + 1] = part[h * 4 + 1] * alpha + ssum;
+        part[h * 4 + 2] = alpha;
       }
     }
     __syncthreads();
+    // P.V: thread (column pair cp, row group rg) sums rows rg, rg + PVG, ... for every head,
+    // then the PVG partial sums of each output go through shared memory (the K rows'
+    // buffer, free once the logits are done)
+    {
+      const int cp = tid % (D / 2), rg = tid / (D / 2);
+      float pacc[G][2];
 #pragma unroll
-    for (int q = 0; q < OPT; ++q) {
-      const int e = tid + q * kFThreads;
-      if (e < G * D) {
-        const int h = e / D, i = e % D;
-        float o = oacc[q] * part[h * (D + 2) + 2];
-#pragma unroll 8
-        for (int r = 0; r < nr; ++r) o = fmaf(lg[h * GB + r], to_f32(Vr[(size_t)r * D + i]), o);
-        oacc[q] = o;
+      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = 0.f;
+      for (int r = rg; r < nr; r += PVG) {
+        float v0, v1;
+        if constexpr (ESZ == 2) {
+          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * D)[cp]);
+          v0 = f.x;
+          v1 = f.y;
+        } else {
+          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * D)[cp];
+          v0 = f.x;
+          v1 = f.y;
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pr_ = lg[h * GB + r];
+          pacc[h][0] = fmaf(pr_, v0, pacc[h][0]);
+          pacc[h][1] = fmaf(pr_, v1, pacc[h][1]);
+        }
+      }
+      float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < OPT; ++q) {
+        const int e = tid + q * kFThreads;
+        if (e < G * D) {
+          const int h = e / D, i = e % D;
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
+          oacc[q] = fmaf(oacc[q], part[h * 4 + 2], sum);
+        }
       }
     }
   }
-  ptx::cp_async_wait_all();
   __syncthreads();
 
   // ---- 9. partials to the CTAs owning each output column, then merge ----------
@@ -755,7 +776,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   for (int e = tid; e < 2 * G * CS; e += kFThreads) {
     const int owner = e / (2 * G), w = e % (2 * G);
-    ptx::st_dsmem_f32(ptx::dsmem_addr(&mslot[rank * stride + w], owner), part[(w >> 1) * (D + 2) + (w & 1)]);
+    ptx::st_dsmem_f32(ptx::dsmem_addr(&mslot[rank * stride + w], owner), part[(w >> 1) * 4 + (w & 1)]);
   }
   ptx::cluster_sync();  // #4: every CTA holds the partials of its columns
   for (int col = tid; col < mc; col += kFThreads) {
@@ -794,18 +815,6 @@ struct Plan {
   int CS, tok_cap, sel_cap, nbins, wcols, stages;
   size_t smem;
 };
-
-int num_sms() {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
-  }
-  return cached[dev];
-}
 
 // Clusters of CS CTAs that can be resident at once (one CTA per SM), cached per
 // (kernel, device, CS, shared memory).
