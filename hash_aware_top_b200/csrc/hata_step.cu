@@ -4,19 +4,19 @@
 //
 // A unit's L cached tokens are split evenly over the CS CTAs of its cluster.
 // Each CTA:
-//   1. streams its slice of the code cache into a 4-8 stage shared-memory ring
+//   1. streams its slice of the code cache into a 2-6 stage shared-memory ring
 //      with bulk (TMA) copies, evict-first in L2, issued as soon as L is known;
-//   2. encodes the G queries and the new key for its slice of the W_H columns
-//      (warp_dot128: the same arithmetic as hata_encode_append's decode form),
-//      stores its code bits into a per-source slot of every CTA of the cluster;
-//      after a cluster barrier each CTA ORs the slots locally, and the CTA
-//      owning slot L - 1 appends the key code to the cache;
+//   2. encodes the G queries and the new key over all r columns of W_H itself
+//      (the arithmetic of warp_dot128, so the codes equal hata_encode_append's
+//      decode form bit for bit; no exchange between CTAs); the CTA owning slot
+//      L - 1 appends the key code to the cache;
 //   3. scores every token of its slice (xor + popc with the GQA sum folded into
 //      per-word constants and a carry-save popc sum), keeping the u16 scores and
 //      their histogram in shared memory; warps release ring stages on their own;
 //   4. turns the histogram into a cumulative one and stores it (u16) into its
-//      slot of every CTA; guesses its own share of the selection from it and
-//      starts gathering those candidate K/V rows (cp.async) right away;
+//      slot of every CTA; takes as candidates every token scoring at most Tc
+//      (the largest score whose count fits about 1.5x its fair share of the
+//      selection) and starts gathering those K/V rows (cp.async) right away;
 //   5. after a cluster barrier, every CTA sums the CS cumulative histograms
 //      (one bin per thread) to find the unit's threshold T (the smallest score
 //      with at least n = min(k, L) tokens at or below it), the tie quota m and
@@ -24,13 +24,13 @@
 //      as in a global sort;
 //   6. computes the flash-decode partial (max, sum, weighted V) of each of the G
 //      query heads over its selected rows (falling back to a second gather when
-//      the guess missed), and stores each partial's column slice into the CTA
-//      that owns those output columns; after a last cluster barrier every CTA
-//      merges its columns (log-sum-exp) and writes them.
+//      T > Tc), and stores each partial's column slice into the CTA that owns
+//      those output columns; after a last cluster barrier every CTA merges its
+//      columns (log-sum-exp) and writes them.
 // Cross-CTA traffic is only stores into other CTAs' shared memory before a
 // hardware cluster barrier: no remote loads, no global-memory flags, no
 // workspace.  The only waits are bounded mbarrier waits on this CTA's own
-// bulk copies.
+// bulk copies and cp.async completion.
 #include <algorithm>
 #include <climits>
 #include <map>
@@ -46,13 +46,14 @@ namespace {
 
 constexpr int kFThreads = 512;
 constexpr int kNWarp = kFThreads / 32;
+static_assert(256 < kFThreads, "candidate passes give each candidate its own thread");
 constexpr int kMaxStages = 6;        // ring stages (32 KB each), 2..6 depending on shared memory left
 constexpr int kMinStages = 2;
 constexpr int kStageBytes = 32768;
 constexpr int kTokCap = 65520;       // max tokens per CTA: u16 scores and u16 cumulative counts
-constexpr int kWCols = 32;           // W_H columns staged per encode batch
+constexpr int kXS = 36;              // floats per residue row of an encoded vector (32 used, padded)
 constexpr int kMaxCS = 16;           // largest cluster
-constexpr int kMaxGB = 256;          // largest gather batch (rows)
+constexpr int kMaxGB = 256;          // largest gather batch (rows); below kFThreads: one candidate per thread
 constexpr int kOneCtaSmem = 116 * 1024;  // dynamic shared memory that keeps one CTA per SM
 constexpr uint32_t kWaitTries = 1u << 22;
 
@@ -67,12 +68,12 @@ struct FusedParams {
   uint32_t* qcode_out;
   int32_t* idx_out;
   uint32_t* status;
-  int Hq, Hkv, max_seq, k, nbins, tok_cap, sel_cap, wcols, flags, stages;
+  int Hq, Hkv, max_seq, k, nbins, tok_cap, sel_cap, flags, stages;
   float scale_log2;
 };
 
 struct SmemLayout {
-  uint32_t ring, D, hist, hslot, xs, wsl, enc, qslot, sel, lg, part, mslot, stat, mbar, total;
+  uint32_t ring, D, hist, hslot, xr, sel, lg, part, mslot, stat, mbar, total;
   int nbp, mcols, gb;
 };
 
@@ -86,15 +87,11 @@ struct Bump {
   }
 };
 
-// W_H columns encoded by each CTA of a cluster of CS: ceil(r / CS) rounded up to
-// a multiple of 4 (the last ranks may get fewer, or none).
-__host__ __device__ inline int enc_cols_per_cta(int R, int CS) { return ((R + CS - 1) / CS + 3) / 4 * 4; }
-
 // Output columns merged by each CTA of a cluster of CS (the last one may have fewer).
 __host__ __device__ inline int merge_cols(int G, int CS) { return (G * kHeadDim + CS - 1) / CS; }
 
 __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int tok_cap, int sel_cap, int nbins,
-                                                  int wcols, int CS, int stages) {
+                                                  int CS, int stages) {
   SmemLayout s;
   Bump b;
   s.nbp = (nbins + 7) / 8 * 8;  // histogram bins padded to whole 16-byte groups of u16
@@ -102,22 +99,26 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int 
   s.gb = stages * kStageBytes / (2 * kHeadDim * esize);
   if (s.gb > kMaxGB) s.gb = kMaxGB;
   s.ring = b.take(stages * kStageBytes, 128);
-  s.D = b.take(tok_cap * 2, 16);
+  s.D = b.take(max(tok_cap * 2, (G + 1) * 4 * NW * 32 * 4), 16);  // scores; first the encode's residue sums
   s.hist = b.take(s.nbp * 4, 16);                     // local counts, then cumulative, then unit totals
   s.hslot = b.take(CS * s.nbp * 2, 16);               // u16 cumulative histograms from every CTA
-  s.xs = b.take((G + 1) * kHeadDim * 4, 16);          // G queries + new key, fp32
-  s.wsl = b.take(wcols * kHeadDim * 4, 16);           // W_H column slice, transposed
-  s.enc = b.take((G + 1) * NW * 4, 16);               // this CTA's code bits
-  s.qslot = b.take(CS * (G + 1) * NW * 4, 16);        // code bits from every CTA
+  s.xr = b.take((G + 1) * 4 * kXS * 4, 16);           // G queries + new key, fp32, residue-major
   s.sel = b.take(sel_cap * 4, 16);                    // selected rows (fallback path)
   s.lg = b.take(G * s.gb * 4, 16);                    // logits / probabilities
   s.part = b.take(G * 4 * 4, 16);                     // running (max, sum, alpha) per head
   s.mslot = b.take(CS * (s.mcols + 2 * G) * 4, 16);   // partials for this CTA's output columns
   s.stat = b.take(16 * 4, 16);
-  s.mbar = b.take((kMaxStages + 1) * 8, 8);  // ring stages + the row-gather barrier
+  s.mbar = b.take(kMaxStages * 8, 8);  // ring stages
   s.total = b.take(0, 128);
   return s;
 }
+
+// Order-preserving map of a float (not NaN) to an int, for integer atomicMax.
+__device__ __forceinline__ int ord_of(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float float_of_ord(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
 enum { ST_T = 0, ST_M, ST_LESS_BEFORE, ST_EQ_BEFORE, ST_SPEC, ST_ABORT, ST_MYLESS, ST_MYEQ, ST_NBELOW };
 
@@ -167,31 +168,31 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int D = kHeadDim;
   constexpr int ESZ = (int)sizeof(T);
+  constexpr int R = NW * 32;                      // hash bits
   constexpr int ST = kStageBytes / (4 * NW);      // tokens per ring stage
   constexpr int NV = G + 1;                       // encoded vectors: G queries + new key
   constexpr int BULK_Q = NW >= 4 ? 1 : 4 / NW;    // tokens per 16 bytes
   constexpr int XV = NV * D * ESZ / 16;           // 16-byte vectors of q + new key
   constexpr int QV = G * D * ESZ / 16;            // ... of which the queries
   constexpr int EPV = 16 / ESZ;                   // elements per 16-byte vector
+  constexpr int RPR = D * ESZ / 16;               // 16-byte pieces per K or V row
   constexpr int LT = 16;                          // threads per row in the logits
   constexpr int LE = D / LT;                      // elements per thread in the logits (8)
   constexpr int PVG = kFThreads / (D / 2);        // row groups in P.V (8): thread = (column pair, row group)
   static_assert(XV <= kFThreads, "one vector of q / new key per thread");
+  static_assert((4 * R) % 32 == 0, "encode items fill whole warps");
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int CS = (int)ptx::cluster_nctarank();
   const int rank = (int)ptx::cluster_ctarank();
   const int kStages = p.stages;
-  const SmemLayout S = smem_layout(G, NW, ESZ, p.tok_cap, p.sel_cap, p.nbins, p.wcols, CS, kStages);
+  const SmemLayout S = smem_layout(G, NW, ESZ, p.tok_cap, p.sel_cap, p.nbins, CS, kStages);
   const int GB = S.gb, nbp = S.nbp;
   unsigned char* ring = smem + S.ring;
   uint16_t* Ds = reinterpret_cast<uint16_t*>(smem + S.D);
   int* hist = reinterpret_cast<int*>(smem + S.hist);
   uint16_t* hslot = reinterpret_cast<uint16_t*>(smem + S.hslot);
-  float* xs = reinterpret_cast<float*>(smem + S.xs);
-  float* wsl = reinterpret_cast<float*>(smem + S.wsl);
-  uint32_t* enc = reinterpret_cast<uint32_t*>(smem + S.enc);
-  uint32_t* qslot = reinterpret_cast<uint32_t*>(smem + S.qslot);
+  float* xr = reinterpret_cast<float*>(smem + S.xr);
   int* sel = reinterpret_cast<int*>(smem + S.sel);
   float* lg = reinterpret_cast<float*>(smem + S.lg);
   float* part = reinterpret_cast<float*>(smem + S.part);
@@ -200,9 +201,13 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + S.mbar);
   __shared__ int warp_sums[kNWarp];
   __shared__ int done[kMaxStages];
-  __shared__ int cand[kMaxGB];
-  __shared__ uint8_t candf[kMaxGB];
-  __shared__ uint32_t qc[NV * NW];
+  __shared__ int lastv[kMaxStages];       // last virtual stage issued into each ring buffer
+  __shared__ __align__(16) int cand[kMaxGB];  // candidate token indices
+  __shared__ uint16_t rowl[kMaxGB];       // gathered rows that are selected (any order)
+  __shared__ __align__(16) uint32_t qc[NV * NW];
+  __shared__ int bmaxi[G];                // per-head logit maximum of a row batch (order-preserving int)
+  __shared__ float redl[PVG * G];         // per-row-group probability sums
+  __shared__ int s_ncand, s_nrow;
 
   const int u = blockIdx.x / CS;
   const int b = u / p.Hkv, g = u % p.Hkv;
@@ -212,53 +217,70 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   if (!early) ptx::pdl_wait();
   ptx::pdl_launch_dependents();
 
-  // ---- 1. first wave of loads: W_H slice, seq_lens; then the codes stream -----
-  const int R = NW * 32;
-  const int cpr = enc_cols_per_cta(R, CS);  // a multiple of 4: 16-byte aligned W_H slices
-  const int j0 = rank * cpr;
-  const int ncols = max(0, min(cpr, R - j0));  // the last ranks may get fewer (or no) columns
-  const uint64_t pol_keep = ptx::policy_evict_last();
-  const float* Wg = p.W + (size_t)g * D * R + j0;
-  const int nc0 = min(p.wcols, ncols);  // a multiple of 4
-  float4 wv[2];
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int e = tid + q * kFThreads;
-    wv[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (e < D * nc0 / 4) wv[q] = ptx::ld_f4_policy(Wg + (size_t)(e / (nc0 / 4)) * R + (e % (nc0 / 4)) * 4, pol_keep);
-  }
-  // query vectors do not depend on L: load them now unless they may still be being written
+  // ---- 1. loads: seq_lens and q; W_H (bulk copy) into the first WS ring buffers;
+  //         then the codes stream into the others ------------------------------
+  // The ring's virtual stages are: 0..WS-1 the W_H matrix of this KV head (row-major
+  // fp32, contiguous across buffers), then WS + s for stage s of the codes stream.
+  // Virtual stage vs lives in buffer vs % kStages and completes phase (vs / kStages) & 1
+  // of that buffer's mbarrier.
+  constexpr int WBYTES = D * R * 4;
+  constexpr int WS = (WBYTES + kStageBytes - 1) / kStageBytes;
+  const int Lraw = p.seq_lens ? p.seq_lens[b] : p.max_seq;
   const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
   uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+  // query vectors do not depend on L: load them now unless they may still be being written
   if (!early && tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
-  const int L = clamp_len(p.seq_lens, b, p.max_seq, p.status);
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) ptx::mbar_init(&mbar[s], 1);
+    ptx::fence_mbarrier_init();
+  }
+  if (tid < kStages) {
+    done[tid] = 0;
+    lastv[tid] = tid < WS ? tid : -1;
+  }
+  if (tid == 0) {
+    stat[ST_ABORT] = 0;
+    s_ncand = 0;
+    s_nrow = 0;
+  }
+  for (int v = tid; v < nbp; v += kFThreads) hist[v] = 0;
+  __syncthreads();
+  if (tid == 0) {
+    const char* Wsrc = reinterpret_cast<const char*>(p.W + (size_t)g * D * R);
+    const uint64_t pol_keep = ptx::policy_evict_last();  // every CTA of the cluster reads it
+    for (int w = 0; w < WS; ++w) {
+      const uint32_t bytes = (uint32_t)min(kStageBytes, WBYTES - w * kStageBytes);
+      ptx::mbar_arrive_expect_tx(&mbar[w], bytes);
+      ptx::bulk_g2s(ring + w * kStageBytes, Wsrc + (size_t)w * kStageBytes, bytes, &mbar[w], pol_keep);
+    }
+  }
+  int L = Lraw;
+  if (L > p.max_seq) {
+    set_status(p.status, HATA_ERR_INVALID_ARG);
+    L = p.max_seq;
+  }
+  L = max(L, 0);
   int C = (L + CS - 1) / CS;
   C = (C + 15) & ~15;
   const int t0 = min(L, rank * C), t1 = min(L, t0 + C);
   const int nmine = t1 - t0;
   const int nst = (nmine + ST - 1) / ST;
   uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) ptx::mbar_init(&mbar[s], 1);
-    ptx::mbar_init(&mbar[kMaxStages], 1);
-    ptx::fence_mbarrier_init();
-  }
-  if (tid < kStages) done[tid] = 0;
-  if (tid == 0) stat[ST_ABORT] = 0;
-  __syncthreads();
   const uint64_t pol_stream = ptx::policy_evict_first();
   auto issue = [&](int s) {
+    const int vs = s + WS;
     const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
     const int nb = nt / BULK_Q * BULK_Q;  // tokens moved by the bulk copy (16-byte multiple)
     const uint32_t bytes = (uint32_t)nb * NW * 4;
-    uint64_t* bar = &mbar[s % kStages];
+    uint64_t* bar = &mbar[vs % kStages];
+    lastv[vs % kStages] = vs;
     ptx::mbar_arrive_expect_tx(bar, bytes);
-    if (bytes) ptx::bulk_g2s(ring + (s % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
+    if (bytes) ptx::bulk_g2s(ring + (vs % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
   };
   if (tid == 0)
-    for (int s = 0; s < min(nst, kStages); ++s) issue(s);
+    for (int s = 0; s < min(nst, kStages - WS); ++s) issue(s);
 
-  // ---- 2. encode the G queries and the new key, this CTA's column slice --------
+  // ---- 2. every CTA encodes the G queries and the new key (all r columns) -----
   if (early) {
     ptx::pdl_wait();  // q and the new key row come from the preceding kernel
     if (tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
@@ -267,70 +289,69 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     const T* kn = static_cast<const T*>(p.K) + (((size_t)u * p.max_seq) + (L > 0 ? L - 1 : 0)) * D;
     if (tid >= QV && tid < XV && L > 0) xv = reinterpret_cast<const uint4*>(kn)[tid - QV];
   }
-#pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int e = tid + q * kFThreads;
-    if (e < D * nc0 / 4) {
-      const int i = e / (nc0 / 4), c4 = (e % (nc0 / 4)) * 4;
-      wsl[(c4 + 0) * D + i] = wv[q].x;
-      wsl[(c4 + 1) * D + i] = wv[q].y;
-      wsl[(c4 + 2) * D + i] = wv[q].z;
-      wsl[(c4 + 3) * D + i] = wv[q].w;
-    }
-  }
+  // fp32 copies in residue-major order: element i of vector v at xr[(v * 4 + i % 4) * kXS + (i / 32) * 8 + (i / 4) % 8]
   if (tid < XV) {
     float xe[EPV];
     Vec16<T>::convert(xv, xe);
+    const int v = tid * EPV / D;
 #pragma unroll
-    for (int j = 0; j < EPV; ++j) xs[tid * EPV + j] = xe[j];
+    for (int e = 0; e < EPV; ++e) {
+      const int i = (tid * EPV + e) % D;
+      xr[(v * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)] = xe[e];
+    }
   }
-  if (tid < NV * NW) enc[tid] = 0u;
-  for (int v = tid; v < nbp; v += kFThreads) hist[v] = 0;
-  for (int cb = 0; cb < ncols; cb += p.wcols) {
-    const int nc = min(p.wcols, ncols - cb);
-    if (cb > 0) {  // further column batches (small clusters): scalar staging
-      __syncthreads();
-      for (int e = tid; e < D * nc; e += kFThreads) {
-        const int i = e / nc, c = e % nc;
-        wsl[c * D + i] = __ldg(Wg + cb + (size_t)i * R + c);
+  for (int w = 0; w < WS; ++w)
+    if (!ptx::mbar_wait_spin(&mbar[w], 0u, kWaitTries)) {
+      set_status(p.status, HATA_ERR_TIMEOUT);
+      stat[ST_ABORT] = 1;
+    }
+  __syncthreads();
+  // y = x . W_H[:, j] in the order of warp_dot128: lane l of that function is
+  // (residue s = l % 4, a = l / 4); its partial (u = 0 product, then FMAs for +32,
+  // +64, +96) and the butterfly levels 16, 8, 4 stay inside one residue, so a
+  // thread here computes the residue sum S_s for one column, and the levels 2 and 1
+  // give y = (S_0 + S_2) + (S_1 + S_3).  Warp item wi: residue wi % 4, columns
+  // 32 (wi / 4) + lane.
+  {
+    const float* Wsm = reinterpret_cast<const float*>(ring);
+    float* sb = reinterpret_cast<float*>(smem + S.D);  // [NV][4][R] residue sums (the scores' space, unused yet)
+    for (int wi = warp; wi < 4 * NW; wi += kNWarp) {
+      const int s = wi & 3, j = (wi >> 2) * 32 + lane;
+      float wr[32];
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = Wsm[(s + 4 * a + 32 * u4) * R + j];
+#pragma unroll 1
+      for (int v = 0; v < NV; ++v) {
+        const float* xs_ = xr + (v * 4 + s) * kXS;
+        float P[8];
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
+          const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
+          const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int a = 0; a < 8; ++a) P[a] = u4 == 0 ? xx[a] * wr[a] : fmaf(xx[a], wr[u4 * 8 + a], P[a]);
+        }
+        const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
+        sb[(v * 4 + s) * R + j] = (q0 + q2) + (q1 + q3);
       }
     }
     __syncthreads();
-    // each warp takes up to 4 (vector, column) pairs at a time, interleaved
-    for (int d0 = warp * 4; d0 < NV * nc; d0 += kNWarp * 4) {
-      const int nd = min(4, NV * nc - d0);
-      const float* xp[4];
-      const float* wp[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int dj = d0 + min(j, nd - 1);
-        xp[j] = xs + (dj / nc) * D;
-        wp[j] = wsl + (dj % nc) * D;
-      }
-      float y[4];
-      warp_dot128_multi<4>(xp, wp, lane, y);
-      float yl = y[0];
-#pragma unroll
-      for (int j = 1; j < 4; ++j) yl = lane == j ? y[j] : yl;
-      if (lane < nd && yl > 0.f) {  // lane j (< nd) publishes pair j's bit
-        const int dj = d0 + lane, col = j0 + cb + dj % nc;
-        atomicOr(&enc[(dj / nc) * NW + (col >> 5)], 1u << (col & 31));
-      }
+    for (int pi = warp; pi < NV * NW; pi += kNWarp) {
+      const int v = pi / NW, jw = pi % NW, j = jw * 32 + lane;
+      const float* sv = sb + v * 4 * R;
+      const float y = (sv[j] + sv[2 * R + j]) + (sv[R + j] + sv[3 * R + j]);
+      const unsigned bits = __ballot_sync(0xffffffffu, y > 0.f);
+      if (lane == 0) qc[v * NW + jw] = bits;
     }
   }
-  __syncthreads();
-  ptx::cluster_wait();  // every CTA of the cluster has started
-  for (int e = tid; e < NV * NW * CS; e += kFThreads) {  // this CTA's bits into slot `rank` of every CTA
-    const int w = e % (NV * NW), c = e / (NV * NW);
-    ptx::st_dsmem_u32(ptx::dsmem_addr(&qslot[rank * NV * NW + w], c), enc[w]);
+  __syncthreads();  // codes ready; W_H and the residue sums are consumed
+  if (tid == 0 && !stat[ST_ABORT]) {
+    ptx::fence_proxy_async_smem();  // generic reads of the W_H buffers before the copies that overwrite them
+    for (int s = kStages - WS; s < min(nst, kStages); ++s) issue(s);
   }
-  ptx::cluster_sync();  // #1: every CTA holds every CTA's code bits
-  if (tid < NV * NW) {
-    uint32_t acc = 0;
-    for (int c = 0; c < CS; ++c) acc |= qslot[c * NV * NW + tid];
-    qc[tid] = acc;
-  }
-  __syncthreads();
   if (rank == 0 && p.qcode_out && tid < G * NW) p.qcode_out[((size_t)b * p.Hq + (size_t)g * G) * NW + tid] = qc[tid];
   const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
   if (own_last && tid < NW) cu[(size_t)(L - 1) * NW + tid] = qc[G * NW + tid];
@@ -343,18 +364,19 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     for (int w = 0; w < NW; ++w) keyc[w] = qc[G * NW + w];
     // Each thread scores TPS tokens of a stage (all loads first, then the
     // arithmetic, for ILP).  Warps release stages on their own: lane 0 adds to the
-    // stage's counter and checks the returned count one stage later, so no lane
-    // waits on the atomic; the warp that completed a stage refills it.
+    // buffer's counter and checks the returned count one stage later, so no lane
+    // waits on the atomic; the warp that completed a stage refills its buffer.
     constexpr int TPS = ST / kFThreads;
     int rel_old = -1, rel_s = -1;  // lane 0: ticket of the previous stage's release
     for (int s = 0; s < nst; ++s) {
-      if (!ptx::mbar_wait_spin(&mbar[s % kStages], (uint32_t)(s / kStages) & 1u, kWaitTries)) {
+      const int vs = s + WS, buf_i = vs % kStages;
+      if (!stat[ST_ABORT] && !ptx::mbar_wait_spin(&mbar[buf_i], (uint32_t)(vs / kStages) & 1u, kWaitTries)) {
         set_status(p.status, HATA_ERR_TIMEOUT);
         stat[ST_ABORT] = 1;
       }
       const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
       const int nb = nt / BULK_Q * BULK_Q;
-      const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + (s % kStages) * kStageBytes);
+      const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + buf_i * kStageBytes);
       uint32_t kw[TPS][NW];
 #pragma unroll
       for (int j = 0; j < TPS; ++j) {
@@ -392,12 +414,16 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       }
       __syncwarp();
       if (lane == 0) {
-        // counters never reset: the k-th use of buffer s % kStages ends at count k * kNWarp
-        if (rel_s >= 0 && rel_old == ((rel_s / kStages) + 1) * kNWarp - 1 && rel_s + kStages < nst) {
-          ptx::fence_proxy_async_smem();
-          issue(rel_s + kStages);
+        // counters never reset: the k-th stream use of a buffer ends at count (k + 1) * kNWarp
+        if (rel_s >= 0) {
+          const int rvs = rel_s + WS;
+          const int k_use = rvs / kStages - (rvs % kStages < WS ? 1 : 0);
+          if (rel_old == (k_use + 1) * kNWarp - 1 && rel_s + kStages < nst) {
+            ptx::fence_proxy_async_smem();
+            issue(rel_s + kStages);
+          }
         }
-        rel_old = atomicAdd(&done[s % kStages], 1);
+        rel_old = atomicAdd(&done[buf_i], 1);
         rel_s = s;
       }
     }
@@ -415,28 +441,104 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   __syncthreads();
 
-  // ---- 4. cumulative histogram -> every CTA; local guess; speculative gather ---
+  // ---- 4. cumulative histogram -> every CTA; candidates; speculative gather ----
   const int n = min(p.k, L);
+  // Candidates: every token of this slice scoring at most Tc, the largest score
+  // whose cumulative count stays within `want` (about 1.5x this CTA's fair share
+  // of the selection), so the candidate rows always fit the gather buffers.
+  const int want = min(nmine, min(GB, 3 * ((n + CS - 1) / CS) / 2 + 16));
   {
     // inclusive cumulative counts in place (each thread a contiguous span of bins)
     const int span = (nbp + kFThreads - 1) / kFThreads;
     const int v0 = min(nbp, tid * span), v1 = min(nbp, v0 + span);
     int local = 0;
     for (int v = v0; v < v1; ++v) local += hist[v];
+    if (tid == 0) stat[ST_SPEC] = p.nbins - 1;  // when no count exceeds `want`
     int total;
     int run = block_exclusive_scan<kFThreads>(local, warp_sums, &total);
-    // guess: enough local rows for about 1.5x this CTA's fair share of the budget
-    const int want = min(nmine, min(GB, 5 * ((n + CS - 1) / CS) / 4 + 8));
-    if (tid == 0) stat[ST_SPEC] = want > 0 ? INT_MAX : -1;
-    __syncthreads();
     for (int v = v0; v < v1; ++v) {
       const int before = run;
       run += hist[v];
       hist[v] = run;
-      if (want > 0 && before < want && run >= want) stat[ST_SPEC] = v;
+      if (before <= want && run > want) stat[ST_SPEC] = v - 1;  // unique: counts never decrease
     }
   }
   __syncthreads();
+  const int Tc = stat[ST_SPEC];
+  // one pass over the scores, 8 at a time with paired 16-bit compares; the few hits
+  // take a slot from a shared counter (order does not matter: ties are ranked by index later)
+  if (Tc >= 0 && !stat[ST_ABORT]) {
+    const uint32_t t2 = (uint32_t)Tc * 0x10001u;
+    const int nvec = (nmine + 7) / 8;  // whole vectors inside tok_cap (a multiple of 16)
+    for (int e = tid; e < nvec; e += kFThreads) {
+      const uint4 w4 = reinterpret_cast<const uint4*>(Ds)[e];
+      uint32_t mk[4] = {__vcmpleu2(w4.x, t2), __vcmpleu2(w4.y, t2), __vcmpleu2(w4.z, t2), __vcmpleu2(w4.w, t2)};
+      const int valid = nmine - e * 8;
+      if (valid < 8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (2 * q >= valid) mk[q] &= 0xffff0000u;
+          if (2 * q + 1 >= valid) mk[q] &= 0x0000ffffu;
+        }
+      }
+      const int c = (__popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3])) >> 4;
+      if (c) {
+        int pos = atomicAdd(&s_ncand, c);
+#pragma unroll
+        for (int h = 0; h < 8; ++h)
+          if ((mk[h >> 1] >> ((h & 1) * 16)) & 1u) {
+            if (pos < GB) cand[pos] = t0 + e * 8 + h;
+            ++pos;
+          }
+      }
+    }
+  }
+  __syncthreads();
+  const int ncand = min(s_ncand, GB);  // <= want <= GB by construction
+  // ascending token order (the counter hands out slots in no fixed order): every
+  // later sum then runs over the rows in one order, so results repeat bit for bit
+  {
+    int t = 0, rk = 0;
+    if (tid < ncand) {
+      t = cand[tid];
+      const int4* c4 = reinterpret_cast<const int4*>(cand);
+      int r2 = 0;
+      for (; r2 + 4 <= ncand; r2 += 4) {
+        const int4 x = c4[r2 >> 2];
+        rk += (x.x < t) + (x.y < t) + (x.z < t) + (x.w < t);
+      }
+      for (; r2 < ncand; ++r2) rk += cand[r2] < t;
+    }
+    __syncthreads();
+    if (tid < ncand) cand[rk] = t;
+    __syncthreads();
+  }
+
+  const T* Kb = static_cast<const T*>(p.K) + (size_t)u * p.max_seq * D;
+  const T* Vb = static_cast<const T*>(p.V) + (size_t)u * p.max_seq * D;
+  T* Kr = reinterpret_cast<T*>(ring);
+  T* Vr = reinterpret_cast<T*>(ring) + (size_t)GB * D;
+  // Row gathers: 16-byte cp.async pieces, one warp per K + V row pair.  An index
+  // outside this CTA's slice (never expected) is flagged and replaced by row t0.
+  auto gather_issue = [&](const int* list, int nr) {
+    for (int e = tid; e < nr * 2 * RPR; e += kFThreads) {
+      const int r = e / (2 * RPR), w = e % (2 * RPR);
+      int t = list[r];
+      if (t < t0 || t >= t1) {
+        set_status(p.status, HATA_ERR_INVALID_ARG);
+        t = t0;
+      }
+      if (w < RPR) ptx::cp_async16(Kr + (size_t)r * D + w * EPV, Kb + (size_t)t * D + w * EPV);
+      else ptx::cp_async16(Vr + (size_t)r * D + (w - RPR) * EPV, Vb + (size_t)t * D + (w - RPR) * EPV);
+    }
+  };
+  auto gather_wait = [&]() {
+    ptx::cp_async_wait_all();
+    __syncthreads();
+  };
+  gather_issue(cand, ncand);  // speculative: waited for in section 8
+
+  ptx::cluster_wait();  // every CTA of the cluster has started: remote stores are safe
   // u16 cumulative histogram into slot `rank` of every CTA (8 bins per 16-byte store)
   for (int e = tid; e < (nbp / 8) * CS; e += kFThreads) {
     const int v8 = e % (nbp / 8), c = e / (nbp / 8);
@@ -448,81 +550,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     pk.w = (uint32_t)h[6] | ((uint32_t)h[7] << 16);
     ptx::st_dsmem_v4(ptx::dsmem_addr(&hslot[rank * nbp + v8 * 8], c), pk);
   }
-  const int Tspec = stat[ST_SPEC];
-
-  const T* Kb = static_cast<const T*>(p.K) + (size_t)u * p.max_seq * D;
-  const T* Vb = static_cast<const T*>(p.V) + (size_t)u * p.max_seq * D;
-  T* Kr = reinterpret_cast<T*>(ring);
-  T* Vr = reinterpret_cast<T*>(ring) + (size_t)GB * D;
-  // Row gathers: one bulk copy per K row and per V row, all completing on the
-  // gather mbarrier (one phase per gather).  An index outside this CTA's slice
-  // (never expected) is flagged and replaced by row t0, so the byte count holds.
-  uint64_t* gbar = &mbar[kMaxStages];
-  uint32_t gphase = 0;
-  const uint64_t pol_rows = ptx::policy_evict_first();
-  auto gather = [&](const int* list, int nr) {
-    if (tid == 0) ptx::mbar_arrive_expect_tx(gbar, (uint32_t)(2 * nr * D * ESZ));
-    for (int e = tid; e < 2 * nr; e += kFThreads) {
-      const int r = e >> 1;
-      int t = list[r];
-      if (t < t0 || t >= t1) {
-        set_status(p.status, HATA_ERR_INVALID_ARG);
-        t = t0;
-      }
-      if (e & 1) ptx::bulk_g2s(Vr + (size_t)r * D, Vb + (size_t)t * D, D * ESZ, gbar, pol_rows);
-      else ptx::bulk_g2s(Kr + (size_t)r * D, Kb + (size_t)t * D, D * ESZ, gbar, pol_rows);
-    }
-  };
-  auto gather_wait = [&]() {
-    if (!ptx::mbar_wait_spin(gbar, gphase & 1u, kWaitTries)) {
-      set_status(p.status, HATA_ERR_TIMEOUT);
-      stat[ST_ABORT] = 1;
-    }
-    ++gphase;
-  };
-  // Passes over this CTA's scores go 8192 at a time: each thread owns 16
-  // consecutive scores of the pass (two 16-byte loads); scores past nmine read as 0xffff.
-  constexpr int TPT = 16, CHUNK = kFThreads * TPT;
-  auto load16 = [&](int base, uint16_t (&dv)[TPT]) {
-    const int a = base + tid * TPT;  // a multiple of 16; a < nmine <= tok_cap keeps both loads in the array
-    uint4 v0 = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu), v1 = v0;
-    if (a < nmine) {
-      v0 = reinterpret_cast<const uint4*>(Ds + a)[0];
-      v1 = reinterpret_cast<const uint4*>(Ds + a)[1];
-    }
-    const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&v0);
-    const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&v1);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      dv[i] = a + i < nmine ? h0[i] : (uint16_t)0xffffu;
-      dv[8 + i] = a + 8 + i < nmine ? h1[i] : (uint16_t)0xffffu;
-    }
-  };
-  int ncand = 0;
-  for (int base = 0; base < nmine && Tspec >= 0; base += CHUNK) {
-    uint16_t dv[TPT];
-    load16(base, dv);
-    int mine = 0;
-#pragma unroll
-    for (int i = 0; i < TPT; ++i) mine += (int)dv[i] <= Tspec;
-    int tot;
-    int pos = ncand + block_exclusive_scan<kFThreads>(mine, warp_sums, &tot);
-#pragma unroll
-    for (int i = 0; i < TPT; ++i)
-      if ((int)dv[i] <= Tspec) {
-        if (pos < GB) cand[pos] = t0 + base + tid * TPT + i;
-        ++pos;
-      }
-    ncand += tot;
-  }
-  const bool truncated = ncand > GB;
-  ncand = min(ncand, GB);
-  if (stat[ST_ABORT]) ncand = 0;  // a bulk copy never completed: the ring may still be written
-  __syncthreads();
-  gather(cand, ncand);  // speculative: waited for in section 8
 
   // ---- 5. unit threshold from the CS cumulative histograms -------------------
-  ptx::cluster_sync();  // #2: every CTA holds every CTA's cumulative histogram
+  ptx::cluster_sync();  // #1: every CTA holds every CTA's cumulative histogram
   {
     // unit totals, one bin per thread; T = number of bins whose cumulative total is below n
     int below = 0;
@@ -544,12 +574,12 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       int Tth = lane < kNWarp ? warp_sums[lane] : 0;
 #pragma unroll
       for (int o = 16; o; o >>= 1) Tth += __shfl_xor_sync(0xffffffffu, Tth, o);
-      const int Tc = min(Tth, p.nbins - 1);
+      const int Tcl = min(Tth, p.nbins - 1);
       // per source CTA (lane c): cumulative count below T and at T
       int cb = 0, ce = 0;
       if (lane < CS) {
-        cb = Tc > 0 ? (int)hslot[lane * nbp + Tc - 1] : 0;
-        ce = (int)hslot[lane * nbp + Tc] - cb;
+        cb = Tcl > 0 ? (int)hslot[lane * nbp + Tcl - 1] : 0;
+        ce = (int)hslot[lane * nbp + Tcl] - cb;
       }
       const int lb = __reduce_add_sync(0xffffffffu, lane < rank ? cb : 0);
       const int eb = __reduce_add_sync(0xffffffffu, lane < rank ? ce : 0);
@@ -557,7 +587,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       const int mye = __shfl_sync(0xffffffffu, ce, rank);
       if (lane == 0) {
         stat[ST_T] = n == 0 ? 0 : Tth;
-        stat[ST_M] = n == 0 ? 0 : n - (Tc > 0 ? hist[Tc - 1] : 0);
+        stat[ST_M] = n == 0 ? 0 : n - (Tcl > 0 ? hist[Tcl - 1] : 0);
         stat[ST_LESS_BEFORE] = lb;
         stat[ST_EQ_BEFORE] = eb;
         stat[ST_MYLESS] = myl;
@@ -571,11 +601,29 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int sel_before = less_before + min(eq_before, m);
   const int ties_here = max(0, min(m - eq_before, stat[ST_MYEQ]));
   const int nsel_here = stat[ST_MYLESS] + ties_here;  // this CTA's share of the selection
-  // the candidates cover the selection when every selected score is <= Tspec and none was cut off
-  const bool covered = nsel_here == 0 || (!truncated && Tt <= Tspec);
+  // the candidates hold every selected token of this slice when T <= Tc
+  const bool covered = nsel_here == 0 || Tt <= Tc;
 
   // ---- 7. ascending indices (only when asked for) and the row list --------------
   int32_t* ix = p.idx_out ? p.idx_out + (size_t)u * p.k : nullptr;
+  // Passes over this CTA's scores go 8192 at a time: each thread owns 16
+  // consecutive scores of the pass (two 16-byte loads); scores past nmine read as 0xffff.
+  constexpr int TPT = 16, CHUNK = kFThreads * TPT;
+  auto load16 = [&](int base, uint16_t (&dv)[TPT]) {
+    const int a = base + tid * TPT;  // a multiple of 16; a < nmine <= tok_cap keeps both loads in the array
+    uint4 v0 = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu), v1 = v0;
+    if (a < nmine) {
+      v0 = reinterpret_cast<const uint4*>(Ds + a)[0];
+      v1 = reinterpret_cast<const uint4*>(Ds + a)[1];
+    }
+    const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&v0);
+    const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&v1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      dv[i] = a + i < nmine ? h0[i] : (uint16_t)0xffffu;
+      dv[8 + i] = a + 8 + i < nmine ? h1[i] : (uint16_t)0xffffu;
+    }
+  };
   if (ix || !covered) {
     // one packed scan per pass: low half counts scores < T, high half scores == T
     int lp_carry = 0, ep_carry = 0;
@@ -611,19 +659,28 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     if (ix && rank == 0)
       for (int j = n + tid; j < p.k; j += kFThreads) ix[j] = -1;
   }
-  // selection flags of the candidates (covered case): every tie of this CTA is a
-  // candidate, in index order, so a tie's rank is eq_before + ties among earlier candidates
-  if (covered && warp == 0) {
-    int run = eq_before;
-    for (int r0 = 0; r0 < ncand; r0 += 32) {
-      const int r = r0 + lane;
-      const int dv = r < ncand ? (int)Ds[cand[r] - t0] : INT_MAX;
-      const bool is_eq = dv == Tt;
-      const unsigned eqm = __ballot_sync(0xffffffffu, is_eq);
-      const int rk = run + __popc(eqm & ((1u << lane) - 1u));
-      if (r < ncand) candf[r] = (uint8_t)(dv < Tt || (is_eq && rk < m));
-      run += __popc(eqm);
+  // selected candidates (covered case), kept in ascending token order: scores below
+  // T, and the first quota = m - (ties of earlier CTAs) ties at T (the candidates
+  // hold every tie of this slice, sorted by index)
+  if (covered && nsel_here > 0) {
+    int dv = INT_MAX;
+    if (tid < ncand) dv = Ds[cand[tid] - t0];  // ncand <= GB < kFThreads
+    const bool lt = dv < Tt, eq = dv == Tt;
+    const unsigned blt = __ballot_sync(0xffffffffu, lt), beq = __ballot_sync(0xffffffffu, eq);
+    __syncthreads();  // warp_sums is free again
+    if (lane == 0) warp_sums[warp] = __popc(blt) | (__popc(beq) << 16);
+    __syncthreads();
+    int pre = 0, tot = 0;
+    for (int w = 0; w < kNWarp; ++w) {
+      const int x = warp_sums[w];
+      pre += w < warp ? x : 0;
+      tot += x;
     }
+    const unsigned lm = (1u << lane) - 1u;
+    const int ltpre = (pre & 0xffff) + __popc(blt & lm), eqpre = (pre >> 16) + __popc(beq & lm);
+    const int quota = max(0, m - eq_before);
+    if (lt || (eq && eqpre < quota)) rowl[ltpre + min(eqpre, quota)] = (uint16_t)tid;
+    if (tid == 0) s_nrow = (tot & 0xffff) + min(tot >> 16, quota);
   }
 
   // ---- 8. attention partials over this CTA's selected rows -----------------------
@@ -634,43 +691,43 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   if (tid < G) {
     part[tid * 4] = -INFINITY;
     part[tid * 4 + 1] = 0.f;
+    bmaxi[tid] = ord_of(-INFINITY);
   }
-  const int nrows_total = covered ? ncand : (stat[ST_ABORT] ? 0 : min(nsel_here, p.sel_cap));
-  gather_wait();  // the speculative rows (they were issued before the threshold was known)
+  gather_wait();  // the speculative rows (issued before the threshold was known); also publishes s_nrow
+  const int nrows_total = stat[ST_ABORT] ? 0 : (covered ? s_nrow : min(nsel_here, p.sel_cap));
   for (int r0 = 0; r0 < nrows_total; r0 += GB) {
     const int nr = min(GB, nrows_total - r0);
     if (!covered) {  // the guess missed: gather the selected rows batch by batch
       __syncthreads();  // previous batch's readers are done with the buffers
-      gather(sel + r0, nr);
+      gather_issue(sel + r0, nr);
       gather_wait();
     }
-    __syncthreads();
     // logits (exp2 domain): 16 threads per row, 8 elements each, every head at once;
     // each thread keeps its 8-element slice of the G query vectors in registers
     {
       const int sgi = lane % LT;
       float xq[G][LE];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float4 a = reinterpret_cast<const float4*>(xs + h * D + sgi * LE)[0];
-        const float4 c = reinterpret_cast<const float4*>(xs + h * D + sgi * LE)[1];
-        xq[h][0] = a.x; xq[h][1] = a.y; xq[h][2] = a.z; xq[h][3] = a.w;
-        xq[h][4] = c.x; xq[h][5] = c.y; xq[h][6] = c.z; xq[h][7] = c.w;
-      }
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int j = 0; j < LE; ++j) {
+          const int i = sgi * LE + j;
+          xq[h][j] = xr[(h * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)];
+        }
+      float mx[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
       for (int rb = warp * (32 / LT); rb < nr; rb += kFThreads / LT) {  // warp-uniform trip count
         const int r = rb + lane / LT;
         const bool valid = r < nr;
+        const int rr = valid ? (covered ? (int)rowl[r] : r) : 0;
         float kv[LE];
 #pragma unroll
-        for (int j = 0; j < LE; ++j) kv[j] = 0.f;
-        if (valid) {
+        for (int v = 0; v < LE / EPV; ++v) {
+          float t8[EPV];
+          Vec16<T>::load(Kr + (size_t)rr * D + sgi * LE + v * EPV, t8);
 #pragma unroll
-          for (int v = 0; v < LE / EPV; ++v) {
-            float t8[EPV];
-            Vec16<T>::load(Kr + (size_t)r * D + sgi * LE + v * EPV, t8);
-#pragma unroll
-            for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
-          }
+          for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
         }
         float acc[G];
 #pragma unroll
@@ -685,54 +742,45 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
 #pragma unroll
           for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
         if (valid && sgi == 0) {
-          const bool use = !covered || candf[r];
 #pragma unroll
-          for (int h = 0; h < G; ++h) lg[h * GB + r] = use ? acc[h] * p.scale_log2 : -INFINITY;
+          for (int h = 0; h < G; ++h) {
+            const float lv = acc[h] * p.scale_log2;
+            lg[h * GB + r] = lv;
+            mx[h] = fmaxf(mx[h], lv);
+          }
         }
       }
-    }
-    __syncthreads();
-    for (int h = warp; h < G; h += kNWarp) {
-      float mx = -INFINITY;
-      for (int r = lane; r < nr; r += 32) mx = fmaxf(mx, lg[h * GB + r]);
 #pragma unroll
-      for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = part[h * 4];
-      const float m_new = fmaxf(m_old, mx);
-      float ssum = 0.f;
-      for (int r = lane; r < nr; r += 32) {
-        const float lv = lg[h * GB + r];
-        const float pr_ = lv == -INFINITY ? 0.f : exp2f(lv - m_new);
-        lg[h * GB + r] = pr_;
-        ssum += pr_;
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-      __syncwarp();
-      if (lane == 0) {
-        const float alpha = (m_old == -INFINITY) ? 0.f : exp2f(m_old - m_new);
-        part[h * 4] = m_new;
-        part[h * 4 + 1] = part[h * 4 + 1] * alpha + ssum;
-        part[h * 4 + 2] = alpha;
+      for (int h = 0; h < G; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], LT));
+        if (lane == 0 && mx[h] != -INFINITY) atomicMax(&bmaxi[h], ord_of(mx[h]));
       }
     }
     __syncthreads();
-    // P.V: thread (column pair cp, row group rg) sums rows rg, rg + PVG, ... for every head,
-    // then the PVG partial sums of each output go through shared memory (the K rows'
-    // buffer, free once the logits are done)
+    // probabilities against the running maximum, every thread a few
+    for (int e = tid; e < G * nr; e += kFThreads) {
+      const int h = e / nr, r = e - h * nr;
+      const float mn = fmaxf(part[h * 4], float_of_ord(bmaxi[h]));
+      lg[h * GB + r] = exp2f(lg[h * GB + r] - mn);
+    }
+    __syncthreads();
+    // P.V: thread (column pair cp, row group rg) sums rows rg, rg + PVG, ... for every head
+    // (column pair 0 also sums the probabilities), then the PVG partial sums of each
+    // output go through shared memory (the K rows' buffer, free once the logits are done)
     {
       const int cp = tid % (D / 2), rg = tid / (D / 2);
-      float pacc[G][2];
+      float pacc[G][2], lsum[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = 0.f;
+      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
       for (int r = rg; r < nr; r += PVG) {
+        const int rr = covered ? (int)rowl[r] : r;
         float v0, v1;
         if constexpr (ESZ == 2) {
-          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * D)[cp]);
+          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)rr * D)[cp]);
           v0 = f.x;
           v1 = f.y;
         } else {
-          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * D)[cp];
+          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)rr * D)[cp];
           v0 = f.x;
           v1 = f.y;
         }
@@ -741,23 +789,43 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
           const float pr_ = lg[h * GB + r];
           pacc[h][0] = fmaf(pr_, v0, pacc[h][0]);
           pacc[h][1] = fmaf(pr_, v1, pacc[h][1]);
+          lsum[h] += pr_;
         }
       }
       float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
 #pragma unroll
       for (int h = 0; h < G; ++h)
         reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
+      if (cp == 0)
+#pragma unroll
+        for (int h = 0; h < G; ++h) redl[rg * G + h] = lsum[h];
       __syncthreads();
 #pragma unroll
       for (int q = 0; q < OPT; ++q) {
         const int e = tid + q * kFThreads;
         if (e < G * D) {
           const int h = e / D, i = e % D;
+          const float m_old = part[h * 4];
+          const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
+          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
           float sum = 0.f;
 #pragma unroll
           for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
-          oacc[q] = fmaf(oacc[q], part[h * 4 + 2], sum);
+          oacc[q] = fmaf(oacc[q], alpha, sum);
         }
+      }
+      __syncthreads();  // every thread has read the running maxima of this batch
+      if (tid < G) {
+        const int h = tid;
+        const float m_old = part[h * 4];
+        const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
+        const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+        float ls = 0.f;
+#pragma unroll
+        for (int j = 0; j < PVG; ++j) ls += redl[j * G + h];
+        part[h * 4 + 1] = part[h * 4 + 1] * alpha + ls;
+        part[h * 4] = mn;
+        bmaxi[h] = ord_of(-INFINITY);
       }
     }
   }
@@ -799,10 +867,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   if (stat[ST_ABORT] && tid == 0) {
     // give outstanding bulk copies one more bounded chance to land before exit
-    for (int s = 0; s < min(nst, kStages); ++s) {
-      const int last = nst - 1 - ((nst - 1 - s) % kStages);
-      ptx::mbar_wait_bounded(&mbar[s], (uint32_t)(last / kStages) & 1u, kWaitTries);
-    }
+    for (int bi = 0; bi < kStages; ++bi)
+      if (lastv[bi] >= 0) ptx::mbar_wait_bounded(&mbar[bi], (uint32_t)(lastv[bi] / kStages) & 1u, kWaitTries);
   }
 }
 
@@ -812,7 +878,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
 
 struct Plan {
   bool ok;
-  int CS, tok_cap, sel_cap, nbins, wcols, stages;
+  int CS, tok_cap, sel_cap, nbins, stages;
   size_t smem;
 };
 
@@ -891,11 +957,17 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
     pl.tok_cap = tok_cap;
     pl.sel_cap = std::min(k, tok_cap);
     pl.nbins = G * d.hash_bits + 1;
-    pl.wcols = std::min(kWCols, enc_cols_per_cta(R, CS));
     pl.stages = 0;
-    for (int st = kMaxStages; st >= kMinStages; --st) {
-      const size_t sm = smem_layout(G, NW, esize, tok_cap, pl.sel_cap, pl.nbins, pl.wcols, CS, st).total;
-      if (sm + 2048 <= 227 * 1024) {  // + static shared memory
+    // W_H occupies the first ceil(d r 4 / stage) ring buffers until the encode is done
+    const int w_stages = (kHeadDim * R * 4 + kStageBytes - 1) / kStageBytes;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return best;
+    }
+    for (int st = kMaxStages; st >= std::max(kMinStages, w_stages + 1); --st) {
+      const size_t sm = smem_layout(G, NW, esize, tok_cap, pl.sel_cap, pl.nbins, CS, st).total;
+      if (sm + fa.sharedSizeBytes <= 227 * 1024) {  // + static shared memory
         pl.stages = st;
         pl.smem = std::max<size_t>(sm, kOneCtaSmem);
         break;
@@ -1044,7 +1116,6 @@ cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const voi
   prm.nbins = pl.nbins;
   prm.tok_cap = pl.tok_cap;
   prm.sel_cap = pl.sel_cap;
-  prm.wcols = pl.wcols;
   prm.flags = d.flags;
   prm.stages = pl.stages;
   prm.scale_log2 = scale * 1.4426950408889634f;
