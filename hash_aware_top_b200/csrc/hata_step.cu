@@ -51,11 +51,17 @@ constexpr int kMaxStages = 6;        // ring stages (32 KB each), 2..6 depending
 constexpr int kMinStages = 2;
 constexpr int kStageBytes = 32768;
 constexpr int kTokCap = 65520;       // max tokens per CTA: u16 scores and u16 cumulative counts
+constexpr int kWCols = 32;           // W_H columns staged per encode batch
 constexpr int kXS = 36;              // floats per residue row of an encoded vector (32 used, padded)
 constexpr int kMaxCS = 16;           // largest cluster
 constexpr int kMaxGB = 256;          // largest gather batch (rows); below kFThreads: one candidate per thread
 constexpr int kOneCtaSmem = 116 * 1024;  // dynamic shared memory that keeps one CTA per SM
 constexpr uint32_t kWaitTries = 1u << 22;
+
+struct SmemLayout {
+  uint32_t ring, D, hist, hslot, xr, xp, sel, lg, part, mslot, stat, mbar, total;
+  int nbp, mcols, gb;
+};
 
 struct FusedParams {
   const void* q;
@@ -70,11 +76,7 @@ struct FusedParams {
   uint32_t* status;
   int Hq, Hkv, max_seq, k, nbins, tok_cap, sel_cap, flags, stages;
   float scale_log2;
-};
-
-struct SmemLayout {
-  uint32_t ring, D, hist, hslot, xr, sel, lg, part, mslot, stat, mbar, total;
-  int nbp, mcols, gb;
+  SmemLayout lay;  // shared-memory layout of the launch (computed on the host)
 };
 
 struct Bump {
@@ -88,6 +90,10 @@ struct Bump {
 };
 
 // Output columns merged by each CTA of a cluster of CS (the last one may have fewer).
+// W_H columns encoded by each CTA of a cluster of CS: ceil(r / CS) rounded up to
+// whole bytes of the code (the last ranks may get fewer, or none).
+__host__ __device__ inline int enc_cols_per_cta(int R, int CS) { return ((R + CS - 1) / CS + 7) / 8 * 8; }
+
 __host__ __device__ inline int merge_cols(int G, int CS) { return (G * kHeadDim + CS - 1) / CS; }
 
 __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int tok_cap, int sel_cap, int nbins,
@@ -99,16 +105,17 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int 
   s.gb = stages * kStageBytes / (2 * kHeadDim * esize);
   if (s.gb > kMaxGB) s.gb = kMaxGB;
   s.ring = b.take(stages * kStageBytes, 128);
-  s.D = b.take(max(tok_cap * 2, (G + 1) * 4 * NW * 32 * 4), 16);  // scores; first the encode's residue sums
-  s.hist = b.take(s.nbp * 4, 16);                     // local counts, then cumulative, then unit totals
+  s.D = b.take(max(tok_cap * 2, kHeadDim * kWCols * 4 + (G + 1) * 4 * enc_cols_per_cta(NW * 32, CS) * 4), 16);  // scores; first the encode's W_H columns and residue sums
+  s.hist = b.take((s.nbp + kFThreads - 1) / kFThreads * kFThreads * 4, 16);  // counts, then cumulative (padded)
   s.hslot = b.take(CS * s.nbp * 2, 16);               // u16 cumulative histograms from every CTA
   s.xr = b.take((G + 1) * 4 * kXS * 4, 16);           // G queries + new key, fp32, residue-major
+  s.xp = b.take(G * kHeadDim * 4, 16);                // G queries, fp32
   s.sel = b.take(sel_cap * 4, 16);                    // selected rows (fallback path)
   s.lg = b.take(G * s.gb * 4, 16);                    // logits / probabilities
   s.part = b.take(G * 4 * 4, 16);                     // running (max, sum, alpha) per head
   s.mslot = b.take(CS * (s.mcols + 2 * G) * 4, 16);   // partials for this CTA's output columns
   s.stat = b.take(16 * 4, 16);
-  s.mbar = b.take(kMaxStages * 8, 8);  // ring stages
+  s.mbar = b.take((kMaxStages + 1) * 8, 8);  // ring stages + the row gathers
   s.total = b.take(0, 128);
   return s;
 }
@@ -120,7 +127,7 @@ __device__ __forceinline__ int ord_of(float f) {
 }
 __device__ __forceinline__ float float_of_ord(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
-enum { ST_T = 0, ST_M, ST_LESS_BEFORE, ST_EQ_BEFORE, ST_SPEC, ST_ABORT, ST_MYLESS, ST_MYEQ, ST_NBELOW };
+enum { ST_T = 0, ST_M, ST_LESS_BEFORE, ST_EQ_BEFORE, ST_SPEC, ST_ABORT, ST_MYLESS, ST_MYEQ, ST_LO, ST_HI };
 
 template <typename T>
 struct Vec16;  // 16-byte vector of T as fp32
@@ -179,35 +186,39 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   constexpr int LT = 16;                          // threads per row in the logits
   constexpr int LE = D / LT;                      // elements per thread in the logits (8)
   constexpr int PVG = kFThreads / (D / 2);        // row groups in P.V (8): thread = (column pair, row group)
+  constexpr int NBP = (G * R + 1 + 7) / 8 * 8;    // histogram bins padded to whole 8-bin groups
+  constexpr int BPT = (NBP + kFThreads - 1) / kFThreads;  // bins per thread in the cumulative sum
   static_assert(XV <= kFThreads, "one vector of q / new key per thread");
-  static_assert((4 * R) % 32 == 0, "encode items fill whole warps");
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int CS = (int)ptx::cluster_nctarank();
   const int rank = (int)ptx::cluster_ctarank();
   const int kStages = p.stages;
-  const SmemLayout S = smem_layout(G, NW, ESZ, p.tok_cap, p.sel_cap, p.nbins, CS, kStages);
-  const int GB = S.gb, nbp = S.nbp;
+  const SmemLayout& S = p.lay;
+  const int GB = S.gb;
   unsigned char* ring = smem + S.ring;
   uint16_t* Ds = reinterpret_cast<uint16_t*>(smem + S.D);
   int* hist = reinterpret_cast<int*>(smem + S.hist);
   uint16_t* hslot = reinterpret_cast<uint16_t*>(smem + S.hslot);
   float* xr = reinterpret_cast<float*>(smem + S.xr);
+  float* xp = reinterpret_cast<float*>(smem + S.xp);
   int* sel = reinterpret_cast<int*>(smem + S.sel);
   float* lg = reinterpret_cast<float*>(smem + S.lg);
   float* part = reinterpret_cast<float*>(smem + S.part);
   float* mslot = reinterpret_cast<float*>(smem + S.mslot);
   int* stat = reinterpret_cast<int*>(smem + S.stat);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + S.mbar);
+  uint64_t* gbar = &mbar[kMaxStages];  // completion of the row gathers (cp.async)
   __shared__ int warp_sums[kNWarp];
   __shared__ int done[kMaxStages];
-  __shared__ int lastv[kMaxStages];       // last virtual stage issued into each ring buffer
-  __shared__ __align__(16) int cand[kMaxGB];  // candidate token indices
-  __shared__ uint16_t rowl[kMaxGB];       // gathered rows that are selected (any order)
+  __shared__ int lastv[kMaxStages];       // last stage issued into each ring buffer
+  __shared__ __align__(16) int cand[kMaxGB];  // candidate token indices, ascending
+  __shared__ uint16_t rowl[kMaxGB];       // slots of the selected candidates, ascending token index
   __shared__ __align__(16) uint32_t qc[NV * NW];
   __shared__ int bmaxi[G];                // per-head logit maximum of a row batch (order-preserving int)
   __shared__ float redl[PVG * G];         // per-row-group probability sums
-  __shared__ int s_ncand, s_nrow;
+  __shared__ int s_nrow;
+  __shared__ __align__(16) int hdr[kMaxCS * 4];  // per source CTA: range [lo, hi) of the histogram bins it sent
 
   const int u = blockIdx.x / CS;
   const int b = u / p.Hkv, g = u % p.Hkv;
@@ -217,43 +228,41 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   if (!early) ptx::pdl_wait();
   ptx::pdl_launch_dependents();
 
-  // ---- 1. loads: seq_lens and q; W_H (bulk copy) into the first WS ring buffers;
-  //         then the codes stream into the others ------------------------------
-  // The ring's virtual stages are: 0..WS-1 the W_H matrix of this KV head (row-major
-  // fp32, contiguous across buffers), then WS + s for stage s of the codes stream.
-  // Virtual stage vs lives in buffer vs % kStages and completes phase (vs / kStages) & 1
-  // of that buffer's mbarrier.
-  constexpr int WBYTES = D * R * 4;
-  constexpr int WS = (WBYTES + kStageBytes - 1) / kStageBytes;
+  // ---- 1. loads: seq_lens, q, this CTA's W_H columns; then the codes stream ---
   const int Lraw = p.seq_lens ? p.seq_lens[b] : p.max_seq;
   const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
   uint4 xv = make_uint4(0u, 0u, 0u, 0u);
   // query vectors do not depend on L: load them now unless they may still be being written
   if (!early && tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
+  // This CTA encodes columns [j0, j0 + ncols) of W_H (whole bytes of the code), in
+  // batches of up to kWCols columns staged in shared memory (one batch from CS = 4 on).
+  const int cpr = enc_cols_per_cta(R, CS);
+  const int j0 = rank * cpr, ncols = max(0, min(cpr, R - j0));
+  float* wsl = reinterpret_cast<float*>(smem + S.D);       // [D][kWCols] W_H columns (the scores' space, unused yet)
+  float* sb = wsl + D * kWCols;                             // [NV][4][cpr] residue sums
+  const float* Wg = p.W + (size_t)g * D * R;
+  auto issue_w = [&](int cb) {
+    const int nq = min(kWCols, ncols - cb) / 4;  // 16-byte pieces per row
+    for (int e = tid; e < D * nq; e += kFThreads) {
+      const int i = e / nq, q4 = e % nq;
+      ptx::cp_async16(wsl + i * kWCols + q4 * 4, Wg + (size_t)i * R + j0 + cb + q4 * 4);
+    }
+  };
+  if (ncols > 0) issue_w(0);
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) ptx::mbar_init(&mbar[s], 1);
+    for (int s = 0; s <= kMaxStages; ++s) ptx::mbar_init(&mbar[s], s < kMaxStages ? 1u : (uint32_t)kFThreads);
     ptx::fence_mbarrier_init();
   }
-  if (tid < kStages) {
+  if (tid < kMaxStages) {
     done[tid] = 0;
-    lastv[tid] = tid < WS ? tid : -1;
+    lastv[tid] = -1;
   }
   if (tid == 0) {
     stat[ST_ABORT] = 0;
-    s_ncand = 0;
     s_nrow = 0;
   }
-  for (int v = tid; v < nbp; v += kFThreads) hist[v] = 0;
+  for (int v = tid; v < kFThreads * BPT; v += kFThreads) hist[v] = 0;
   __syncthreads();
-  if (tid == 0) {
-    const char* Wsrc = reinterpret_cast<const char*>(p.W + (size_t)g * D * R);
-    const uint64_t pol_keep = ptx::policy_evict_last();  // every CTA of the cluster reads it
-    for (int w = 0; w < WS; ++w) {
-      const uint32_t bytes = (uint32_t)min(kStageBytes, WBYTES - w * kStageBytes);
-      ptx::mbar_arrive_expect_tx(&mbar[w], bytes);
-      ptx::bulk_g2s(ring + w * kStageBytes, Wsrc + (size_t)w * kStageBytes, bytes, &mbar[w], pol_keep);
-    }
-  }
   int L = Lraw;
   if (L > p.max_seq) {
     set_status(p.status, HATA_ERR_INVALID_ARG);
@@ -268,19 +277,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;
   const uint64_t pol_stream = ptx::policy_evict_first();
   auto issue = [&](int s) {
-    const int vs = s + WS;
     const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
     const int nb = nt / BULK_Q * BULK_Q;  // tokens moved by the bulk copy (16-byte multiple)
     const uint32_t bytes = (uint32_t)nb * NW * 4;
-    uint64_t* bar = &mbar[vs % kStages];
-    lastv[vs % kStages] = vs;
+    uint64_t* bar = &mbar[s % kStages];
+    lastv[s % kStages] = s;
     ptx::mbar_arrive_expect_tx(bar, bytes);
-    if (bytes) ptx::bulk_g2s(ring + (vs % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
+    if (bytes) ptx::bulk_g2s(ring + (s % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
   };
   if (tid == 0)
-    for (int s = 0; s < min(nst, kStages - WS); ++s) issue(s);
+    for (int s = 0; s < min(nst, kStages); ++s) issue(s);
 
-  // ---- 2. every CTA encodes the G queries and the new key (all r columns) -----
+  // ---- 2. encode this CTA's W_H columns for the G queries and the new key --------
   if (early) {
     ptx::pdl_wait();  // q and the new key row come from the preceding kernel
     if (tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
@@ -289,7 +297,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     const T* kn = static_cast<const T*>(p.K) + (((size_t)u * p.max_seq) + (L > 0 ? L - 1 : 0)) * D;
     if (tid >= QV && tid < XV && L > 0) xv = reinterpret_cast<const uint4*>(kn)[tid - QV];
   }
-  // fp32 copies in residue-major order: element i of vector v at xr[(v * 4 + i % 4) * kXS + (i / 32) * 8 + (i / 4) % 8]
+  // fp32 copies: residue-major for the encode (element i of vector v at
+  // xr[(v * 4 + i % 4) * kXS + (i / 32) * 8 + (i / 4) % 8]) and plain for the logits
   if (tid < XV) {
     float xe[EPV];
     Vec16<T>::convert(xv, xe);
@@ -298,60 +307,61 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     for (int e = 0; e < EPV; ++e) {
       const int i = (tid * EPV + e) % D;
       xr[(v * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)] = xe[e];
+      if (v < G) xp[v * D + i] = xe[e];
     }
   }
-  for (int w = 0; w < WS; ++w)
-    if (!ptx::mbar_wait_spin(&mbar[w], 0u, kWaitTries)) {
-      set_status(p.status, HATA_ERR_TIMEOUT);
-      stat[ST_ABORT] = 1;
-    }
-  __syncthreads();
   // y = x . W_H[:, j] in the order of warp_dot128: lane l of that function is
   // (residue s = l % 4, a = l / 4); its partial (u = 0 product, then FMAs for +32,
-  // +64, +96) and the butterfly levels 16, 8, 4 stay inside one residue, so a
-  // thread here computes the residue sum S_s for one column, and the levels 2 and 1
-  // give y = (S_0 + S_2) + (S_1 + S_3).  Warp item wi: residue wi % 4, columns
-  // 32 (wi / 4) + lane.
-  {
-    const float* Wsm = reinterpret_cast<const float*>(ring);
-    float* sb = reinterpret_cast<float*>(smem + S.D);  // [NV][4][R] residue sums (the scores' space, unused yet)
-    for (int wi = warp; wi < 4 * NW; wi += kNWarp) {
-      const int s = wi & 3, j = (wi >> 2) * 32 + lane;
-      float wr[32];
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4)
-#pragma unroll
-        for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = Wsm[(s + 4 * a + 32 * u4) * R + j];
-#pragma unroll 1
-      for (int v = 0; v < NV; ++v) {
-        const float* xs_ = xr + (v * 4 + s) * kXS;
-        float P[8];
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
-          const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
-          const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-          for (int a = 0; a < 8; ++a) P[a] = u4 == 0 ? xx[a] * wr[a] : fmaf(xx[a], wr[u4 * 8 + a], P[a]);
-        }
-        const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
-        sb[(v * 4 + s) * R + j] = (q0 + q2) + (q1 + q3);
-      }
+  // +64, +96) and the butterfly levels 16, 8, 4 stay inside one residue, so one
+  // thread here computes the residue sum S_s of one (vector, column), and the
+  // levels 2 and 1 give y = (S_0 + S_2) + (S_1 + S_3).
+  for (int cb = 0; cb < ncols; cb += kWCols) {
+    const int nb = min(kWCols, ncols - cb);
+    if (cb > 0) {
+      __syncthreads();  // the previous batch's readers are done with the staged columns
+      issue_w(cb);
     }
+    ptx::cp_async_wait_all();
     __syncthreads();
-    for (int pi = warp; pi < NV * NW; pi += kNWarp) {
-      const int v = pi / NW, jw = pi % NW, j = jw * 32 + lane;
-      const float* sv = sb + v * 4 * R;
-      const float y = (sv[j] + sv[2 * R + j]) + (sv[R + j] + sv[3 * R + j]);
-      const unsigned bits = __ballot_sync(0xffffffffu, y > 0.f);
-      if (lane == 0) qc[v * NW + jw] = bits;
+    for (int it = tid; it < NV * 4 * nb; it += kFThreads) {
+      const int jj = it % nb, vs4 = it / nb, s = vs4 & 3;
+      const float* xs_ = xr + vs4 * kXS;
+      const float* wc = wsl + s * kWCols + jj;
+      float P[8];
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
+        const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
+        const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const float wv = wc[(4 * a + 32 * u4) * kWCols];
+          P[a] = u4 == 0 ? xx[a] * wv : fmaf(xx[a], wv, P[a]);
+        }
+      }
+      const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
+      sb[vs4 * cpr + cb + jj] = (q0 + q2) + (q1 + q3);
     }
   }
-  __syncthreads();  // codes ready; W_H and the residue sums are consumed
-  if (tid == 0 && !stat[ST_ABORT]) {
-    ptx::fence_proxy_async_smem();  // generic reads of the W_H buffers before the copies that overwrite them
-    for (int s = kStages - WS; s < min(nst, kStages); ++s) issue(s);
+  __syncthreads();
+  // 8 columns per byte of the code, stored straight into the code array of every
+  // CTA of the cluster (each byte has exactly one writer)
+  ptx::cluster_wait();  // every CTA of the cluster has started (arrive at kernel start)
+  {
+    const int nb8 = ncols / 8;
+    for (int e = tid; e < NV * nb8 * CS; e += kFThreads) {
+      const int c = e / (NV * nb8), vb = e % (NV * nb8), v = vb / nb8, jb = vb % nb8;
+      const float* sv = sb + v * 4 * cpr + jb * 8;
+      uint32_t byte = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float y = (sv[k] + sv[2 * cpr + k]) + (sv[cpr + k] + sv[3 * cpr + k]);
+        byte |= (y > 0.f ? 1u : 0u) << k;
+      }
+      ptx::st_dsmem_u8(ptx::dsmem_addr(reinterpret_cast<uint8_t*>(qc) + v * NW * 4 + (j0 >> 3) + jb, c), byte);
+    }
   }
+  ptx::cluster_sync();  // #1: every CTA holds all code bits
   if (rank == 0 && p.qcode_out && tid < G * NW) p.qcode_out[((size_t)b * p.Hq + (size_t)g * G) * NW + tid] = qc[tid];
   const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
   if (own_last && tid < NW) cu[(size_t)(L - 1) * NW + tid] = qc[G * NW + tid];
@@ -364,19 +374,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     for (int w = 0; w < NW; ++w) keyc[w] = qc[G * NW + w];
     // Each thread scores TPS tokens of a stage (all loads first, then the
     // arithmetic, for ILP).  Warps release stages on their own: lane 0 adds to the
-    // buffer's counter and checks the returned count one stage later, so no lane
-    // waits on the atomic; the warp that completed a stage refills its buffer.
+    // stage's counter and checks the returned count one stage later, so no lane
+    // waits on the atomic; the warp that completed a stage refills it.
     constexpr int TPS = ST / kFThreads;
     int rel_old = -1, rel_s = -1;  // lane 0: ticket of the previous stage's release
     for (int s = 0; s < nst; ++s) {
-      const int vs = s + WS, buf_i = vs % kStages;
-      if (!stat[ST_ABORT] && !ptx::mbar_wait_spin(&mbar[buf_i], (uint32_t)(vs / kStages) & 1u, kWaitTries)) {
+      if (!stat[ST_ABORT] && !ptx::mbar_wait_spin(&mbar[s % kStages], (uint32_t)(s / kStages) & 1u, kWaitTries)) {
         set_status(p.status, HATA_ERR_TIMEOUT);
         stat[ST_ABORT] = 1;
       }
       const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
       const int nb = nt / BULK_Q * BULK_Q;
-      const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + buf_i * kStageBytes);
+      const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + (s % kStages) * kStageBytes);
       uint32_t kw[TPS][NW];
 #pragma unroll
       for (int j = 0; j < TPS; ++j) {
@@ -414,16 +423,12 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       }
       __syncwarp();
       if (lane == 0) {
-        // counters never reset: the k-th stream use of a buffer ends at count (k + 1) * kNWarp
-        if (rel_s >= 0) {
-          const int rvs = rel_s + WS;
-          const int k_use = rvs / kStages - (rvs % kStages < WS ? 1 : 0);
-          if (rel_old == (k_use + 1) * kNWarp - 1 && rel_s + kStages < nst) {
-            ptx::fence_proxy_async_smem();
-            issue(rel_s + kStages);
-          }
+        // counters never reset: the k-th use of buffer s % kStages ends at count k * kNWarp
+        if (rel_s >= 0 && rel_old == ((rel_s / kStages) + 1) * kNWarp - 1 && rel_s + kStages < nst) {
+          ptx::fence_proxy_async_smem();
+          issue(rel_s + kStages);
         }
-        rel_old = atomicAdd(&done[buf_i], 1);
+        rel_old = atomicAdd(&done[s % kStages], 1);
         rel_s = s;
       }
     }
@@ -448,78 +453,78 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   // of the selection), so the candidate rows always fit the gather buffers.
   const int want = min(nmine, min(GB, 3 * ((n + CS - 1) / CS) / 2 + 16));
   {
-    // inclusive cumulative counts in place (each thread a contiguous span of bins)
-    const int span = (nbp + kFThreads - 1) / kFThreads;
-    const int v0 = min(nbp, tid * span), v1 = min(nbp, v0 + span);
-    int local = 0;
-    for (int v = v0; v < v1; ++v) local += hist[v];
-    if (tid == 0) stat[ST_SPEC] = p.nbins - 1;  // when no count exceeds `want`
+    // inclusive cumulative counts in place, BPT consecutive bins per thread; also the
+    // range of bins the other CTAs can need: from the first non-empty bin (below it
+    // every count is 0) to the first bin whose count reaches n (the unit threshold is
+    // never above it, so higher bins are sent as "at least n")
+    if (tid == 0) {
+      stat[ST_SPEC] = p.nbins - 1;  // no crossing: every bin fits
+      stat[ST_LO] = NBP;
+      stat[ST_HI] = NBP;
+    }
+    const int v0 = tid * BPT;
+    int hv[BPT], local = 0;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      hv[i] = hist[v0 + i];
+      local += hv[i];
+    }
     int total;
     int run = block_exclusive_scan<kFThreads>(local, warp_sums, &total);
-    for (int v = v0; v < v1; ++v) {
-      const int before = run;
-      run += hist[v];
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int v = v0 + i, before = run;
+      run += hv[i];
       hist[v] = run;
-      if (before <= want && run > want) stat[ST_SPEC] = v - 1;  // unique: counts never decrease
+      if (before <= want && run > want) stat[ST_SPEC] = v - 1;  // each crossing is unique: counts never decrease
+      if (before < n && run >= n) stat[ST_HI] = min(NBP, (v + 8) & ~7);
+      if (before == 0 && run > 0) stat[ST_LO] = v & ~7;
     }
   }
   __syncthreads();
-  const int Tc = stat[ST_SPEC];
-  // one pass over the scores, 8 at a time with paired 16-bit compares; the few hits
-  // take a slot from a shared counter (order does not matter: ties are ranked by index later)
-  if (Tc >= 0 && !stat[ST_ABORT]) {
-    const uint32_t t2 = (uint32_t)Tc * 0x10001u;
-    const int nvec = (nmine + 7) / 8;  // whole vectors inside tok_cap (a multiple of 16)
-    for (int e = tid; e < nvec; e += kFThreads) {
-      const uint4 w4 = reinterpret_cast<const uint4*>(Ds)[e];
-      uint32_t mk[4] = {__vcmpleu2(w4.x, t2), __vcmpleu2(w4.y, t2), __vcmpleu2(w4.z, t2), __vcmpleu2(w4.w, t2)};
-      const int valid = nmine - e * 8;
-      if (valid < 8) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (2 * q >= valid) mk[q] &= 0xffff0000u;
-          if (2 * q + 1 >= valid) mk[q] &= 0x0000ffffu;
-        }
-      }
-      const int c = (__popc(mk[0]) + __popc(mk[1]) + __popc(mk[2]) + __popc(mk[3])) >> 4;
-      if (c) {
-        int pos = atomicAdd(&s_ncand, c);
-#pragma unroll
-        for (int h = 0; h < 8; ++h)
-          if ((mk[h >> 1] >> ((h & 1) * 16)) & 1u) {
-            if (pos < GB) cand[pos] = t0 + e * 8 + h;
-            ++pos;
-          }
-      }
-    }
-  }
-  __syncthreads();
-  const int ncand = min(s_ncand, GB);  // <= want <= GB by construction
-  // ascending token order (the counter hands out slots in no fixed order): every
-  // later sum then runs over the rows in one order, so results repeat bit for bit
+  // bins [lo, hi) of the u16 cumulative histogram into slot `rank` of every CTA (8
+  // bins per 16-byte store), with (lo, hi) in the header
   {
-    int t = 0, rk = 0;
-    if (tid < ncand) {
-      t = cand[tid];
-      const int4* c4 = reinterpret_cast<const int4*>(cand);
-      int r2 = 0;
-      for (; r2 + 4 <= ncand; r2 += 4) {
-        const int4 x = c4[r2 >> 2];
-        rk += (x.x < t) + (x.y < t) + (x.z < t) + (x.w < t);
+    const int plo = stat[ST_LO], phi = stat[ST_HI];
+    const int ng = (phi - plo) / 8;
+    for (int e = tid; e < (ng + 1) * CS; e += kFThreads) {
+      const int c = e / (ng + 1), k = e % (ng + 1);
+      if (k == ng) {
+        ptx::st_dsmem_v4(ptx::dsmem_addr(&hdr[rank * 4], c), make_uint4((uint32_t)plo, (uint32_t)phi, 0u, 0u));
+      } else {
+        const int v = plo + k * 8;
+        const int* h = hist + v;
+        uint4 pk;
+        pk.x = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
+        pk.y = (uint32_t)h[2] | ((uint32_t)h[3] << 16);
+        pk.z = (uint32_t)h[4] | ((uint32_t)h[5] << 16);
+        pk.w = (uint32_t)h[6] | ((uint32_t)h[7] << 16);
+        ptx::st_dsmem_v4(ptx::dsmem_addr(&hslot[rank * NBP + v], c), pk);
       }
-      for (; r2 < ncand; ++r2) rk += cand[r2] < t;
     }
-    __syncthreads();
-    if (tid < ncand) cand[rk] = t;
-    __syncthreads();
   }
+  ptx::cluster_arrive_release();  // #2, completed by the threshold warp and after the logits (below)
+  const int Tc = stat[ST_SPEC];
+  const bool scan_cands = Tc >= 0 && !stat[ST_ABORT];
 
   const T* Kb = static_cast<const T*>(p.K) + (size_t)u * p.max_seq * D;
   const T* Vb = static_cast<const T*>(p.V) + (size_t)u * p.max_seq * D;
   T* Kr = reinterpret_cast<T*>(ring);
   T* Vr = reinterpret_cast<T*>(ring) + (size_t)GB * D;
-  // Row gathers: 16-byte cp.async pieces, one warp per K + V row pair.  An index
-  // outside this CTA's slice (never expected) is flagged and replaced by row t0.
+  // Row gathers complete on the gather mbarrier: every thread arrives once per
+  // gather (cp.async.mbarrier.arrive.noinc), so the phase ends when all its copies
+  // have landed, and any thread may wait for it.
+  uint32_t gphase = 0;
+  auto gather_commit = [&]() { ptx::cp_async_mbar_arrive_noinc(gbar); };
+  auto gather_wait = [&]() {
+    if (!ptx::mbar_wait_spin(gbar, gphase & 1u, kWaitTries)) {
+      set_status(p.status, HATA_ERR_TIMEOUT);
+      stat[ST_ABORT] = 1;
+    }
+    ++gphase;
+  };
+  // Fallback gathers (selected rows listed in `list`): every thread takes pieces.
+  // An index outside this CTA's slice (never expected) is flagged and replaced by row t0.
   auto gather_issue = [&](const int* list, int nr) {
     for (int e = tid; e < nr * 2 * RPR; e += kFThreads) {
       const int r = e / (2 * RPR), w = e % (2 * RPR);
@@ -531,71 +536,255 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       if (w < RPR) ptx::cp_async16(Kr + (size_t)r * D + w * EPV, Kb + (size_t)t * D + w * EPV);
       else ptx::cp_async16(Vr + (size_t)r * D + (w - RPR) * EPV, Vb + (size_t)t * D + (w - RPR) * EPV);
     }
+    gather_commit();
   };
-  auto gather_wait = [&]() {
-    ptx::cp_async_wait_all();
-    __syncthreads();
+  // logits (exp2 domain) of gather slots 0..nr-1 into lg[h * GB + slot], by warps
+  // w_first.. (nw of them): 16 threads per row, 8 elements each, every head at once;
+  // each thread keeps its 8-element slice of the G query vectors in registers.  With
+  // track_max, the per-head maximum goes into bmaxi.
+  auto compute_logits = [&](int nr, bool track_max, int w_first, int nw) {
+    const int sgi = lane % LT;
+    float xq[G][LE];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float4 a = reinterpret_cast<const float4*>(xp + h * D + sgi * LE)[0];
+      const float4 c = reinterpret_cast<const float4*>(xp + h * D + sgi * LE)[1];
+      xq[h][0] = a.x; xq[h][1] = a.y; xq[h][2] = a.z; xq[h][3] = a.w;
+      xq[h][4] = c.x; xq[h][5] = c.y; xq[h][6] = c.z; xq[h][7] = c.w;
+    }
+    float mx[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
+#pragma unroll 2
+    for (int rb = (warp - w_first) * (32 / LT); rb < nr; rb += nw * (32 / LT)) {  // warp-uniform trip count
+      const int r = rb + lane / LT;
+      const bool valid = r < nr;
+      const int rr = valid ? r : 0;
+      float kv[LE];
+#pragma unroll
+      for (int v = 0; v < LE / EPV; ++v) {
+        float t8[EPV];
+        Vec16<T>::load(Kr + (size_t)rr * D + sgi * LE + v * EPV, t8);
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
+      }
+      float acc[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float a = xq[h][0] * kv[0];
+#pragma unroll
+        for (int j = 1; j < LE; ++j) a = fmaf(xq[h][j], kv[j], a);
+        acc[h] = a;
+      }
+#pragma unroll
+      for (int o = 1; o < LT; o <<= 1)
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+      if (valid && sgi == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float lv = acc[h] * p.scale_log2;
+          lg[h * GB + r] = lv;
+          mx[h] = fmaxf(mx[h], lv);
+        }
+      }
+    }
+    if (track_max) {
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], LT));
+        if (lane == 0 && mx[h] != -INFINITY) atomicMax(&bmaxi[h], ord_of(mx[h]));
+      }
+    }
   };
-  gather_issue(cand, ncand);  // speculative: waited for in section 8
-
-  ptx::cluster_wait();  // every CTA of the cluster has started: remote stores are safe
-  // u16 cumulative histogram into slot `rank` of every CTA (8 bins per 16-byte store)
-  for (int e = tid; e < (nbp / 8) * CS; e += kFThreads) {
-    const int v8 = e % (nbp / 8), c = e / (nbp / 8);
-    uint4 pk;
-    const int* h = hist + v8 * 8;
-    pk.x = (uint32_t)h[0] | ((uint32_t)h[1] << 16);
-    pk.y = (uint32_t)h[2] | ((uint32_t)h[3] << 16);
-    pk.z = (uint32_t)h[4] | ((uint32_t)h[5] << 16);
-    pk.w = (uint32_t)h[6] | ((uint32_t)h[7] << 16);
-    ptx::st_dsmem_v4(ptx::dsmem_addr(&hslot[rank * nbp + v8 * 8], c), pk);
-  }
-
-  // ---- 5. unit threshold from the CS cumulative histograms -------------------
-  ptx::cluster_sync();  // #1: every CTA holds every CTA's cumulative histogram
+  // Candidates in token order, without atomics: warp w owns a contiguous run of
+  // 8-score vectors; a first pass counts its hits, a second one writes them at the
+  // warp's offset, then the warp gathers their K and V rows.  Scores are below
+  // 2^15, so in each 16-bit half of (x + (0x7fff - Tc) * 0x10001) bit 15 is set
+  // exactly when that score exceeds Tc; halves past nmine are read as 0x7fff.
+  const int nvec = (nmine + 7) / 8;  // whole vectors inside tok_cap (a multiple of 16)
+  const int nvw = (nvec + kNWarp - 1) / kNWarp;
+  const int wv0 = min(nvec, warp * nvw), wv1 = min(nvec, wv0 + nvw);
+  const uint32_t addc = (uint32_t)(0x7fff - max(Tc, 0)) * 0x10001u;
+  auto load_vec = [&](int e) -> uint4 {
+    uint4 w4 = reinterpret_cast<const uint4*>(Ds)[min(e, max(nvec - 1, 0))];
+    const int valid = e < wv1 ? nmine - e * 8 : 0;
+    if (valid < 8) {
+      uint32_t* wq = reinterpret_cast<uint32_t*>(&w4);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (2 * q >= valid) wq[q] = (wq[q] & 0xffff0000u) | 0x7fffu;
+        if (2 * q + 1 >= valid) wq[q] = (wq[q] & 0x0000ffffu) | 0x7fff0000u;
+      }
+    }
+    return w4;
+  };
+  auto hit_bits = [&](const uint4& w4, uint32_t (&x)[4]) {  // bit 15 / 31 of x[q]: score 2q / 2q+1 <= Tc
+    x[0] = ~(w4.x + addc) & 0x80008000u;
+    x[1] = ~(w4.y + addc) & 0x80008000u;
+    x[2] = ~(w4.z + addc) & 0x80008000u;
+    x[3] = ~(w4.w + addc) & 0x80008000u;
+  };
   {
-    // unit totals, one bin per thread; T = number of bins whose cumulative total is below n
-    int below = 0;
-    for (int v = tid; v < nbp; v += kFThreads) {
-      int cv[kMaxCS];
+    int c = 0;
+    if (scan_cands)
+      for (int e = wv0 + lane; e < wv1; e += 128) {  // four vectors per lane per trip, loads first
+        uint4 w4[4];
 #pragma unroll
-      for (int c = 0; c < kMaxCS; ++c) cv[c] = c < CS ? (int)hslot[c * nbp + v] : 0;
-      int tv = 0;
+        for (int i = 0; i < 4; ++i) w4[i] = load_vec(e + 32 * i);
 #pragma unroll
-      for (int c = 0; c < kMaxCS; ++c) tv += cv[c];
-      hist[v] = tv;  // the local counts are no longer needed (this CTA's are in hslot[rank])
-      below += (v < p.nbins && tv < n);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
-    if (lane == 0) warp_sums[warp] = below;
-    __syncthreads();
-    if (warp == 0) {
-      int Tth = lane < kNWarp ? warp_sums[lane] : 0;
-#pragma unroll
-      for (int o = 16; o; o >>= 1) Tth += __shfl_xor_sync(0xffffffffu, Tth, o);
-      const int Tcl = min(Tth, p.nbins - 1);
-      // per source CTA (lane c): cumulative count below T and at T
-      int cb = 0, ce = 0;
-      if (lane < CS) {
-        cb = Tcl > 0 ? (int)hslot[lane * nbp + Tcl - 1] : 0;
-        ce = (int)hslot[lane * nbp + Tcl] - cb;
+        for (int i = 0; i < 4; ++i) {
+          uint32_t x[4];
+          hit_bits(w4[i], x);
+          c += __popc(x[0]) + __popc(x[1]) + __popc(x[2]) + __popc(x[3]);
+        }
       }
-      const int lb = __reduce_add_sync(0xffffffffu, lane < rank ? cb : 0);
-      const int eb = __reduce_add_sync(0xffffffffu, lane < rank ? ce : 0);
-      const int myl = __shfl_sync(0xffffffffu, cb, rank);
-      const int mye = __shfl_sync(0xffffffffu, ce, rank);
-      if (lane == 0) {
-        stat[ST_T] = n == 0 ? 0 : Tth;
-        stat[ST_M] = n == 0 ? 0 : n - (Tcl > 0 ? hist[Tcl - 1] : 0);
-        stat[ST_LESS_BEFORE] = lb;
-        stat[ST_EQ_BEFORE] = eb;
-        stat[ST_MYLESS] = myl;
-        stat[ST_MYEQ] = mye;
-      }
-    }
-    __syncthreads();
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) warp_sums[warp] = c;
   }
+  __syncthreads();
+  int wbase = 0, ncand_all = 0;
+#pragma unroll
+  for (int w = 0; w < kNWarp; ++w) {
+    const int x = warp_sums[w];
+    wbase += w < warp ? x : 0;
+    ncand_all += x;
+  }
+  const int ncand = min(ncand_all, GB);  // <= want <= GB by construction
+  if (scan_cands) {
+    const int wstart = wbase;
+    const unsigned lm = (1u << lane) - 1u;
+    for (int e0 = wv0; e0 < wv1; e0 += 128) {  // warp-uniform trip count
+      uint4 w4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w4[i] = load_vec(e0 + 32 * i + lane);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t x[4];
+        hit_bits(w4[i], x);
+        const int ci = __popc(x[0]) + __popc(x[1]) + __popc(x[2]) + __popc(x[3]);  // <= 8
+        if (__ballot_sync(0xffffffffu, ci != 0) == 0u) continue;
+        const unsigned b0 = __ballot_sync(0xffffffffu, ci & 1), b1 = __ballot_sync(0xffffffffu, ci & 2),
+                       b2 = __ballot_sync(0xffffffffu, ci & 4), b3 = __ballot_sync(0xffffffffu, ci & 8);
+        int pos = wbase + __popc(b0 & lm) + 2 * __popc(b1 & lm) + 4 * __popc(b2 & lm) + 8 * __popc(b3 & lm);
+        wbase += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2) + 8 * __popc(b3);
+        const int tb = t0 + (e0 + 32 * i + lane) * 8;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (x[q] & 0x8000u) {
+            if (pos < GB) cand[pos] = tb + 2 * q;
+            ++pos;
+          }
+          if (x[q] & 0x80000000u) {
+            if (pos < GB) cand[pos] = tb + 2 * q + 1;
+            ++pos;
+          }
+        }
+      }
+    }
+    __syncwarp();
+    // this warp's candidate rows: (candidate, 16-byte piece) pairs over the lanes
+    const int q0 = min(wstart, GB), nq = min(wbase, GB) - q0;
+#pragma unroll 2
+    for (int e = lane; e < nq * 2 * RPR; e += 32) {
+      const int q = q0 + e / (2 * RPR), pc = e % (2 * RPR);
+      const int t = cand[q];
+      if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kb + (size_t)t * D + pc * EPV);
+      else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vb + (size_t)t * D + (pc - RPR) * EPV);
+    }
+  }
+  gather_commit();  // gather phase 0: the candidates' rows
+  if (tid < G) {
+    part[tid * 4] = -INFINITY;
+    part[tid * 4 + 1] = 0.f;
+    bmaxi[tid] = ord_of(-INFINITY);
+  }
+
+  // ---- 5. warp 0: unit threshold and the selected candidates; the other warps:
+  //         the candidates' logits (as soon as their rows have landed) -----------
+  if (warp == 0) {
+    ptx::cluster_wait();  // #2: every CTA holds every CTA's cumulative histogram range
+    // T = the smallest score v whose unit total (sum of the CS cumulative counts)
+    // is at least n; the total at the top bin is L >= n.  Rounds of a 32-way split
+    // of [lo, hi], one probe per lane.  Source c sent bins [lo_c, hi_c): below
+    // lo_c its count is 0, from hi_c on it is at least n (counted as n).
+    int loc[kMaxCS], hic[kMaxCS];
+#pragma unroll
+    for (int c = 0; c < kMaxCS; ++c) {  // sources past CS: an empty range below every bin
+      const int cc = min(c, CS - 1);
+      const int l_ = hdr[cc * 4], h_ = hdr[cc * 4 + 1];
+      loc[c] = c < CS ? l_ : NBP;
+      hic[c] = c < CS ? h_ : NBP + 1;
+    }
+    auto total_at = [&](int v) {
+      int hv[kMaxCS];
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) hv[c] = hslot[min(c, CS - 1) * NBP + v];
+      int t = 0;
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) t += v < loc[c] ? 0 : (v >= hic[c] ? n : hv[c]);
+      return t;
+    };
+    int lo = 0, hi = p.nbins - 1;
+    while (lo < hi) {  // warp-uniform
+      const int step = (hi - lo + 32) / 32;
+      const int v = min(hi, lo + (lane + 1) * step - 1);
+      const unsigned ok = __ballot_sync(0xffffffffu, total_at(v) >= n);
+      const int f = __ffs(ok) - 1;  // lane 31 probes hi, which always qualifies
+      hi = min(hi, lo + (f + 1) * step - 1);
+      lo = lo + f * step;
+    }
+    const int Tth = n == 0 ? 0 : lo;
+    // per source CTA (lane c): cumulative count below T and at T (exact: T <= hi_c - 1)
+    int cb = 0, ce = 0;
+    if (lane < CS) {
+      const int lo_c = hdr[lane * 4];
+      const int h1 = Tth - 1 < lo_c ? 0 : (int)hslot[lane * NBP + max(Tth - 1, 0)];
+      const int h0 = Tth < lo_c ? 0 : (int)hslot[lane * NBP + Tth];
+      cb = Tth > 0 ? h1 : 0;
+      ce = h0 - cb;
+    }
+    const int lb = __reduce_add_sync(0xffffffffu, lane < rank ? cb : 0);
+    const int eb = __reduce_add_sync(0xffffffffu, lane < rank ? ce : 0);
+    const int below_all = __reduce_add_sync(0xffffffffu, cb);
+    const int myl = __shfl_sync(0xffffffffu, cb, rank);
+    const int mye = __shfl_sync(0xffffffffu, ce, rank);
+    const int mq = n == 0 ? 0 : n - below_all;
+    if (lane == 0) {
+      stat[ST_T] = Tth;
+      stat[ST_M] = mq;
+      stat[ST_LESS_BEFORE] = lb;
+      stat[ST_EQ_BEFORE] = eb;
+      stat[ST_MYLESS] = myl;
+      stat[ST_MYEQ] = mye;
+    }
+    // the selected candidates (when they hold the whole selection of this slice),
+    // in ascending token order: scores below T, and the first quota = m - (ties of
+    // earlier CTAs) ties at T
+    const int nsel_w = myl + max(0, min(mq - eb, mye));
+    if ((nsel_w == 0 || Tth <= Tc) && nsel_w > 0) {
+      const int quota = max(0, mq - eb);
+      const unsigned lm = (1u << lane) - 1u;
+      int lt_run = 0, eq_run = 0;
+      for (int r0 = 0; r0 < ncand; r0 += 32) {
+        const int r = r0 + lane;
+        const int dv = r < ncand ? (int)Ds[cand[r] - t0] : INT_MAX;
+        const bool lt = dv < Tth, eq = dv == Tth;
+        const unsigned blt = __ballot_sync(0xffffffffu, lt), beq = __ballot_sync(0xffffffffu, eq);
+        const int ltpre = lt_run + __popc(blt & lm), eqpre = eq_run + __popc(beq & lm);
+        if (lt || (eq && eqpre < quota)) rowl[ltpre + min(eqpre, quota)] = (uint16_t)r;
+        lt_run += __popc(blt);
+        eq_run += __popc(beq);
+      }
+      if (lane == 0) s_nrow = lt_run + min(eq_run, quota);
+    }
+  } else {
+    gather_wait();  // phase 0
+    compute_logits(ncand, false, 1, kNWarp - 1);
+    ptx::cluster_wait();  // #2 (these warps' side)
+  }
+  if (warp == 0) gphase = 1;  // warp 0 did not wait on phase 0; the barrier below orders it after
+  __syncthreads();
   const int Tt = stat[ST_T], m = stat[ST_M];
   const int less_before = stat[ST_LESS_BEFORE], eq_before = stat[ST_EQ_BEFORE];
   const int sel_before = less_before + min(eq_before, m);
@@ -604,7 +793,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   // the candidates hold every selected token of this slice when T <= Tc
   const bool covered = nsel_here == 0 || Tt <= Tc;
 
-  // ---- 7. ascending indices (only when asked for) and the row list --------------
+  // ---- 7. ascending indices (only when asked for) and the fallback row list -----
   int32_t* ix = p.idx_out ? p.idx_out + (size_t)u * p.k : nullptr;
   // Passes over this CTA's scores go 8192 at a time: each thread owns 16
   // consecutive scores of the pass (two 16-byte loads); scores past nmine read as 0xffff.
@@ -659,174 +848,108 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     if (ix && rank == 0)
       for (int j = n + tid; j < p.k; j += kFThreads) ix[j] = -1;
   }
-  // selected candidates (covered case), kept in ascending token order: scores below
-  // T, and the first quota = m - (ties of earlier CTAs) ties at T (the candidates
-  // hold every tie of this slice, sorted by index)
-  if (covered && nsel_here > 0) {
-    int dv = INT_MAX;
-    if (tid < ncand) dv = Ds[cand[tid] - t0];  // ncand <= GB < kFThreads
-    const bool lt = dv < Tt, eq = dv == Tt;
-    const unsigned blt = __ballot_sync(0xffffffffu, lt), beq = __ballot_sync(0xffffffffu, eq);
-    __syncthreads();  // warp_sums is free again
-    if (lane == 0) warp_sums[warp] = __popc(blt) | (__popc(beq) << 16);
-    __syncthreads();
-    int pre = 0, tot = 0;
-    for (int w = 0; w < kNWarp; ++w) {
-      const int x = warp_sums[w];
-      pre += w < warp ? x : 0;
-      tot += x;
-    }
-    const unsigned lm = (1u << lane) - 1u;
-    const int ltpre = (pre & 0xffff) + __popc(blt & lm), eqpre = (pre >> 16) + __popc(beq & lm);
-    const int quota = max(0, m - eq_before);
-    if (lt || (eq && eqpre < quota)) rowl[ltpre + min(eqpre, quota)] = (uint16_t)tid;
-    if (tid == 0) s_nrow = (tot & 0xffff) + min(tot >> 16, quota);
-  }
 
   // ---- 8. attention partials over this CTA's selected rows -----------------------
   constexpr int OPT = (G * D + kFThreads - 1) / kFThreads;  // output elements per thread
   float oacc[OPT];
 #pragma unroll
   for (int q = 0; q < OPT; ++q) oacc[q] = 0.f;
-  if (tid < G) {
-    part[tid * 4] = -INFINITY;
-    part[tid * 4 + 1] = 0.f;
-    bmaxi[tid] = ord_of(-INFINITY);
-  }
-  gather_wait();  // the speculative rows (issued before the threshold was known); also publishes s_nrow
-  const int nrows_total = stat[ST_ABORT] ? 0 : (covered ? s_nrow : min(nsel_here, p.sel_cap));
-  for (int r0 = 0; r0 < nrows_total; r0 += GB) {
-    const int nr = min(GB, nrows_total - r0);
-    if (!covered) {  // the guess missed: gather the selected rows batch by batch
-      __syncthreads();  // previous batch's readers are done with the buffers
-      gather_issue(sel + r0, nr);
-      gather_wait();
+  // Softmax and P.V over nr rows whose logits are in lg (slot rmap[i], or i without
+  // a map) against the running maximum max(part.m, bmaxi), folded into oacc and
+  // the running (max, sum) in part.
+  auto softmax_pv = [&](int nr, const uint16_t* rmap) {
+    for (int e = tid; e < G * nr; e += kFThreads) {
+      const int h = e / nr, i = e - h * nr;
+      const int sl = rmap ? (int)rmap[i] : i;
+      const float mn = fmaxf(part[h * 4], float_of_ord(bmaxi[h]));
+      lg[h * GB + sl] = exp2f(lg[h * GB + sl] - mn);
     }
-    // logits (exp2 domain): 16 threads per row, 8 elements each, every head at once;
-    // each thread keeps its 8-element slice of the G query vectors in registers
-    {
-      const int sgi = lane % LT;
-      float xq[G][LE];
+    __syncthreads();
+    // P.V: thread (column pair cp, row group rg) sums rows rg, rg + PVG, ... for every
+    // head (and the probabilities), then the PVG partial sums of each output go
+    // through shared memory (the K rows' buffer, free once the logits are done)
+    const int cp = tid % (D / 2), rg = tid / (D / 2);
+    float pacc[G][2], lsum[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int j = 0; j < LE; ++j) {
-          const int i = sgi * LE + j;
-          xq[h][j] = xr[(h * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)];
-        }
-      float mx[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
-      for (int rb = warp * (32 / LT); rb < nr; rb += kFThreads / LT) {  // warp-uniform trip count
-        const int r = rb + lane / LT;
-        const bool valid = r < nr;
-        const int rr = valid ? (covered ? (int)rowl[r] : r) : 0;
-        float kv[LE];
-#pragma unroll
-        for (int v = 0; v < LE / EPV; ++v) {
-          float t8[EPV];
-          Vec16<T>::load(Kr + (size_t)rr * D + sgi * LE + v * EPV, t8);
-#pragma unroll
-          for (int j = 0; j < EPV; ++j) kv[v * EPV + j] = t8[j];
-        }
-        float acc[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float a = xq[h][0] * kv[0];
-#pragma unroll
-          for (int j = 1; j < LE; ++j) a = fmaf(xq[h][j], kv[j], a);
-          acc[h] = a;
-        }
-#pragma unroll
-        for (int o = 1; o < LT; o <<= 1)
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-        if (valid && sgi == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float lv = acc[h] * p.scale_log2;
-            lg[h * GB + r] = lv;
-            mx[h] = fmaxf(mx[h], lv);
-          }
-        }
+    for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
+#pragma unroll 4
+    for (int r = rg; r < nr; r += PVG) {
+      const int sl = rmap ? (int)rmap[r] : r;
+      float v0, v1;
+      if constexpr (ESZ == 2) {
+        const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)sl * D)[cp]);
+        v0 = f.x;
+        v1 = f.y;
+      } else {
+        const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)sl * D)[cp];
+        v0 = f.x;
+        v1 = f.y;
       }
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], LT));
-        if (lane == 0 && mx[h] != -INFINITY) atomicMax(&bmaxi[h], ord_of(mx[h]));
+        const float pr_ = lg[h * GB + sl];
+        pacc[h][0] = fmaf(pr_, v0, pacc[h][0]);
+        pacc[h][1] = fmaf(pr_, v1, pacc[h][1]);
+        lsum[h] += pr_;
       }
     }
+    float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
+    if (cp == 0)
+#pragma unroll
+      for (int h = 0; h < G; ++h) redl[rg * G + h] = lsum[h];
     __syncthreads();
-    // probabilities against the running maximum, every thread a few
-    for (int e = tid; e < G * nr; e += kFThreads) {
-      const int h = e / nr, r = e - h * nr;
-      const float mn = fmaxf(part[h * 4], float_of_ord(bmaxi[h]));
-      lg[h * GB + r] = exp2f(lg[h * GB + r] - mn);
-    }
-    __syncthreads();
-    // P.V: thread (column pair cp, row group rg) sums rows rg, rg + PVG, ... for every head
-    // (column pair 0 also sums the probabilities), then the PVG partial sums of each
-    // output go through shared memory (the K rows' buffer, free once the logits are done)
-    {
-      const int cp = tid % (D / 2), rg = tid / (D / 2);
-      float pacc[G][2], lsum[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
-      for (int r = rg; r < nr; r += PVG) {
-        const int rr = covered ? (int)rowl[r] : r;
-        float v0, v1;
-        if constexpr (ESZ == 2) {
-          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)rr * D)[cp]);
-          v0 = f.x;
-          v1 = f.y;
-        } else {
-          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)rr * D)[cp];
-          v0 = f.x;
-          v1 = f.y;
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float pr_ = lg[h * GB + r];
-          pacc[h][0] = fmaf(pr_, v0, pacc[h][0]);
-          pacc[h][1] = fmaf(pr_, v1, pacc[h][1]);
-          lsum[h] += pr_;
-        }
-      }
-      float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
-      if (cp == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) redl[rg * G + h] = lsum[h];
-      __syncthreads();
-#pragma unroll
-      for (int q = 0; q < OPT; ++q) {
-        const int e = tid + q * kFThreads;
-        if (e < G * D) {
-          const int h = e / D, i = e % D;
-          const float m_old = part[h * 4];
-          const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
-          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
-          oacc[q] = fmaf(oacc[q], alpha, sum);
-        }
-      }
-      __syncthreads();  // every thread has read the running maxima of this batch
-      if (tid < G) {
-        const int h = tid;
+    for (int q = 0; q < OPT; ++q) {
+      const int e = tid + q * kFThreads;
+      if (e < G * D) {
+        const int h = e / D, i = e % D;
         const float m_old = part[h * 4];
         const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
         const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
-        float ls = 0.f;
+        float sum = 0.f;
 #pragma unroll
-        for (int j = 0; j < PVG; ++j) ls += redl[j * G + h];
-        part[h * 4 + 1] = part[h * 4 + 1] * alpha + ls;
-        part[h * 4] = mn;
-        bmaxi[h] = ord_of(-INFINITY);
+        for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
+        oacc[q] = fmaf(oacc[q], alpha, sum);
       }
+    }
+    __syncthreads();  // every thread has read the running maxima of this batch
+    if (tid < G) {
+      const int h = tid;
+      const float m_old = part[h * 4];
+      const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
+      const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+      float ls = 0.f;
+#pragma unroll
+      for (int j = 0; j < PVG; ++j) ls += redl[j * G + h];
+      part[h * 4 + 1] = part[h * 4 + 1] * alpha + ls;
+      part[h * 4] = mn;
+      bmaxi[h] = ord_of(-INFINITY);
+    }
+  };
+  if (covered) {
+    // the candidates' rows and logits are in place: one batch over the selected ones
+    const int nsel = stat[ST_ABORT] ? 0 : s_nrow;
+    for (int i = tid; i < nsel; i += kFThreads) {  // per-head maximum over the selected rows
+      const int sl = rowl[i];
+#pragma unroll
+      for (int h = 0; h < G; ++h) atomicMax(&bmaxi[h], ord_of(lg[h * GB + sl]));
+    }
+    __syncthreads();
+    if (nsel > 0) softmax_pv(nsel, rowl);
+  } else if (!stat[ST_ABORT]) {
+    // the guess missed: gather the selected rows batch by batch
+    const int nrows_total = min(nsel_here, p.sel_cap);
+    for (int r0 = 0; r0 < nrows_total; r0 += GB) {
+      const int nr = min(GB, nrows_total - r0);
+      __syncthreads();  // previous batch's readers are done with the buffers
+      gather_issue(sel + r0, nr);
+      gather_wait();
+      compute_logits(nr, true, 0, kNWarp);
+      __syncthreads();
+      softmax_pv(nr, nullptr);
     }
   }
   __syncthreads();
@@ -846,23 +969,33 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     const int owner = e / (2 * G), w = e % (2 * G);
     ptx::st_dsmem_f32(ptx::dsmem_addr(&mslot[rank * stride + w], owner), part[(w >> 1) * 4 + (w & 1)]);
   }
-  ptx::cluster_sync();  // #4: every CTA holds the partials of its columns
+  ptx::cluster_sync();  // #3: every CTA holds the partials of its columns
   for (int col = tid; col < mc; col += kFThreads) {
     const int e = rank * mc + col;
     if (e < G * D) {
-      const int h = e / D, i = e % D;
+      const int h = e / D;
+      // all sources' (max, sum, column) first, then the log-sum-exp merge
+      float mv[kMaxCS], lv[kMaxCS], ov[kMaxCS];
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) {
+        const int cc = min(c, CS - 1);
+        mv[c] = c < CS ? mslot[cc * stride + 2 * h] : -INFINITY;
+        lv[c] = mslot[cc * stride + 2 * h + 1];
+        ov[c] = mslot[cc * stride + 2 * G + col];
+      }
       float M = -INFINITY;
-      for (int c = 0; c < CS; ++c) M = fmaxf(M, mslot[c * stride + 2 * h]);
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) M = fmaxf(M, mv[c]);
       float l = 0.f, o = 0.f;
       if (M != -INFINITY)
-        for (int c = 0; c < CS; ++c) {
-          const float mcv = mslot[c * stride + 2 * h];
-          if (mcv == -INFINITY) continue;
-          const float w = exp2f(mcv - M);
-          l = fmaf(mslot[c * stride + 2 * h + 1], w, l);
-          o = fmaf(mslot[c * stride + 2 * G + col], w, o);
+#pragma unroll
+        for (int c = 0; c < kMaxCS; ++c) {
+          if (mv[c] == -INFINITY) continue;
+          const float w = exp2f(mv[c] - M);
+          l = fmaf(lv[c], w, l);
+          o = fmaf(ov[c], w, o);
         }
-      static_cast<T*>(p.out)[((size_t)b * p.Hq + (size_t)g * G + h) * D + i] = from_f32<T>(l > 0.f ? o / l : 0.f);
+      static_cast<T*>(p.out)[((size_t)b * p.Hq + (size_t)g * G + h) * D + (e % D)] = from_f32<T>(l > 0.f ? o / l : 0.f);
     }
   }
   if (stat[ST_ABORT] && tid == 0) {
@@ -880,6 +1013,7 @@ struct Plan {
   bool ok;
   int CS, tok_cap, sel_cap, nbins, stages;
   size_t smem;
+  SmemLayout lay;
 };
 
 // Clusters of CS CTAs that can be resident at once (one CTA per SM), cached per
@@ -958,17 +1092,16 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
     pl.sel_cap = std::min(k, tok_cap);
     pl.nbins = G * d.hash_bits + 1;
     pl.stages = 0;
-    // W_H occupies the first ceil(d r 4 / stage) ring buffers until the encode is done
-    const int w_stages = (kHeadDim * R * 4 + kStageBytes - 1) / kStageBytes;
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
       (void)cudaGetLastError();
       return best;
     }
-    for (int st = kMaxStages; st >= std::max(kMinStages, w_stages + 1); --st) {
+    for (int st = kMaxStages; st >= kMinStages; --st) {
       const size_t sm = smem_layout(G, NW, esize, tok_cap, pl.sel_cap, pl.nbins, CS, st).total;
       if (sm + fa.sharedSizeBytes <= 227 * 1024) {  // + static shared memory
         pl.stages = st;
+        pl.lay = smem_layout(G, NW, esize, tok_cap, pl.sel_cap, pl.nbins, CS, st);
         pl.smem = std::max<size_t>(sm, kOneCtaSmem);
         break;
       }
@@ -1118,6 +1251,7 @@ cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const voi
   prm.sel_cap = pl.sel_cap;
   prm.flags = d.flags;
   prm.stages = pl.stages;
+  prm.lay = pl.lay;
   prm.scale_log2 = scale * 1.4426950408889634f;
   return dispatch<LaunchFn>(d, pl, d, prm, st);
 }
