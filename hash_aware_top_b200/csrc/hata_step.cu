@@ -4,33 +4,34 @@
 //
 // A unit's L cached tokens are split evenly over the CS CTAs of its cluster.
 // Each CTA:
-//   1. streams its slice of the code cache into a 2-6 stage shared-memory ring
-//      with bulk (TMA) copies, evict-first in L2, issued as soon as L is known;
-//   2. encodes the G queries and the new key over all r columns of W_H itself
-//      (the arithmetic of warp_dot128, so the codes equal hata_encode_append's
-//      decode form bit for bit; no exchange between CTAs); the CTA owning slot
-//      L - 1 appends the key code to the cache;
+//   1. streams its slice of the code cache into a shared-memory ring with bulk
+//      (TMA) copies, evict-first in L2, issued as soon as L is known, and copies
+//      the KV head's W_H (bulk, kept in L2) into shared memory;
+//   2. encodes the G queries and the new key over all r columns itself (the
+//      arithmetic of warp_dot128, so the codes equal hata_encode_append's decode
+//      form bit for bit; no exchange between CTAs); the CTA owning slot L - 1
+//      appends the key code to the cache;
 //   3. scores every token of its slice (xor + popc with the GQA sum folded into
 //      per-word constants and a carry-save popc sum), keeping the u16 scores and
 //      their histogram in shared memory; warps release ring stages on their own;
-//   4. turns the histogram into a cumulative one and stores it (u16) into its
-//      slot of every CTA; takes as candidates every token scoring at most Tc
-//      (the largest score whose count fits about 1.5x its fair share of the
-//      selection) and starts gathering those K/V rows (cp.async) right away;
-//   5. after a cluster barrier, every CTA sums the CS cumulative histograms
-//      (one bin per thread) to find the unit's threshold T (the smallest score
-//      with at least n = min(k, L) tokens at or below it), the tie quota m and
-//      the counts of earlier CTAs, so ties go to the lower token index exactly
-//      as in a global sort;
+//   4. turns the histogram into a cumulative one and stores the bins the others
+//      can need (u16) into its slot of every CTA; takes as candidates, in token
+//      order, every token scoring at most Tc (the largest score whose count fits
+//      about 1.5x its fair share of the selection), gathers their K/V rows with
+//      cp.async and computes their logits while the cluster barrier completes;
+//   5. one warp sums the CS cumulative histograms to find the unit's threshold T
+//      (the smallest score with at least n = min(k, L) tokens at or below it), the
+//      tie quota m and the counts of earlier CTAs, so ties go to the lower token
+//      index exactly as in a global sort, and marks the selected candidates;
 //   6. computes the flash-decode partial (max, sum, weighted V) of each of the G
-//      query heads over its selected rows (falling back to a second gather when
+//      query heads over its selected rows (falling back to gathering them when
 //      T > Tc), and stores each partial's column slice into the CTA that owns
 //      those output columns; after a last cluster barrier every CTA merges its
 //      columns (log-sum-exp) and writes them.
 // Cross-CTA traffic is only stores into other CTAs' shared memory before a
 // hardware cluster barrier: no remote loads, no global-memory flags, no
 // workspace.  The only waits are bounded mbarrier waits on this CTA's own
-// bulk copies and cp.async completion.
+// copies.
 #include <algorithm>
 #include <climits>
 #include <map>
@@ -51,7 +52,6 @@ constexpr int kMaxStages = 6;        // ring stages (32 KB each), 2..6 depending
 constexpr int kMinStages = 2;
 constexpr int kStageBytes = 32768;
 constexpr int kTokCap = 65520;       // max tokens per CTA: u16 scores and u16 cumulative counts
-constexpr int kWCols = 32;           // W_H columns staged per encode batch
 constexpr int kXS = 36;              // floats per residue row of an encoded vector (32 used, padded)
 constexpr int kMaxCS = 16;           // largest cluster
 constexpr int kMaxGB = 256;          // largest gather batch (rows); below kFThreads: one candidate per thread
@@ -59,7 +59,7 @@ constexpr int kOneCtaSmem = 116 * 1024;  // dynamic shared memory that keeps one
 constexpr uint32_t kWaitTries = 1u << 22;
 
 struct SmemLayout {
-  uint32_t ring, D, hist, hslot, xr, xp, sel, lg, part, mslot, stat, mbar, total;
+  uint32_t ring, W, D, hist, hslot, xr, xp, sel, lg, part, mslot, stat, mbar, total;
   int nbp, mcols, gb;
 };
 
@@ -90,10 +90,6 @@ struct Bump {
 };
 
 // Output columns merged by each CTA of a cluster of CS (the last one may have fewer).
-// W_H columns encoded by each CTA of a cluster of CS: ceil(r / CS) rounded up to
-// whole bytes of the code (the last ranks may get fewer, or none).
-__host__ __device__ inline int enc_cols_per_cta(int R, int CS) { return ((R + CS - 1) / CS + 7) / 8 * 8; }
-
 __host__ __device__ inline int merge_cols(int G, int CS) { return (G * kHeadDim + CS - 1) / CS; }
 
 __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int tok_cap, int sel_cap, int nbins,
@@ -105,7 +101,8 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int 
   s.gb = stages * kStageBytes / (2 * kHeadDim * esize);
   if (s.gb > kMaxGB) s.gb = kMaxGB;
   s.ring = b.take(stages * kStageBytes, 128);
-  s.D = b.take(max(tok_cap * 2, kHeadDim * kWCols * 4 + (G + 1) * 4 * enc_cols_per_cta(NW * 32, CS) * 4), 16);  // scores; first the encode's W_H columns and residue sums
+  s.W = b.take(kHeadDim * NW * 32 * 4, 128);        // W_H of the unit's KV head, fp32
+  s.D = b.take(max(tok_cap * 2, (G + 1) * 4 * NW * 32 * 4), 16);  // scores; first the encode's residue sums
   s.hist = b.take((s.nbp + kFThreads - 1) / kFThreads * kFThreads * 4, 16);  // counts, then cumulative (padded)
   s.hslot = b.take(CS * s.nbp * 2, 16);               // u16 cumulative histograms from every CTA
   s.xr = b.take((G + 1) * 4 * kXS * 4, 16);           // G queries + new key, fp32, residue-major
@@ -115,7 +112,7 @@ __host__ __device__ inline SmemLayout smem_layout(int G, int NW, int esize, int 
   s.part = b.take(G * 4 * 4, 16);                     // running (max, sum, alpha) per head
   s.mslot = b.take(CS * (s.mcols + 2 * G) * 4, 16);   // partials for this CTA's output columns
   s.stat = b.take(16 * 4, 16);
-  s.mbar = b.take((kMaxStages + 1) * 8, 8);  // ring stages + the row gathers
+  s.mbar = b.take((kMaxStages + 2) * 8, 8);  // ring stages, the row gathers, W_H
   s.total = b.take(0, 128);
   return s;
 }
@@ -228,30 +225,24 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   if (!early) ptx::pdl_wait();
   ptx::pdl_launch_dependents();
 
-  // ---- 1. loads: seq_lens, q, this CTA's W_H columns; then the codes stream ---
+  // ---- 1. loads: seq_lens, q, W_H (bulk copy); then the codes stream ----------
   const int Lraw = p.seq_lens ? p.seq_lens[b] : p.max_seq;
   const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
   uint4 xv = make_uint4(0u, 0u, 0u, 0u);
   // query vectors do not depend on L: load them now unless they may still be being written
   if (!early && tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
-  // This CTA encodes columns [j0, j0 + ncols) of W_H (whole bytes of the code), in
-  // batches of up to kWCols columns staged in shared memory (one batch from CS = 4 on).
-  const int cpr = enc_cols_per_cta(R, CS);
-  const int j0 = rank * cpr, ncols = max(0, min(cpr, R - j0));
-  float* wsl = reinterpret_cast<float*>(smem + S.D);       // [D][kWCols] W_H columns (the scores' space, unused yet)
-  float* sb = wsl + D * kWCols;                             // [NV][4][cpr] residue sums
-  const float* Wg = p.W + (size_t)g * D * R;
-  auto issue_w = [&](int cb) {
-    const int nq = min(kWCols, ncols - cb) / 4;  // 16-byte pieces per row
-    for (int e = tid; e < D * nq; e += kFThreads) {
-      const int i = e / nq, q4 = e % nq;
-      ptx::cp_async16(wsl + i * kWCols + q4 * 4, Wg + (size_t)i * R + j0 + cb + q4 * 4);
-    }
-  };
-  if (ncols > 0) issue_w(0);
+  float* Wsm = reinterpret_cast<float*>(smem + S.W);  // W_H of this KV head, [D][R] fp32
+  uint64_t* wbar = &mbar[kMaxStages + 1];
   if (tid == 0) {
-    for (int s = 0; s <= kMaxStages; ++s) ptx::mbar_init(&mbar[s], s < kMaxStages ? 1u : (uint32_t)kFThreads);
+    for (int s = 0; s < kMaxStages + 2; ++s) ptx::mbar_init(&mbar[s], s == kMaxStages ? (uint32_t)kFThreads : 1u);
     ptx::fence_mbarrier_init();
+    // W_H: every CTA of the cluster reads the same matrix, so keep it in L2
+    constexpr uint32_t WB = D * R * 4, WCH = 32768;
+    const char* Wsrc = reinterpret_cast<const char*>(p.W + (size_t)g * D * R);
+    const uint64_t pol_keep = ptx::policy_evict_last();
+    ptx::mbar_arrive_expect_tx(wbar, WB);
+    for (uint32_t o = 0; o < WB; o += WCH)
+      ptx::bulk_g2s(reinterpret_cast<char*>(Wsm) + o, Wsrc + o, min(WCH, WB - o), wbar, pol_keep);
   }
   if (tid < kMaxStages) {
     done[tid] = 0;
@@ -288,7 +279,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   if (tid == 0)
     for (int s = 0; s < min(nst, kStages); ++s) issue(s);
 
-  // ---- 2. encode this CTA's W_H columns for the G queries and the new key --------
+  // ---- 2. every CTA encodes the G queries and the new key itself (all r columns) --
   if (early) {
     ptx::pdl_wait();  // q and the new key row come from the preceding kernel
     if (tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
@@ -310,58 +301,52 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       if (v < G) xp[v * D + i] = xe[e];
     }
   }
-  // y = x . W_H[:, j] in the order of warp_dot128: lane l of that function is
-  // (residue s = l % 4, a = l / 4); its partial (u = 0 product, then FMAs for +32,
-  // +64, +96) and the butterfly levels 16, 8, 4 stay inside one residue, so one
-  // thread here computes the residue sum S_s of one (vector, column), and the
-  // levels 2 and 1 give y = (S_0 + S_2) + (S_1 + S_3).
-  for (int cb = 0; cb < ncols; cb += kWCols) {
-    const int nb = min(kWCols, ncols - cb);
-    if (cb > 0) {
-      __syncthreads();  // the previous batch's readers are done with the staged columns
-      issue_w(cb);
-    }
-    ptx::cp_async_wait_all();
-    __syncthreads();
-    for (int it = tid; it < NV * 4 * nb; it += kFThreads) {
-      const int jj = it % nb, vs4 = it / nb, s = vs4 & 3;
-      const float* xs_ = xr + vs4 * kXS;
-      const float* wc = wsl + s * kWCols + jj;
-      float P[8];
-#pragma unroll
-      for (int u4 = 0; u4 < 4; ++u4) {
-        const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
-        const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
-        const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-        for (int a = 0; a < 8; ++a) {
-          const float wv = wc[(4 * a + 32 * u4) * kWCols];
-          P[a] = u4 == 0 ? xx[a] * wv : fmaf(xx[a], wv, P[a]);
-        }
-      }
-      const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
-      sb[vs4 * cpr + cb + jj] = (q0 + q2) + (q1 + q3);
-    }
+  if (!ptx::mbar_wait_spin(wbar, 0u, kWaitTries)) {
+    set_status(p.status, HATA_ERR_TIMEOUT);
+    stat[ST_ABORT] = 1;
   }
   __syncthreads();
-  // 8 columns per byte of the code, stored straight into the code array of every
-  // CTA of the cluster (each byte has exactly one writer)
-  ptx::cluster_wait();  // every CTA of the cluster has started (arrive at kernel start)
+  // y = x . W_H[:, j] in the order of warp_dot128: lane l of that function is
+  // (residue s = l % 4, a = l / 4); its partial (u = 0 product, then FMAs for +32,
+  // +64, +96) and the butterfly levels 16, 8, 4 stay inside one residue, so thread
+  // (s, j) computes the residue sums S_s of column j for every vector, and the
+  // levels 2 and 1 give y = (S_0 + S_2) + (S_1 + S_3).  A warp takes one residue and
+  // 32 consecutive columns; the thread keeps its 32 W_H values in registers.
   {
-    const int nb8 = ncols / 8;
-    for (int e = tid; e < NV * nb8 * CS; e += kFThreads) {
-      const int c = e / (NV * nb8), vb = e % (NV * nb8), v = vb / nb8, jb = vb % nb8;
-      const float* sv = sb + v * 4 * cpr + jb * 8;
-      uint32_t byte = 0;
+    float* sb = reinterpret_cast<float*>(smem + S.D);  // [NV][4][R] residue sums (the scores' space, unused yet)
+    for (int it = tid; it < 4 * R; it += kFThreads) {
+      const int s = (it >> 5) & 3, j = (it >> 7) * 32 + (it & 31);
+      float wr[32];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float y = (sv[k] + sv[2 * cpr + k]) + (sv[cpr + k] + sv[3 * cpr + k]);
-        byte |= (y > 0.f ? 1u : 0u) << k;
+      for (int u4 = 0; u4 < 4; ++u4)
+#pragma unroll
+        for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = Wsm[(s + 4 * a + 32 * u4) * R + j];
+#pragma unroll 1
+      for (int v = 0; v < NV; ++v) {
+        const float* xs_ = xr + (v * 4 + s) * kXS;
+        float P[8];
+#pragma unroll
+        for (int u4 = 0; u4 < 4; ++u4) {
+          const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
+          const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
+          const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int a = 0; a < 8; ++a) P[a] = u4 == 0 ? xx[a] * wr[u4 * 8 + a] : fmaf(xx[a], wr[u4 * 8 + a], P[a]);
+        }
+        const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
+        sb[(v * 4 + s) * R + j] = (q0 + q2) + (q1 + q3);
       }
-      ptx::st_dsmem_u8(ptx::dsmem_addr(reinterpret_cast<uint8_t*>(qc) + v * NW * 4 + (j0 >> 3) + jb, c), byte);
+    }
+    __syncthreads();
+    for (int pi = warp; pi < NV * NW; pi += kNWarp) {  // one code word per warp item
+      const int v = pi / NW, jw = pi % NW, j = jw * 32 + lane;
+      const float* sv = sb + v * 4 * R;
+      const float y = (sv[j] + sv[2 * R + j]) + (sv[R + j] + sv[3 * R + j]);
+      const unsigned bits = __ballot_sync(0xffffffffu, y > 0.f);
+      if (lane == 0) qc[v * NW + jw] = bits;
     }
   }
-  ptx::cluster_sync();  // #1: every CTA holds all code bits
+  __syncthreads();  // codes ready; the residue sums are consumed
   if (rank == 0 && p.qcode_out && tid < G * NW) p.qcode_out[((size_t)b * p.Hq + (size_t)g * G) * NW + tid] = qc[tid];
   const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
   if (own_last && tid < NW) cu[(size_t)(L - 1) * NW + tid] = qc[G * NW + tid];
@@ -484,6 +469,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   __syncthreads();
   // bins [lo, hi) of the u16 cumulative histogram into slot `rank` of every CTA (8
   // bins per 16-byte store), with (lo, hi) in the header
+  ptx::cluster_wait();  // every CTA of the cluster has started (arrive at kernel start)
   {
     const int plo = stat[ST_LO], phi = stat[ST_HI];
     const int ng = (phi - plo) / 8;
@@ -503,7 +489,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       }
     }
   }
-  ptx::cluster_arrive_release();  // #2, completed by the threshold warp and after the logits (below)
+  ptx::cluster_arrive_release();  // #1, completed by the threshold warp and after the logits (below)
   const int Tc = stat[ST_SPEC];
   const bool scan_cands = Tc >= 0 && !stat[ST_ABORT];
 
@@ -598,10 +584,15 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     }
   };
   // Candidates in token order, without atomics: warp w owns a contiguous run of
-  // 8-score vectors; a first pass counts its hits, a second one writes them at the
-  // warp's offset, then the warp gathers their K and V rows.  Scores are below
-  // 2^15, so in each 16-bit half of (x + (0x7fff - Tc) * 0x10001) bit 15 is set
-  // exactly when that score exceeds Tc; halves past nmine are read as 0x7fff.
+  // 8-score vectors, lane l the vectors wv0 + 128 tr + 32 i + l (trip tr < 4, group
+  // i < 4).  One pass packs each lane's hit flags of a trip into one word and
+  // counts them; after the warps' totals are known, a second step places the hits
+  // at the warp's offset (a shuffle scan per group) and the warp gathers their K and
+  // V rows.  Scores are below 2^15, so in each 16-bit half of
+  // (x + (0x7fff - Tc) * 0x10001) bit 15 is set exactly when that score exceeds Tc;
+  // halves past nmine are read as 0x7fff.  Flag layout of group i: bit 4i + q for
+  // token 2q of the vector, bit 16 + 4i + q for token 2q + 1.
+  constexpr int MAXTRIP = 4;  // 4 trips x 128 vectors x 16 warps x 8 tokens >= kTokCap
   const int nvec = (nmine + 7) / 8;  // whole vectors inside tok_cap (a multiple of 16)
   const int nvw = (nvec + kNWarp - 1) / kNWarp;
   const int wv0 = min(nvec, warp * nvw), wv1 = min(nvec, wv0 + nvw);
@@ -619,26 +610,27 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     }
     return w4;
   };
-  auto hit_bits = [&](const uint4& w4, uint32_t (&x)[4]) {  // bit 15 / 31 of x[q]: score 2q / 2q+1 <= Tc
-    x[0] = ~(w4.x + addc) & 0x80008000u;
-    x[1] = ~(w4.y + addc) & 0x80008000u;
-    x[2] = ~(w4.z + addc) & 0x80008000u;
-    x[3] = ~(w4.w + addc) & 0x80008000u;
-  };
+  uint32_t Mt[MAXTRIP];
   {
     int c = 0;
-    if (scan_cands)
-      for (int e = wv0 + lane; e < wv1; e += 128) {  // four vectors per lane per trip, loads first
+#pragma unroll
+    for (int tr = 0; tr < MAXTRIP; ++tr) {
+      Mt[tr] = 0u;
+      if (scan_cands && wv0 + tr * 128 < wv1) {  // warp-uniform
         uint4 w4[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) w4[i] = load_vec(e + 32 * i);
+        for (int i = 0; i < 4; ++i) w4[i] = load_vec(wv0 + tr * 128 + 32 * i + lane);
+        uint32_t M = 0u;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          uint32_t x[4];
-          hit_bits(w4[i], x);
-          c += __popc(x[0]) + __popc(x[1]) + __popc(x[2]) + __popc(x[3]);
+          const uint32_t x0 = ~(w4[i].x + addc) & 0x80008000u, x1 = ~(w4[i].y + addc) & 0x80008000u;
+          const uint32_t x2 = ~(w4[i].z + addc) & 0x80008000u, x3 = ~(w4[i].w + addc) & 0x80008000u;
+          M |= ((x0 >> 15) | (x1 >> 14) | (x2 >> 13) | (x3 >> 12)) << (4 * i);
         }
+        Mt[tr] = M;
+        c += __popc(M);
       }
+    }
     c = __reduce_add_sync(0xffffffffu, c);
     if (lane == 0) warp_sums[warp] = c;
   }
@@ -653,33 +645,42 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int ncand = min(ncand_all, GB);  // <= want <= GB by construction
   if (scan_cands) {
     const int wstart = wbase;
-    const unsigned lm = (1u << lane) - 1u;
-    for (int e0 = wv0; e0 < wv1; e0 += 128) {  // warp-uniform trip count
-      uint4 w4[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w4[i] = load_vec(e0 + 32 * i + lane);
+    for (int tr = 0; tr < MAXTRIP; ++tr) {
+      if (__any_sync(0xffffffffu, Mt[tr] != 0u)) {
+        const uint32_t M = Mt[tr];
+        int cg[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t x[4];
-        hit_bits(w4[i], x);
-        const int ci = __popc(x[0]) + __popc(x[1]) + __popc(x[2]) + __popc(x[3]);  // <= 8
-        if (__ballot_sync(0xffffffffu, ci != 0) == 0u) continue;
-        const unsigned b0 = __ballot_sync(0xffffffffu, ci & 1), b1 = __ballot_sync(0xffffffffu, ci & 2),
-                       b2 = __ballot_sync(0xffffffffu, ci & 4), b3 = __ballot_sync(0xffffffffu, ci & 8);
-        int pos = wbase + __popc(b0 & lm) + 2 * __popc(b1 & lm) + 4 * __popc(b2 & lm) + 8 * __popc(b3 & lm);
-        wbase += __popc(b0) + 2 * __popc(b1) + 4 * __popc(b2) + 8 * __popc(b3);
-        const int tb = t0 + (e0 + 32 * i + lane) * 8;
+        for (int i = 0; i < 4; ++i) cg[i] = __popc(M & ((0xfu << (4 * i)) | (0xfu << (16 + 4 * i))));
+        // inclusive scans over the lanes of the four groups' counts, two per word
+        int s01 = cg[0] | (cg[1] << 16), s23 = cg[2] | (cg[3] << 16);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (x[q] & 0x8000u) {
-            if (pos < GB) cand[pos] = tb + 2 * q;
-            ++pos;
-          }
-          if (x[q] & 0x80000000u) {
-            if (pos < GB) cand[pos] = tb + 2 * q + 1;
-            ++pos;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y01 = __shfl_up_sync(0xffffffffu, s01, o), y23 = __shfl_up_sync(0xffffffffu, s23, o);
+          if (lane >= o) {
+            s01 += y01;
+            s23 += y23;
           }
         }
+        const int t01 = __shfl_sync(0xffffffffu, s01, 31), t23 = __shfl_sync(0xffffffffu, s23, 31);
+        const int tot[4] = {t01 & 0xffff, t01 >> 16, t23 & 0xffff, t23 >> 16};
+        const int inc[4] = {s01 & 0xffff, s01 >> 16, s23 & 0xffff, s23 >> 16};
+        if (M) {
+          int gbase = wbase;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            int pos = gbase + inc[i] - cg[i];
+            const int tb = t0 + (wv0 + tr * 128 + 32 * i + lane) * 8;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              if ((M >> ((k & 1) * 16 + 4 * i + (k >> 1))) & 1u) {
+                if (pos < GB) cand[pos] = tb + k;
+                ++pos;
+              }
+            gbase += tot[i];
+          }
+        }
+        wbase += tot[0] + tot[1] + tot[2] + tot[3];
       }
     }
     __syncwarp();
@@ -703,7 +704,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   // ---- 5. warp 0: unit threshold and the selected candidates; the other warps:
   //         the candidates' logits (as soon as their rows have landed) -----------
   if (warp == 0) {
-    ptx::cluster_wait();  // #2: every CTA holds every CTA's cumulative histogram range
+    ptx::cluster_wait();  // #1: every CTA holds every CTA's cumulative histogram range
     // T = the smallest score v whose unit total (sum of the CS cumulative counts)
     // is at least n; the total at the top bin is L >= n.  Rounds of a 32-way split
     // of [lo, hi], one probe per lane.  Source c sent bins [lo_c, hi_c): below
@@ -781,7 +782,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   } else {
     gather_wait();  // phase 0
     compute_logits(ncand, false, 1, kNWarp - 1);
-    ptx::cluster_wait();  // #2 (these warps' side)
+    ptx::cluster_wait();  // #1 (these warps' side)
   }
   if (warp == 0) gphase = 1;  // warp 0 did not wait on phase 0; the barrier below orders it after
   __syncthreads();
@@ -969,7 +970,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     const int owner = e / (2 * G), w = e % (2 * G);
     ptx::st_dsmem_f32(ptx::dsmem_addr(&mslot[rank * stride + w], owner), part[(w >> 1) * 4 + (w & 1)]);
   }
-  ptx::cluster_sync();  // #3: every CTA holds the partials of its columns
+  ptx::cluster_sync();  // #2: every CTA holds the partials of its columns
   for (int col = tid; col < mc; col += kFThreads) {
     const int e = rank * mc + col;
     if (e < G * D) {
@@ -1002,6 +1003,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     // give outstanding bulk copies one more bounded chance to land before exit
     for (int bi = 0; bi < kStages; ++bi)
       if (lastv[bi] >= 0) ptx::mbar_wait_bounded(&mbar[bi], (uint32_t)(lastv[bi] / kStages) & 1u, kWaitTries);
+    ptx::mbar_wait_bounded(&mbar[kMaxStages + 1], 0u, kWaitTries);  // the W_H copy
   }
 }
 
