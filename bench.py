@@ -17,6 +17,7 @@ Prints one JSON line.  --impl reference times the CPU oracle on this host
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -52,6 +53,31 @@ def algorithmic_bytes(wl, seq_lens) -> int:
         total += wl.n_kv_heads * (Lb * wl.hash_bits // 8 + 2 * min(wl.k, Lb) * wl.head_dim * e)
     total += 2 * wl.batch * wl.n_q_heads * wl.head_dim * e
     return total
+
+
+# Sources of the fused kernel: a recorded DRAM traffic figure applies only to them.
+KERNEL_SOURCES = ["hata_step.cu", "hata_common.cuh", "hata_ptx.cuh", "hata_kernels.cuh"]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch of the fused kernel from the committed ncu record,
+    or None when there is no record for this workload or the kernel changed since."""
+    rec = os.path.join(ROOT, "profiles", f"fused_step_{workload_name}_traffic.txt")
+    if not os.path.exists(rec):
+        return None
+    fields = {}
+    for line in open(rec):
+        if line.startswith("#") or ":" not in line:
+            continue
+        k, v = line.split(":", 1)
+        fields[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "hash_aware_top_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if fields.get("workload") != workload_name or fields.get("kernel_source_sha256") != h.hexdigest():
+        return None
+    return int(fields["dram_bytes_per_launch"])
 
 
 def peak_hbm():
@@ -419,7 +445,7 @@ def run_gpu(args, wl):
             "peak_kind": peak_kind,
             "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": None,
+            "traffic": recorded_traffic(wl.name),
             "algorithmic_bytes_per_step": step_bytes,
         },
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
