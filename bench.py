@@ -56,7 +56,7 @@ def algorithmic_bytes(wl, seq_lens) -> int:
 
 
 # Sources of the fused kernel: a recorded DRAM traffic figure applies only to them.
-KERNEL_SOURCES = ["hata_step.cu", "hata_common.cuh", "hata_ptx.cuh", "hata_kernels.cuh"]
+KERNEL_SOURCES = ["hata_step.cu", "hata_common.cuh", "hata_ptx.cuh"]
 
 
 def recorded_traffic(workload_name):
@@ -418,8 +418,48 @@ def run_gpu(args, wl):
         e2e_s = float(t.item())
     e2e_value = world * e2e_steps / e2e_s
 
+    # the dense flash-decode baseline on the same layer buffers (the comparison the pages report)
+    dense = None
+    if wl.dtype == "bf16" and wl.n_q_heads // wl.n_kv_heads <= 8:
+        dws = torch.zeros(H.hata_dense_workspace_size(dims), dtype=torch.uint8, device=dev)
+
+        def dense_step(i):
+            L = layers[i % R]
+            H.hata_dense_decode(dims, L["q"], L["K"], L["V"], L["lens"], 0.0, L["out"], dws, stream)
+
+        d_steps = min(args.steps, 2000)
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                dense_step(i)
+        torch.cuda.synchronize()
+        gd = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gd, stream=stream):
+            for i in range(min(d_steps, GRAPH_CHUNK)):
+                dense_step(i)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            gd.replay()  # warm-up
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            reps = max(1, d_steps // min(d_steps, GRAPH_CHUNK))
+            for _ in range(reps):
+                gd.replay()
+            e1.record(stream)
+            e1.synchronize()
+        d_ms = e0.elapsed_time(e1) / (reps * min(d_steps, GRAPH_CHUNK))
+        d_bytes = sum(2 * int(Lb) * wl.n_kv_heads * wl.head_dim * 2 for Lb in inp["seq_lens"]) + \
+            2 * wl.batch * wl.n_q_heads * wl.head_dim * 2
+        dense = {"kernel": "hata_dense_decode (dense flash-decode, bf16 tensor-core tiles)",
+                 "us_per_step": d_ms * 1e3, "bytes_per_step": d_bytes,
+                 "achieved_gbs": d_bytes / (d_ms * 1e-3) / 1e9,
+                 "hata_speedup": d_ms / ms_per_step}
+        del gd
+
     peak, peak_kind = peak_hbm()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    if dense is not None:
+        dense["frac_of_peak"] = dense["achieved_gbs"] / peak
     line = {
         "metric": METRIC,
         "value": value,
@@ -451,6 +491,7 @@ def run_gpu(args, wl):
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
+        "dense_baseline": dense,
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

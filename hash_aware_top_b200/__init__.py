@@ -36,6 +36,8 @@ __all__ = [
     "hata_status_string",
     "hata_version",
     "hata_decode_step_kernel_count",
+    "hata_dense_workspace_size",
+    "hata_dense_decode",
     "HATA_F32",
     "HATA_BF16",
     "EXPORTED_SYMBOLS",
@@ -60,6 +62,8 @@ EXPORTED_SYMBOLS = (
     "hata_version",
     "hata_decode_step_kernel_count",
     "hata_topk_noalloc",
+    "hata_dense_workspace_size",
+    "hata_dense_decode",
 )
 
 
@@ -113,6 +117,8 @@ def _load():
         "hata_version": (I, []),
         "hata_decode_step_kernel_count": (I, [DP, I]),
         "hata_topk_noalloc": (I, [DP, P, P, I, P, P, P]),
+        "hata_dense_workspace_size": (I, [DP, ctypes.POINTER(S)]),
+        "hata_dense_decode": (I, [DP, P, P, P, P, F, P, P, S, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -261,6 +267,26 @@ def hata_sparse_decode(dims: Dims, q, K, V, idx, k, scale, out, ws, stream=None)
             _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_sparse_decode")
+
+
+def hata_dense_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hata_dense_workspace_size(ctypes.byref(dims), ctypes.byref(n)), "hata_dense_workspace_size")
+    return int(n.value)
+
+
+def hata_dense_decode(dims: Dims, q, K, V, seq_lens, scale, out, ws, stream=None):
+    d = dims
+    kv = (d.batch, d.n_kv_heads, d.max_seq, d.head_dim)
+    _check(
+        lib.hata_dense_decode(
+            ctypes.byref(d),
+            _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(K, "K", kv, d.torch_dtype), _ptr(V, "V", kv, d.torch_dtype),
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32, optional=True), float(scale),
+            _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
+        "hata_dense_decode")
 
 
 def hata_decode_step(dims: Dims, q, K, V, W_H, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws,

@@ -120,6 +120,29 @@ hata_status_t hata_sparse_decode(const hata_dims_t* dims, const void* q, const v
                                           static_cast<cudaStream_t>(stream)));
 }
 
+hata_status_t hata_dense_workspace_size(const hata_dims_t* dims, size_t* bytes) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!bytes) return HATA_ERR_INVALID_ARG;
+  *bytes = dense_ws_bytes(*dims);
+  return HATA_OK;
+}
+
+hata_status_t hata_dense_decode(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                const int32_t* seq_lens, float scale, void* out, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (dims->dtype != HATA_BF16 || dims->n_q_heads / dims->n_kv_heads > 8) return HATA_ERR_UNSUPPORTED;
+  if (!q || !K || !V || !out) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return HATA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return HATA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < dense_ws_bytes(*dims)) return HATA_ERR_WORKSPACE;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)dims->head_dim);
+  return cuda_status(launch_dense_decode(*dims, q, K, V, seq_lens, scale, out, static_cast<char*>(workspace),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
 hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const void* K, const void* V,
                                const float* W_H, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
                                void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,

@@ -182,6 +182,26 @@ HATA_API hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, 
                                size_t workspace_bytes, void* stream);
 
 /*
+ * Dense flash-decode, the comparison baseline: exact attention of every query
+ * head over all cached tokens (the dense attention that the "HATA" paper notes'
+ * 实验 section times HATA against, at 32K-128K context):
+ *     out[b][h] = sum_{t < L_b} softmax_t(scale * q[b][h] . K[b][g][t]) V[b][g][t]
+ * with g = h / G and L_b = min(seq_lens[b], max_seq) (seq_lens NULL: max_seq).
+ * Same layouts as hata_decode_step; bf16 only, G <= 8, d = 128 (else
+ * HATA_ERR_UNSUPPORTED).  Logits and P.V run on tensor-core tiles (bf16 in,
+ * fp32 accumulate, probabilities rounded to bf16 for P.V), so results agree
+ * with exact attention within the bf16 tolerance.  The workspace
+ * (hata_dense_workspace_size bytes, 16-byte aligned) holds per-split partials
+ * and arrival counters; zero it once with hata_workspace_init before the first
+ * call; every call leaves the counters at zero.  L_b > max_seq is clamped and
+ * flagged in the workspace's status word (hata_read_device_status).
+ */
+HATA_API hata_status_t hata_dense_workspace_size(const hata_dims_t* dims, size_t* bytes);
+HATA_API hata_status_t hata_dense_decode(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                         const int32_t* seq_lens, float scale, void* out, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
+/*
  * hata_topk without a workspace, for callers that cannot allocate device memory
  * (no counterpart on the pages: it only changes where scratch lives).  Same
  * inputs, outputs and results as hata_topk.  Its scratch is one 8 MiB array of
