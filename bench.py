@@ -456,8 +456,31 @@ def run_gpu(args, wl):
                  "hata_speedup": d_ms / ms_per_step}
         del gd
 
+    # prefill encode (hata_encode_append over every cached key of every layer buffer)
+    pre_reps = max(2, min(R, 8))
+    with torch.cuda.stream(stream):
+        H.hata_encode_append(dims, layers[0]["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, layers[0]["lens"],
+                             layers[0]["W"], layers[0]["codes"], wl.max_seq, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(pre_reps):
+            L = layers[i % R]
+            H.hata_encode_append(dims, L["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L["lens"], L["W"], L["codes"],
+                                 wl.max_seq, stream)
+        e1.record(stream)
+        e1.synchronize()
+    pre_ms = e0.elapsed_time(e1) / pre_reps
+    n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
+    pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + wl.hash_bits // 8)
+    prefill = {"kernel": "hata_encode_append (prefill form)", "us_per_call": pre_ms * 1e3, "keys": n_keys,
+               "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
+               "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
+               "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
+
     peak, peak_kind = peak_hbm()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    prefill["frac_of_peak"] = prefill["achieved_gbs"] / peak
     if dense is not None:
         dense["frac_of_peak"] = dense["achieved_gbs"] / peak
     line = {
@@ -492,6 +515,7 @@ def run_gpu(args, wl):
                 "steps": e2e_steps},
         "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
         "dense_baseline": dense,
+        "prefill_encode": prefill,
         "clocks": sampler.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

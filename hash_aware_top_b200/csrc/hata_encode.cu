@@ -9,7 +9,9 @@
 //     and its 32 columns of W_H (transposed) in shared memory and every (row,
 //     column) projection is one warp_dot128 -- the same arithmetic as the fused
 //     decode step, so both paths produce identical codes.
-//   * prefill form: each CTA owns one (batch, KV group) and a tile of 32 rows;
+//   * prefill form, bf16 keys and r <= 128: the tensor-core kernel of
+//     hata_encode_mma.cu (W_H split in three bf16 parts, fp32 accumulation);
+//   * prefill form otherwise: each CTA owns one (batch, KV group) and a tile of 32 rows;
 //     thread (slice s, column j) accumulates y_j for rows s, s + NS, ... with
 //     fp32 FMAs in ascending i, reading W_H[g][i][j] coalesced along j; the sign
 //     bits of 32 consecutive columns are one warp ballot, i.e. one packed word.
@@ -136,6 +138,10 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
     encode_decode_kernel<T><<<grid, kEncThreads, 0, st>>>(static_cast<const T*>(x), x_heads, x_len, n_tok, seq_end,
                                                           W, codes, codes_len, hpg, d.hash_bits);
     return cudaGetLastError();
+  }
+  if constexpr (sizeof(T) == 2) {  // bf16 keys: the tensor-core prefill (r <= 128)
+    const cudaError_t e = launch_encode_mma(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
+    if (e != cudaErrorNotSupported) return e;
   }
   const long long rows = (long long)hpg * n_tok;
   dim3 grid((unsigned)((rows + kEncRows - 1) / kEncRows), d.n_kv_heads, d.batch);

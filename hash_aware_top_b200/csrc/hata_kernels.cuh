@@ -24,6 +24,9 @@ cudaError_t launch_sparse_decode(const hata_dims_t& d, const WsLayout& L, const 
 bool fused_step_applies(const hata_dims_t& d, int k);
 // Fused decode step: bytes of workspace its plan needs (0 if it does not apply)
 size_t fused_step_ws_bytes(const hata_dims_t& d, int k);
+cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
+                              const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                              cudaStream_t stream);
 size_t dense_ws_bytes(const hata_dims_t& d);
 cudaError_t launch_dense_decode(const hata_dims_t& d, const void* q, const void* K, const void* V,
                                 const int32_t* seq_lens, float scale, void* out, char* ws, cudaStream_t stream);
