@@ -14,7 +14,7 @@
 // Layout of the work: W_H^T is the A operand (rows = 16 output columns, held in
 // registers for the whole kernel: 8 k-steps x 3 parts x 4 registers), the keys
 // are B (8 keys per n-tile, read from a padded shared-memory tile of 64 keys
-// filled by cp.async, double-buffered), y^T accumulates in fp32.  Warp w owns
+// filled by cp.async, four tiles in flight), y^T accumulates in fp32.  Warp w owns
 // 16 columns and a share of the tile's keys; the sign bits of a (key, 16
 // columns) pair are gathered with four ballots and written as one u16, and the
 // tile's codes leave as whole words.  CTAs are persistent per (batch, head).
@@ -29,6 +29,8 @@ namespace {
 constexpr int kEmThreads = 256;
 constexpr int kEmTile = 64;                  // keys per tile
 constexpr int kEmRowB = kHeadDim * 2 + 16;   // bytes per staged key row (padded)
+constexpr int kEmStages = 4;                 // key tiles in flight per CTA
+constexpr int kEmSmem = kEmStages * kEmTile * kEmRowB;
 
 __device__ __forceinline__ void em_cp_async16(void* smem, const void* gmem) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"((unsigned)__cvta_generic_to_shared(smem)),
@@ -72,7 +74,7 @@ __global__ void __launch_bounds__(kEmThreads, 2)
   constexpr int CPW = kEmTile / 8 / KG;  // 8-key chunks per warp per tile
   constexpr int NWd = R / 32;
   static_assert(NCT <= 8 && 8 % NCT == 0, "r in {16..128}");
-  __shared__ __align__(16) unsigned char xs[2][kEmTile * kEmRowB];
+  extern __shared__ __align__(128) unsigned char xsm[];  // kEmStages tiles of kEmTile padded key rows
   __shared__ uint16_t cs[kEmTile][NCT];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, gq = lane >> 2, cq = lane & 3;
@@ -111,23 +113,29 @@ __global__ void __launch_bounds__(kEmThreads, 2)
     const int r0 = ts + tile * kEmTile, nr = min(kEmTile, te - r0);
     for (int e = tid; e < kEmTile * 16; e += kEmThreads) {
       const int row = e >> 4, pc = e & 15;
-      unsigned char* dst = &xs[st][row * kEmRowB + pc * 16];
+      unsigned char* dst = xsm + st * (kEmTile * kEmRowB) + row * kEmRowB + pc * 16;
       if (row < nr) em_cp_async16(dst, xb + (size_t)(r0 + row) * D + pc * 8);
       else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
     }
     em_commit();
   };
-  int st = 0;
-  if ((int)blockIdx.x < ntile) load(blockIdx.x, 0);
-  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x, st ^= 1) {
-    if (tile + (int)gridDim.x < ntile) {
-      load(tile + gridDim.x, st ^ 1);
-      em_wait<1>();
-    } else {
-      em_wait<0>();
-    }
+  // the CTA's tiles are blockIdx.x + i * gridDim.x; tile i goes to stage i % kEmStages,
+  // with kEmStages - 1 tiles in flight ahead of the one being encoded (one cp.async
+  // group per tile; empty groups past the end keep the count uniform)
+#pragma unroll
+  for (int i = 0; i < kEmStages - 1; ++i) {
+    const int tl = blockIdx.x + i * gridDim.x;
+    if (tl < ntile) load(tl, i);
+    else em_commit();
+  }
+  int i = 0;
+  for (int tile = blockIdx.x; tile < ntile; tile += gridDim.x, ++i) {
+    const int ahead = tile + (kEmStages - 1) * gridDim.x;
+    if (ahead < ntile) load(ahead, (i + kEmStages - 1) % kEmStages);
+    else em_commit();
+    em_wait<kEmStages - 1>();
     __syncthreads();  // this tile's keys have landed; cs is free
-    const unsigned char* xt = xs[st];
+    const unsigned char* xt = xsm + (i % kEmStages) * (kEmTile * kEmRowB);
 #pragma unroll
     for (int ch = 0; ch < CPW; ++ch) {
       const int n0 = (kg * CPW + ch) * 8;
@@ -172,17 +180,21 @@ cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, 
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms < 1) sms = 1;
+    cudaFuncSetAttribute(encode_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+    cudaFuncSetAttribute(encode_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+    cudaFuncSetAttribute(encode_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
   }
   const int hpg = x_heads / d.n_kv_heads;
   const long long heads = (long long)d.batch * x_heads;
   const long long tiles = (n_tok + kEmTile - 1) / kEmTile;
-  const unsigned per_head = (unsigned)std::max<long long>(1, std::min<long long>(tiles, (2LL * sms + heads - 1) / heads));
+  // one wave: two CTAs per SM (registers), split evenly over the (batch, head) pairs
+  const unsigned per_head = (unsigned)std::max<long long>(1, std::min<long long>(tiles, (2LL * sms) / heads));
   dim3 grid(per_head, (unsigned)heads);
   const __nv_bfloat16* xp = static_cast<const __nv_bfloat16*>(x);
   switch (d.hash_bits) {
-    case 32: encode_mma_kernel<32><<<grid, kEmThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
-    case 64: encode_mma_kernel<64><<<grid, kEmThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
-    case 128: encode_mma_kernel<128><<<grid, kEmThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 32: encode_mma_kernel<32><<<grid, kEmThreads, kEmSmem, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 64: encode_mma_kernel<64><<<grid, kEmThreads, kEmSmem, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
+    case 128: encode_mma_kernel<128><<<grid, kEmThreads, kEmSmem, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
     default: return cudaErrorNotSupported;
   }
   return cudaGetLastError();
