@@ -420,6 +420,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     __syncthreads();
     // the ring (or global memory) may have held the old code of slot L - 1: rescore it
     // with the appended key code and move its histogram count
+    if (tid < 8 && nmine + tid < ((nmine + 7) & ~7)) Ds[nmine + tid] = (uint16_t)0x7fff;  // whole 8-score vectors
     if (own_last && tid == 0) {
       const int d_new = gq.score(keyc, qc, G), d_old = Ds[L - 1 - t0];
       if (d_new != d_old) {
@@ -585,52 +586,37 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   };
   // Candidates in token order, without atomics: warp w owns a contiguous run of
   // 8-score vectors, lane l the vectors wv0 + 128 tr + 32 i + l (trip tr < 4, group
-  // i < 4).  One pass packs each lane's hit flags of a trip into one word and
-  // counts them; after the warps' totals are known, a second step places the hits
-  // at the warp's offset (a shuffle scan per group) and the warp gathers their K and
-  // V rows.  Scores are below 2^15, so in each 16-bit half of
+  // i < 4).  trip_flags packs the lane's hit flags of a trip into one word, byte i
+  // for group i with bit k for token k of the vector.  Pass 1 counts them; after the
+  // warps' totals are known, pass 2 recomputes the flags, places the hits at the
+  // warp's offset (a shuffle scan per group) and the warp gathers their K and V
+  // rows.  Scores are below 2^15, so in each 16-bit half of
   // (x + (0x7fff - Tc) * 0x10001) bit 15 is set exactly when that score exceeds Tc;
-  // halves past nmine are read as 0x7fff.  Flag layout of group i: bit 4i + q for
-  // token 2q of the vector, bit 16 + 4i + q for token 2q + 1.
-  constexpr int MAXTRIP = 4;  // 4 trips x 128 vectors x 16 warps x 8 tokens >= kTokCap
+  // the scores past nmine read 0x7fff (set after the scan).
   const int nvec = (nmine + 7) / 8;  // whole vectors inside tok_cap (a multiple of 16)
   const int nvw = (nvec + kNWarp - 1) / kNWarp;
   const int wv0 = min(nvec, warp * nvw), wv1 = min(nvec, wv0 + nvw);
+  const int ntrip = scan_cands ? (wv1 - wv0 + 127) / 128 : 0;  // warp-uniform; <= 4 since tok_cap <= kTokCap
   const uint32_t addc = (uint32_t)(0x7fff - max(Tc, 0)) * 0x10001u;
-  auto load_vec = [&](int e) -> uint4 {
-    uint4 w4 = reinterpret_cast<const uint4*>(Ds)[min(e, max(nvec - 1, 0))];
-    const int valid = e < wv1 ? nmine - e * 8 : 0;
-    if (valid < 8) {
-      uint32_t* wq = reinterpret_cast<uint32_t*>(&w4);
+  auto trip_flags = [&](int tr) -> uint32_t {
+    uint32_t M = 0u;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (2 * q >= valid) wq[q] = (wq[q] & 0xffff0000u) | 0x7fffu;
-        if (2 * q + 1 >= valid) wq[q] = (wq[q] & 0x0000ffffu) | 0x7fff0000u;
+    for (int i = 0; i < 4; ++i) {
+      const int e = wv0 + tr * 128 + 32 * i + lane;
+      if (e < wv1) {
+        const uint4 w4 = reinterpret_cast<const uint4*>(Ds)[e];
+        // token 2j's flag to bit 2j, token 2j + 1's to bit 16 + 2j, then folded to 2j + 1
+        const uint32_t y = ((~(w4.x + addc) & 0x80008000u) >> 15) | ((~(w4.y + addc) & 0x80008000u) >> 13) |
+                           ((~(w4.z + addc) & 0x80008000u) >> 11) | ((~(w4.w + addc) & 0x80008000u) >> 9);
+        M |= ((y | (y >> 15)) & 0xffu) << (8 * i);
       }
     }
-    return w4;
+    return M;
   };
-  uint32_t Mt[MAXTRIP];
   {
     int c = 0;
-#pragma unroll
-    for (int tr = 0; tr < MAXTRIP; ++tr) {
-      Mt[tr] = 0u;
-      if (scan_cands && wv0 + tr * 128 < wv1) {  // warp-uniform
-        uint4 w4[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) w4[i] = load_vec(wv0 + tr * 128 + 32 * i + lane);
-        uint32_t M = 0u;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t x0 = ~(w4[i].x + addc) & 0x80008000u, x1 = ~(w4[i].y + addc) & 0x80008000u;
-          const uint32_t x2 = ~(w4[i].z + addc) & 0x80008000u, x3 = ~(w4[i].w + addc) & 0x80008000u;
-          M |= ((x0 >> 15) | (x1 >> 14) | (x2 >> 13) | (x3 >> 12)) << (4 * i);
-        }
-        Mt[tr] = M;
-        c += __popc(M);
-      }
-    }
+#pragma unroll 1
+    for (int tr = 0; tr < ntrip; ++tr) c += __popc(trip_flags(tr));
     c = __reduce_add_sync(0xffffffffu, c);
     if (lane == 0) warp_sums[warp] = c;
   }
@@ -643,17 +629,16 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     ncand_all += x;
   }
   const int ncand = min(ncand_all, GB);  // <= want <= GB by construction
-  if (scan_cands) {
+  if (ntrip > 0) {
     const int wstart = wbase;
-#pragma unroll
-    for (int tr = 0; tr < MAXTRIP; ++tr) {
-      if (__any_sync(0xffffffffu, Mt[tr] != 0u)) {
-        const uint32_t M = Mt[tr];
-        int cg[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) cg[i] = __popc(M & ((0xfu << (4 * i)) | (0xfu << (16 + 4 * i))));
+#pragma unroll 1
+    for (int tr = 0; tr < ntrip; ++tr) {
+      const uint32_t M = trip_flags(tr);
+      if (__any_sync(0xffffffffu, M != 0u)) {
         // inclusive scans over the lanes of the four groups' counts, two per word
-        int s01 = cg[0] | (cg[1] << 16), s23 = cg[2] | (cg[3] << 16);
+        int s01 = __popc(M & 0xffu) | (__popc(M & 0xff00u) << 16);
+        int s23 = __popc(M & 0xff0000u) | (__popc(M & 0xff000000u) << 16);
+        const int c01 = s01, c23 = s23;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y01 = __shfl_up_sync(0xffffffffu, s01, o), y23 = __shfl_up_sync(0xffffffffu, s23, o);
@@ -663,24 +648,27 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
           }
         }
         const int t01 = __shfl_sync(0xffffffffu, s01, 31), t23 = __shfl_sync(0xffffffffu, s23, 31);
-        const int tot[4] = {t01 & 0xffff, t01 >> 16, t23 & 0xffff, t23 >> 16};
-        const int inc[4] = {s01 & 0xffff, s01 >> 16, s23 & 0xffff, s23 >> 16};
-        if (M) {
-          int gbase = wbase;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            int pos = gbase + inc[i] - cg[i];
-            const int tb = t0 + (wv0 + tr * 128 + 32 * i + lane) * 8;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              if ((M >> ((k & 1) * 16 + 4 * i + (k >> 1))) & 1u) {
-                if (pos < GB) cand[pos] = tb + k;
-                ++pos;
-              }
-            gbase += tot[i];
+        // exclusive start of each group's hits of this lane, in token order
+        const int g0 = wbase + (s01 & 0xffff) - (c01 & 0xffff);
+        const int g1 = wbase + (t01 & 0xffff) + (s01 >> 16) - (c01 >> 16);
+        const int g2 = wbase + (t01 & 0xffff) + (t01 >> 16) + (s23 & 0xffff) - (c23 & 0xffff);
+        const int g3 = wbase + (t01 & 0xffff) + (t01 >> 16) + (t23 & 0xffff) + (s23 >> 16) - (c23 >> 16);
+        const int tb = t0 + (wv0 + tr * 128 + lane) * 8;
+        // hits of the lane, group by group, ascending token within a group
+        uint32_t mm = M;
+        int gi = 0, pos = g0;
+        while (mm) {
+          const int bit = __ffs(mm) - 1;
+          mm &= mm - 1u;
+          const int i = bit >> 3;
+          if (i != gi) {
+            gi = i;
+            pos = i == 1 ? g1 : (i == 2 ? g2 : g3);
           }
+          if (pos < GB) cand[pos] = tb + 256 * i + (bit & 7);
+          ++pos;
         }
-        wbase += tot[0] + tot[1] + tot[2] + tot[3];
+        wbase += (t01 & 0xffff) + (t01 >> 16) + (t23 & 0xffff) + (t23 >> 16);
       }
     }
     __syncwarp();
