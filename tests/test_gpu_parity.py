@@ -246,6 +246,11 @@ STEP_CASES = {
                                   seq_len_range=(15001, 30000)),
     "r64_g2": Workload("r64_g2", 2, 4, 2, 128, 5000, 64, 300, "f32"),
     "r256_g8": Workload("r256_g8", 1, 8, 1, 128, 5000, 256, 128, "bf16"),
+    # longer caches with few units, a budget far above a CTA's share, narrow fp32 codes
+    "llama_shape_20k": Workload("llama_shape_20k", 1, 32, 8, 128, 20000, 128, 512, "bf16"),
+    "ragged_24k": Workload("ragged_24k", 2, 16, 4, 128, 24000, 128, 700, "bf16", seq_len_range=(9000, 24000)),
+    "big_k_20k": Workload("big_k_20k", 1, 8, 2, 128, 20000, 128, 4096, "bf16"),
+    "r32_f32_17k": Workload("r32_f32_17k", 1, 8, 2, 128, 17000, 32, 500, "f32", seq_len_range=(16500, 17000)),
 }
 
 
