@@ -32,6 +32,7 @@ __all__ = [
     "hata_topk_noalloc",
     "hata_sparse_decode",
     "hata_decode_step",
+    "hata_decode_step_qk",
     "hata_read_device_status",
     "hata_status_string",
     "hata_version",
@@ -57,6 +58,7 @@ EXPORTED_SYMBOLS = (
     "hata_topk",
     "hata_sparse_decode",
     "hata_decode_step",
+    "hata_decode_step_qk",
     "hata_read_device_status",
     "hata_status_string",
     "hata_version",
@@ -112,6 +114,7 @@ def _load():
         "hata_topk": (I, [DP, P, P, I, P, P, P, S, P]),
         "hata_sparse_decode": (I, [DP, P, P, P, P, I, F, P, P, S, P]),
         "hata_decode_step": (I, [DP, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
+        "hata_decode_step_qk": (I, [DP, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
         "hata_read_device_status": (I, [P, P, ctypes.POINTER(I)]),
         "hata_status_string": (ctypes.c_char_p, [I]),
         "hata_version": (I, []),
@@ -306,6 +309,27 @@ def hata_decode_step(dims: Dims, q, K, V, W_H, codes, seq_lens, k, scale, out, q
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step")
+
+
+def hata_decode_step_qk(dims: Dims, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws,
+                        stream=None):
+    """hata_decode_step with separate query and key encoders (the cache holds codes made with W_k)."""
+    d = dims
+    kv = (d.batch, d.n_kv_heads, d.max_seq, d.head_dim)
+    wshape = (d.n_kv_heads, d.head_dim, d.hash_bits)
+    _check(
+        lib.hata_decode_step_qk(
+            ctypes.byref(d),
+            _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(K, "K", kv, d.torch_dtype), _ptr(V, "V", kv, d.torch_dtype),
+            _ptr(W_q, "W_q", wshape, torch.float32), _ptr(W_k, "W_k", wshape, torch.float32),
+            _ptr(codes, "codes", (d.batch, d.n_kv_heads, d.max_seq, d.words), _codes_dtype(codes)),
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k), float(scale),
+            _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(qcode_out, "qcode_out", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode_out), optional=True),
+            _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
+            _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
+        "hata_decode_step_qk")
 
 
 def hata_read_device_status(ws, stream=None) -> int:

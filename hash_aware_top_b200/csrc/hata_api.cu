@@ -143,14 +143,15 @@ hata_status_t hata_dense_decode(const hata_dims_t* dims, const void* q, const vo
                                          static_cast<cudaStream_t>(stream)));
 }
 
-hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const void* K, const void* V,
-                               const float* W_H, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
-                               void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
-                               size_t workspace_bytes, void* stream) {
+hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                  const float* W_q, const float* W_k, uint32_t* codes, const int32_t* seq_lens, int k,
+                                  float scale, void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
   hata_status_t s = check_dims(dims);
   if (s != HATA_OK) return s;
-  if (!q || !K || !V || !W_H || !codes || !seq_lens || !out || k < 1) return HATA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(W_H) || !aligned16(codes) || !aligned16(out))
+  if (!q || !K || !V || !W_q || !W_k || !codes || !seq_lens || !out || k < 1) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(W_q) || !aligned16(W_k) || !aligned16(codes) ||
+      !aligned16(out))
     return HATA_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return HATA_ERR_INVALID_ARG;
   WsLayout L;
@@ -159,7 +160,8 @@ hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const voi
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
-  cudaError_t e = launch_fused_step(*dims, L, q, K, V, W_H, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws, st);
+  cudaError_t e =
+      launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws, st);
   if (e != cudaErrorNotSupported) return cuda_status(e);
 
   // Chain of the granular kernels (shapes the fused kernel does not cover).
@@ -167,12 +169,20 @@ hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const voi
   uint32_t* qc = qcode_out ? qcode_out : reinterpret_cast<uint32_t*>(ws + L.qcode);
   int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   int32_t* sc = reinterpret_cast<int32_t*>(ws + L.scores);
-  if ((e = launch_encode(d, q, d.n_q_heads, 1, 1, nullptr, W_H, qc, 1, st)) != cudaSuccess) return cuda_status(e);
-  if ((e = launch_encode(d, K, d.n_kv_heads, d.max_seq, 1, seq_lens, W_H, codes, d.max_seq, st)) != cudaSuccess)
+  if ((e = launch_encode(d, q, d.n_q_heads, 1, 1, nullptr, W_q, qc, 1, st)) != cudaSuccess) return cuda_status(e);
+  if ((e = launch_encode(d, K, d.n_kv_heads, d.max_seq, 1, seq_lens, W_k, codes, d.max_seq, st)) != cudaSuccess)
     return cuda_status(e);
   if ((e = launch_hamming(d, qc, codes, seq_lens, sc, st)) != cudaSuccess) return cuda_status(e);
   if ((e = launch_topk(d, L, sc, seq_lens, k, ix, nullptr, ws, st)) != cudaSuccess) return cuda_status(e);
   return cuda_status(launch_sparse_decode(d, L, q, K, V, ix, k, scale, out, ws, st));
+}
+
+hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                               const float* W_H, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
+                               void* out, uint32_t* qcode_out, int32_t* idx_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  return hata_decode_step_qk(dims, q, K, V, W_H, W_H, codes, seq_lens, k, scale, out, qcode_out, idx_out, workspace,
+                             workspace_bytes, stream);
 }
 
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {

@@ -68,6 +68,7 @@ struct FusedParams {
   const void* K;
   const void* V;
   const float* W;
+  const float* Wk;  // separate key encoder [Hkv][d][r] (HashAttention form), or null: W encodes keys too
   uint32_t* codes;
   const int32_t* seq_lens;
   void* out;
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int nmine = t1 - t0;
   const int nst = (nmine + ST - 1) / ST;
   uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;
+  const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;  // this CTA appends the new key's code
   const uint64_t pol_stream = ptx::policy_evict_first();
   auto issue = [&](int s) {
     const int ts = t0 + s * ST, nt = min(ST, t1 - ts);
@@ -314,6 +316,23 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   // 32 consecutive columns; the thread keeps its 32 W_H values in registers.
   {
     float* sb = reinterpret_cast<float*>(smem + S.D);  // [NV][4][R] residue sums (the scores' space, unused yet)
+    // with a separate key encoder only the G queries use the shared-memory W_H; the
+    // CTA that appends the key encodes it below from W_k in global memory
+    const int nv_w = p.Wk ? G : NV;
+    auto residue_sums = [&](const float (&wr)[32], int v, int s, int j) {
+      const float* xs_ = xr + (v * 4 + s) * kXS;
+      float P[8];
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
+        const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
+        const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int a = 0; a < 8; ++a) P[a] = u4 == 0 ? xx[a] * wr[u4 * 8 + a] : fmaf(xx[a], wr[u4 * 8 + a], P[a]);
+      }
+      const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
+      sb[(v * 4 + s) * R + j] = (q0 + q2) + (q1 + q3);
+    };
     for (int it = tid; it < 4 * R; it += kFThreads) {
       const int s = (it >> 5) & 3, j = (it >> 7) * 32 + (it & 31);
       float wr[32];
@@ -322,19 +341,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
 #pragma unroll
         for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = Wsm[(s + 4 * a + 32 * u4) * R + j];
 #pragma unroll 1
-      for (int v = 0; v < NV; ++v) {
-        const float* xs_ = xr + (v * 4 + s) * kXS;
-        float P[8];
+      for (int v = 0; v < nv_w; ++v) residue_sums(wr, v, s, j);
+    }
+    if (p.Wk && own_last) {  // block-uniform
+      const float* Wkg = p.Wk + (size_t)g * D * R;
+      for (int it = tid; it < 4 * R; it += kFThreads) {
+        const int s = (it >> 5) & 3, j = (it >> 7) * 32 + (it & 31);
+        float wr[32];
 #pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
-          const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
-          const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        for (int u4 = 0; u4 < 4; ++u4)
 #pragma unroll
-          for (int a = 0; a < 8; ++a) P[a] = u4 == 0 ? xx[a] * wr[u4 * 8 + a] : fmaf(xx[a], wr[u4 * 8 + a], P[a]);
-        }
-        const float q0 = P[0] + P[4], q1 = P[1] + P[5], q2 = P[2] + P[6], q3 = P[3] + P[7];
-        sb[(v * 4 + s) * R + j] = (q0 + q2) + (q1 + q3);
+          for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = __ldg(Wkg + (size_t)(s + 4 * a + 32 * u4) * R + j);
+        residue_sums(wr, G, s, j);
       }
     }
     __syncthreads();
@@ -348,7 +366,6 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   __syncthreads();  // codes ready; the residue sums are consumed
   if (rank == 0 && p.qcode_out && tid < G * NW) p.qcode_out[((size_t)b * p.Hq + (size_t)g * G) * NW + tid] = qc[tid];
-  const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
   if (own_last && tid < NW) cu[(size_t)(L - 1) * NW + tid] = qc[G * NW + tid];
   // ---- 3. scan: scores + histogram; each warp releases ring stages on its own ---
   {
@@ -1217,8 +1234,9 @@ bool fused_step_applies(const hata_dims_t& d, int k) { return make_plan(d, k).ok
 size_t fused_step_ws_bytes(const hata_dims_t&, int) { return 0; }
 
 cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K, const void* V,
-                              const float* W, uint32_t* codes, const int32_t* seq_lens, int k, float scale,
-                              void* out, uint32_t* qcode_out, int32_t* idx_out, char* ws, cudaStream_t st) {
+                              const float* W, const float* Wk, uint32_t* codes, const int32_t* seq_lens, int k,
+                              float scale, void* out, uint32_t* qcode_out, int32_t* idx_out, char* ws,
+                              cudaStream_t st) {
   const Plan pl = make_plan(d, k);
   if (!pl.ok) return cudaErrorNotSupported;
   FusedParams prm;
@@ -1226,6 +1244,7 @@ cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const voi
   prm.K = K;
   prm.V = V;
   prm.W = W;
+  prm.Wk = Wk == W ? nullptr : Wk;
   prm.codes = codes;
   prm.seq_lens = seq_lens;
   prm.out = out;

@@ -182,6 +182,21 @@ HATA_API hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, 
                                size_t workspace_bytes, void* stream);
 
 /*
+ * The decode step with separate query and key encoders, the form of
+ * "HashAttention: Semantic Sparsity for Faster Inference" (its summary's
+ * Approach: independent key and query mappings into Hamming space, pivotal
+ * tokens found by XOR + popcount): queries are encoded with W_q, the new key
+ * with W_k ([Hkv][d][r] fp32 each, 16-byte aligned), and the cache must hold
+ * codes made with W_k (hata_encode_append with W_H = W_k).  Everything else,
+ * including layouts, outputs and errors, is as in hata_decode_step, which is
+ * this call with W_q = W_k.
+ */
+HATA_API hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                  const float* W_q, const float* W_k, uint32_t* codes, const int32_t* seq_lens,
+                                  int k, float scale, void* out, uint32_t* qcode_out, int32_t* idx_out,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dense flash-decode, the comparison baseline: exact attention of every query
  * head over all cached tokens (the dense attention that the "HATA" paper notes'
  * 实验 section times HATA against, at 32K-128K context):

@@ -175,12 +175,16 @@ def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, S: np.ndarray,
 # The decode step: encode q, encode + append the new key, scan, select, attend
 # ----------------------------------------------------------------------------
 
-def decode_step(q, K, V, W_H, codes, seq_lens, k: int, scale: float | None = None):
+def decode_step(q, K, V, W_H, codes, seq_lens, k: int, scale: float | None = None, W_k=None):
     """One HATA decode step over a batch.
 
     q: [B][Hq][d]; K, V: [B][Hkv][Lmax][d] with the new token already at slot
     L_b - 1; W_H: [Hkv][d][r]; codes: [B][Hkv][Lmax][r/32] holding the codes of
-    slots [0, L_b - 1); seq_lens: [B].
+    slots [0, L_b - 1); seq_lens: [B].  W_k (optional, [Hkv][d][r]) is a separate
+    key encoder, the form of "HashAttention: Semantic Sparsity for Faster
+    Inference" (independent query and key mappings, summary > Approach): the
+    queries are encoded with W_H, the new key with W_k, and `codes` must hold
+    keys encoded with W_k.  Without it W_H encodes both (HATA).
 
     Returns a dict with qcode [B][Hq][W], codes (copy with slot L_b - 1 written),
     y_q / y_k (projections, for the sign-exemption band), D (list over (b, g) of
@@ -209,7 +213,7 @@ def decode_step(q, K, V, W_H, codes, seq_lens, k: int, scale: float | None = Non
             heads = range(g * G, (g + 1) * G)
             for h in heads:
                 qcode[b, h], y_q[b, h] = encode(q[b, h], W_H[g])
-            codes[b, g, Lb - 1], y_k[b, g] = encode(K[b, g, Lb - 1], W_H[g])
+            codes[b, g, Lb - 1], y_k[b, g] = encode(K[b, g, Lb - 1], (W_H if W_k is None else W_k)[g])
             D = gqa_scores(qcode[b, g * G : (g + 1) * G], codes[b, g, :Lb], r)
             S = topk_select(D, k)
             idx[b, g, : len(S)] = S

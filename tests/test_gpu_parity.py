@@ -274,11 +274,12 @@ def run_step(H, wl, inp, codes0, ws=None, with_debug=True):
     }
 
 
-def check_step(wl, inp, codes0, got):
+def check_step(wl, inp, codes0, got, W_k=None):
     """Compare one decode step with the oracle.  Where the GPU's fp32 projection
     lands on the other side of zero inside the exemption band, the downstream
-    results are checked for validity against the codes the GPU chose."""
-    ref = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes0, inp["seq_lens"], wl.k)
+    results are checked for validity against the codes the GPU chose.  W_k: a
+    separate key encoder (codes0 then holds keys encoded with it)."""
+    ref = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes0, inp["seq_lens"], wl.k, W_k=W_k)
     G, r = wl.group, wl.hash_bits
     flips = assert_codes_match(got["qcode"], ref["qcode"], ref["y_q"], r)
     for b in range(wl.batch):
@@ -352,6 +353,46 @@ def test_decode_step_without_debug_outputs_and_repeat(H):
     b = run_step(H, wl, inp, codes0, ws=a["ws"], with_debug=False)
     assert np.array_equal(a["out"], b["out"])
     assert np.array_equal(a["codes"], b["codes"])
+
+
+def run_step_qk(H, wl, inp, W_k, codes0, ws=None):
+    d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype)
+    ws = ws if ws is not None else new_workspace(d, wl.k)
+    codes = dev_codes(codes0)
+    out = torch.full((wl.batch, wl.n_q_heads, 128), float("nan"), dtype=d.torch_dtype, device="cuda")
+    qcode = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda")
+    idx = torch.full((wl.batch, wl.n_kv_heads, wl.k), -99, dtype=torch.int32, device="cuda")
+    H.hata_decode_step_qk(d, dev_float(inp["q"], wl.dtype), dev_float(inp["K"], wl.dtype),
+                          dev_float(inp["V"], wl.dtype), torch.from_numpy(inp["W_H"]).cuda(),
+                          torch.from_numpy(W_k).cuda(), codes, torch.from_numpy(inp["seq_lens"]).cuda(), wl.k, 0.0,
+                          out, qcode, idx, ws)
+    torch.cuda.synchronize()
+    return {"codes": host_codes(codes), "out": out.float().cpu().numpy(), "qcode": host_codes(qcode),
+            "idx": idx.cpu().numpy(), "ws": ws}
+
+
+@pytest.mark.parametrize("name", ["llama_shape_9k", "narrow32", "tiny_f32_4k", "ragged_b3", "g3_chain"])
+def test_decode_step_separate_key_encoder(H, name):
+    """HashAttention form: queries encoded with W_q (= the workload's W_H), keys
+    with an independent W_k; the cache holds W_k codes.  Fused shapes and the
+    granular chain (g3_chain) against the oracle."""
+    wl = STEP_CASES[name]
+    inp = make_inputs(wl, seed=17)
+    W_k = (np.random.default_rng(1717).standard_normal(inp["W_H"].shape) / math.sqrt(128)).astype(np.float32)
+    codes0, _ = oracle.encode_cache(inp["K"], W_k, inp["seq_lens"])
+    got = run_step_qk(H, wl, inp, W_k, codes0)
+    check_step(wl, inp, codes0, got, W_k=W_k)
+    assert H.hata_read_device_status(got["ws"]) == 0
+
+
+def test_decode_step_qk_with_one_encoder_equals_decode_step(H):
+    wl = STEP_CASES["llama_shape_9k"]
+    inp = make_inputs(wl, seed=19)
+    codes0, _ = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"])
+    a = run_step(H, wl, inp, codes0)
+    b = run_step_qk(H, wl, inp, inp["W_H"].copy(), codes0)  # a separate buffer holding the same matrix
+    for k_ in ("codes", "qcode", "idx", "out"):
+        assert np.array_equal(a[k_], b[k_]), k_
 
 
 def test_decode_step_flags_length_beyond_cache(H):

@@ -334,6 +334,39 @@ def test_decode_step_composes_and_finds_planted_keys():
             np.testing.assert_array_equal(res["out"][b, g * G:(g + 1) * G], o)
 
 
+def test_decode_step_separate_key_encoder():
+    """HashAttention form (independent query and key encoders; HashAttention
+    summary, Approach).  Pins: (1) with W_k = W_H it is the HATA step exactly;
+    (2) with W_k = -W_H every key bit flips (y -> -y, and y = 0 has probability 0
+    here), so each head's distance becomes r - Ham and the GQA sum G*r - D: the
+    step then selects the min(k, L) tokens with the LARGEST D of the plain step,
+    ties to the lower index -- checked by a brute-force sort on (-D, t); (3) the
+    appended code is the key's encoding under W_k."""
+    wl = Workload("t", 2, 8, 2, 128, 500, 128, 40, "bf16", seq_len_range=(200, 500), n_planted=5)
+    inp = make_inputs(wl, seed=5)
+    lens = inp["seq_lens"]
+    codes, _ = oracle.encode_cache(inp["K"], inp["W_H"], lens)
+    plain = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes, lens, wl.k)
+    same = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes, lens, wl.k, W_k=inp["W_H"])
+    for key in ("qcode", "codes", "idx", "out"):
+        assert np.array_equal(plain[key], same[key]), key
+    W_neg = -inp["W_H"]
+    codes_neg, _ = oracle.encode_cache(inp["K"], W_neg, lens)
+    flip = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes_neg, lens, wl.k, W_k=W_neg)
+    G, r = wl.group, wl.hash_bits
+    assert np.array_equal(flip["qcode"], plain["qcode"])
+    for b in range(wl.batch):
+        Lb = int(lens[b])
+        for g in range(wl.n_kv_heads):
+            c, _ = oracle.encode(inp["K"][b, g, Lb - 1], W_neg[g])
+            assert np.array_equal(flip["codes"][b, g, Lb - 1], c)
+            D = np.asarray(plain["D"][(b, g)])
+            assert np.array_equal(np.asarray(flip["D"][(b, g)]), G * r - D)
+            want = sorted(sorted(range(Lb), key=lambda t: (-int(D[t]), t))[: min(wl.k, Lb)])
+            got = flip["idx"][b, g][flip["idx"][b, g] >= 0]
+            assert got.tolist() == want
+
+
 def test_bf16_rounding_of_inputs():
     """The input generator's bf16 rounding is round-to-nearest-even (checked against torch)."""
     import torch
