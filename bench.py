@@ -456,6 +456,49 @@ def run_gpu(args, wl):
                  "hata_speedup": d_ms / ms_per_step}
         del gd
 
+    # the same step over a paged cache: every layer's K, V and code buffers seen as
+    # pools of 256-token blocks, reached through a random (non-contiguous) block table
+    paged = None
+    bs_p = 256
+    if wl.max_seq % bs_p == 0 and H.hata_decode_step_kernel_count(dims, wl.k) == 1:
+        max_blocks = wl.max_seq // bs_p
+        n_blocks = wl.batch * max_blocks
+        gen = torch.Generator().manual_seed(args.seed + 1)
+        btab = torch.randperm(n_blocks, generator=gen).to(torch.int32).reshape(wl.batch, max_blocks).to(dev)
+        pool = (n_blocks, wl.n_kv_heads, bs_p)
+
+        def paged_step(i):
+            L = layers[i % R]
+            H.hata_decode_step_paged(dims, L["q"], L["K"].view(*pool, wl.head_dim), L["V"].view(*pool, wl.head_dim),
+                                     L["W"], L["W"], L["codes"].view(*pool, wl.words), btab, bs_p, L["lens"], wl.k,
+                                     0.0, L["out"], None, None, ws, stream)
+
+        p_steps = min(args.steps, 2000)
+        with torch.cuda.stream(stream):
+            for i in range(3):
+                paged_step(i)
+        torch.cuda.synchronize()
+        gp = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gp, stream=stream):
+            for i in range(min(p_steps, GRAPH_CHUNK)):
+                paged_step(i)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            gp.replay()  # warm-up
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            reps = max(1, p_steps // min(p_steps, GRAPH_CHUNK))
+            for _ in range(reps):
+                gp.replay()
+            e1.record(stream)
+            e1.synchronize()
+        p_ms = e0.elapsed_time(e1) / (reps * min(p_steps, GRAPH_CHUNK))
+        paged = {"kernel": "hata_decode_step_paged (256-token blocks, random block table)",
+                 "us_per_step": p_ms * 1e3, "achieved_gbs": step_bytes / (p_ms * 1e-3) / 1e9,
+                 "vs_unpaged": ms_per_step / p_ms}
+        del gp
+
     # prefill encode (hata_encode_append over every cached key of every layer buffer)
     pre_reps = max(2, min(R, 8))
     with torch.cuda.stream(stream):
@@ -515,6 +558,7 @@ def run_gpu(args, wl):
                 "steps": e2e_steps},
         "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
         "dense_baseline": dense,
+        "paged_step": paged,
         "prefill_encode": prefill,
         "clocks": sampler.summary(),
     }

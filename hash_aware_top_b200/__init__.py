@@ -33,6 +33,7 @@ __all__ = [
     "hata_sparse_decode",
     "hata_decode_step",
     "hata_decode_step_qk",
+    "hata_decode_step_paged",
     "hata_read_device_status",
     "hata_status_string",
     "hata_version",
@@ -59,6 +60,7 @@ EXPORTED_SYMBOLS = (
     "hata_sparse_decode",
     "hata_decode_step",
     "hata_decode_step_qk",
+    "hata_decode_step_paged",
     "hata_read_device_status",
     "hata_status_string",
     "hata_version",
@@ -115,6 +117,7 @@ def _load():
         "hata_sparse_decode": (I, [DP, P, P, P, P, I, F, P, P, S, P]),
         "hata_decode_step": (I, [DP, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
         "hata_decode_step_qk": (I, [DP, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
+        "hata_decode_step_paged": (I, [DP, P, P, P, P, P, P, P, I, I, P, I, F, P, P, P, P, S, P]),
         "hata_read_device_status": (I, [P, P, ctypes.POINTER(I)]),
         "hata_status_string": (ctypes.c_char_p, [I]),
         "hata_version": (I, []),
@@ -330,6 +333,31 @@ def hata_decode_step_qk(dims: Dims, q, K, V, W_q, W_k, codes, seq_lens, k, scale
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step_qk")
+
+
+def hata_decode_step_paged(dims: Dims, q, K_pool, V_pool, W_q, W_k, codes_pool, block_table, block_size, seq_lens, k,
+                           scale, out, qcode_out, idx_out, ws, stream=None):
+    """The decode step over a paged cache: pools [n_blocks][Hkv][block_size][...], block_table [B][max_blocks]."""
+    d = dims
+    n_blocks = int(K_pool.shape[0]) if K_pool is not None else 0
+    bs = int(block_size)
+    pool = (n_blocks, d.n_kv_heads, bs, d.head_dim)
+    wshape = (d.n_kv_heads, d.head_dim, d.hash_bits)
+    max_blocks = (d.max_seq + bs - 1) // bs if bs > 0 else 0
+    _check(
+        lib.hata_decode_step_paged(
+            ctypes.byref(d),
+            _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(K_pool, "K_pool", pool, d.torch_dtype), _ptr(V_pool, "V_pool", pool, d.torch_dtype),
+            _ptr(W_q, "W_q", wshape, torch.float32), _ptr(W_k, "W_k", wshape, torch.float32),
+            _ptr(codes_pool, "codes_pool", (n_blocks, d.n_kv_heads, bs, d.words), _codes_dtype(codes_pool)),
+            _ptr(block_table, "block_table", (d.batch, max_blocks), torch.int32), bs, n_blocks,
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k), float(scale),
+            _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
+            _ptr(qcode_out, "qcode_out", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode_out), optional=True),
+            _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
+            _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
+        "hata_decode_step_paged")
 
 
 def hata_read_device_status(ws, stream=None) -> int:

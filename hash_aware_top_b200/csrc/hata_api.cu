@@ -160,8 +160,8 @@ hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
-  cudaError_t e =
-      launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, ws, st);
+  cudaError_t e = launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out,
+                                    nullptr, ws, st);
   if (e != cudaErrorNotSupported) return cuda_status(e);
 
   // Chain of the granular kernels (shapes the fused kernel does not cover).
@@ -183,6 +183,37 @@ hata_status_t hata_decode_step(const hata_dims_t* dims, const void* q, const voi
                                size_t workspace_bytes, void* stream) {
   return hata_decode_step_qk(dims, q, K, V, W_H, W_H, codes, seq_lens, k, scale, out, qcode_out, idx_out, workspace,
                              workspace_bytes, stream);
+}
+
+hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, const void* K_pool, const void* V_pool,
+                                     const float* W_q, const float* W_k, uint32_t* codes_pool,
+                                     const int32_t* block_table, int block_size, int n_blocks,
+                                     const int32_t* seq_lens, int k, float scale, void* out, uint32_t* qcode_out,
+                                     int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!q || !K_pool || !V_pool || !W_q || !W_k || !codes_pool || !block_table || !seq_lens || !out || k < 1)
+    return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K_pool) || !aligned16(V_pool) || !aligned16(W_q) || !aligned16(W_k) ||
+      !aligned16(codes_pool) || !aligned16(out))
+    return HATA_ERR_INVALID_ARG;
+  if (block_size < 16 || block_size > 65536 || (block_size & (block_size - 1)) || n_blocks < 1)
+    return HATA_ERR_INVALID_ARG;
+  if ((long long)n_blocks * dims->n_kv_heads * block_size > 0x7fffffffLL) return HATA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return HATA_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = check_ws(*dims, k, workspace, workspace_bytes, &L)) != HATA_OK) return s;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)dims->head_dim);
+  PagedCache pg;
+  pg.block_table = block_table;
+  pg.block_shift = 0;
+  while ((1 << pg.block_shift) < block_size) ++pg.block_shift;
+  pg.n_blocks = n_blocks;
+  pg.max_blocks = (dims->max_seq + block_size - 1) / block_size;
+  const cudaError_t e = launch_fused_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out,
+                                          qcode_out, idx_out, &pg, static_cast<char*>(workspace),
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaErrorNotSupported ? HATA_ERR_UNSUPPORTED : cuda_status(e);
 }
 
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {

@@ -31,10 +31,18 @@ size_t dense_ws_bytes(const hata_dims_t& d);
 cudaError_t launch_dense_decode(const hata_dims_t& d, const void* q, const void* K, const void* V,
                                 const int32_t* seq_lens, float scale, void* out, char* ws, cudaStream_t stream);
 // Returns cudaErrorNotSupported when the fused kernel does not apply to these dims.
+// Paged cache: K, V and codes are pools [n_blocks][Hkv][1 << block_shift][...] and
+// block_table [B][max_blocks] maps each sequence's logical blocks to pool blocks.
+struct PagedCache {
+  const int32_t* block_table;
+  int block_shift, n_blocks, max_blocks;
+};
+
 // Wk: separate key encoder, or equal to W (one encoder for queries and keys).
+// pg: paged cache, or null for [B][Hkv][max_seq][...] slabs.
 cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K,
                               const void* V, const float* W, const float* Wk, uint32_t* codes,
                               const int32_t* seq_lens, int k, float scale, void* out, uint32_t* qcode_out,
-                              int32_t* idx_out, char* ws, cudaStream_t stream);
+                              int32_t* idx_out, const PagedCache* pg, char* ws, cudaStream_t stream);
 
 }  // namespace hata

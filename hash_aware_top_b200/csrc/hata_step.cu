@@ -78,6 +78,9 @@ struct FusedParams {
   int Hq, Hkv, max_seq, k, nbins, tok_cap, sel_cap, flags, stages;
   float scale_log2;
   SmemLayout lay;  // shared-memory layout of the launch (computed on the host)
+  // paged cache (K, V and codes are pools of blocks [n_blocks][Hkv][1 << block_shift][...])
+  const int32_t* block_table;  // [B][max_blocks] physical block of each logical block
+  int block_shift, n_blocks, max_blocks;
 };
 
 struct Bump {
@@ -168,7 +171,7 @@ struct Vec16<float> {
   }
 };
 
-template <typename T, int NW, int G>
+template <typename T, int NW, int G, bool PAGED>
 __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
   constexpr int D = kHeadDim;
@@ -266,7 +269,24 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int t0 = min(L, rank * C), t1 = min(L, t0 + C);
   const int nmine = t1 - t0;
   const int nst = (nmine + ST - 1) / ST;
-  uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;
+  // Slot of token t of this unit in the K, V and code arrays: slot t of the unit's
+  // slab, or (paged) slot t mod bs of physical block block_table[b][t / bs], whose
+  // KV head g part holds bs consecutive slots.  A block number outside the pool
+  // is flagged and replaced by block 0.
+  const int32_t* btab = PAGED ? p.block_table + (size_t)b * p.max_blocks : nullptr;
+  auto slot_of = [&](int t) -> size_t {
+    if constexpr (PAGED) {
+      int pb = btab[t >> p.block_shift];
+      if ((unsigned)pb >= (unsigned)p.n_blocks) {
+        set_status(p.status, HATA_ERR_INVALID_ARG);
+        pb = 0;
+      }
+      return (((size_t)pb * p.Hkv + g) << p.block_shift) | (size_t)(t & ((1 << p.block_shift) - 1));
+    } else {
+      return (size_t)u * p.max_seq + t;
+    }
+  };
+  uint32_t* cu = p.codes + (size_t)u * p.max_seq * NW;  // the unit's slab (unpaged cache)
   const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;  // this CTA appends the new key's code
   const uint64_t pol_stream = ptx::policy_evict_first();
   auto issue = [&](int s) {
@@ -276,7 +296,18 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     uint64_t* bar = &mbar[s % kStages];
     lastv[s % kStages] = s;
     ptx::mbar_arrive_expect_tx(bar, bytes);
-    if (bytes) ptx::bulk_g2s(ring + (s % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
+    if constexpr (PAGED) {
+      // one copy per block segment (segments start on 16-token boundaries: bs >= 16)
+      const int bsz = 1 << p.block_shift;
+      for (int x = 0; x < nb;) {
+        const int t = ts + x, seg = min(nb - x, bsz - (t & (bsz - 1)));
+        ptx::bulk_g2s(ring + (s % kStages) * kStageBytes + (size_t)x * NW * 4, p.codes + slot_of(t) * NW,
+                      (uint32_t)seg * NW * 4, bar, pol_stream);
+        x += seg;
+      }
+    } else {
+      if (bytes) ptx::bulk_g2s(ring + (s % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
+    }
   };
   if (tid == 0)
     for (int s = 0; s < min(nst, kStages); ++s) issue(s);
@@ -287,7 +318,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     if (tid < QV) xv = reinterpret_cast<const uint4*>(qg)[tid];
   }
   {
-    const T* kn = static_cast<const T*>(p.K) + (((size_t)u * p.max_seq) + (L > 0 ? L - 1 : 0)) * D;
+    const T* kn = static_cast<const T*>(p.K) + slot_of(L > 0 ? L - 1 : 0) * D;
     if (tid >= QV && tid < XV && L > 0) xv = reinterpret_cast<const uint4*>(kn)[tid - QV];
   }
   // fp32 copies: residue-major for the encode (element i of vector v at
@@ -366,7 +397,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   }
   __syncthreads();  // codes ready; the residue sums are consumed
   if (rank == 0 && p.qcode_out && tid < G * NW) p.qcode_out[((size_t)b * p.Hq + (size_t)g * G) * NW + tid] = qc[tid];
-  if (own_last && tid < NW) cu[(size_t)(L - 1) * NW + tid] = qc[G * NW + tid];
+  if (own_last && tid < NW) p.codes[slot_of(L - 1) * NW + tid] = qc[G * NW + tid];
   // ---- 3. scan: scores + histogram; each warp releases ring stages on its own ---
   {
     GroupQuery<NW, G> gq;
@@ -411,7 +442,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
           }
         } else if (i < nt) {
 #pragma unroll
-          for (int w = 0; w < NW; ++w) kw[j][w] = cu[(size_t)(ts + i) * NW + w];
+          for (int w = 0; w < NW; ++w) kw[j][w] = p.codes[slot_of(ts + i) * NW + w];
         }
       }
 #pragma unroll
@@ -511,8 +542,8 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   const int Tc = stat[ST_SPEC];
   const bool scan_cands = Tc >= 0 && !stat[ST_ABORT];
 
-  const T* Kb = static_cast<const T*>(p.K) + (size_t)u * p.max_seq * D;
-  const T* Vb = static_cast<const T*>(p.V) + (size_t)u * p.max_seq * D;
+  const T* Kg = static_cast<const T*>(p.K);
+  const T* Vg = static_cast<const T*>(p.V);
   T* Kr = reinterpret_cast<T*>(ring);
   T* Vr = reinterpret_cast<T*>(ring) + (size_t)GB * D;
   // Row gathers complete on the gather mbarrier: every thread arrives once per
@@ -537,8 +568,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
         set_status(p.status, HATA_ERR_INVALID_ARG);
         t = t0;
       }
-      if (w < RPR) ptx::cp_async16(Kr + (size_t)r * D + w * EPV, Kb + (size_t)t * D + w * EPV);
-      else ptx::cp_async16(Vr + (size_t)r * D + (w - RPR) * EPV, Vb + (size_t)t * D + (w - RPR) * EPV);
+      const size_t row = slot_of(t) * D;
+      if (w < RPR) ptx::cp_async16(Kr + (size_t)r * D + w * EPV, Kg + row + w * EPV);
+      else ptx::cp_async16(Vr + (size_t)r * D + (w - RPR) * EPV, Vg + row + (w - RPR) * EPV);
     }
     gather_commit();
   };
@@ -695,8 +727,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     for (int e = lane; e < nq * 2 * RPR; e += 32) {
       const int q = q0 + e / (2 * RPR), pc = e % (2 * RPR);
       const int t = cand[q];
-      if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kb + (size_t)t * D + pc * EPV);
-      else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vb + (size_t)t * D + (pc - RPR) * EPV);
+      const size_t row = slot_of(t) * D;
+      if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kg + row + pc * EPV);
+      else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vg + row + (pc - RPR) * EPV);
     }
   }
   gather_commit();  // gather phase 0: the candidates' rows
@@ -1085,7 +1118,7 @@ cudaError_t configure_kernel(const void* kern) {
 template <typename T, int NW, int G>
 Plan make_plan_t(const hata_dims_t& d, int k) {
   Plan best{};
-  const void* kern = (const void*)fused_step_kernel<T, NW, G>;
+  const void* kern = (const void*)fused_step_kernel<T, NW, G, false>;
   const int R = NW * 32, esize = (int)sizeof(T);
   const long long units = (long long)d.batch * d.n_kv_heads;
   static const int cands[] = {16, 15, 14, 12, 10, 8, 6, 4, 3, 2, 1};
@@ -1133,9 +1166,9 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
   return best;
 }
 
-template <typename T, int NW, int G>
+template <typename T, int NW, int G, bool PAGED>
 cudaError_t launch_fused_t(const Plan& pl, const hata_dims_t& d, const FusedParams& prm, cudaStream_t st) {
-  auto kern = fused_step_kernel<T, NW, G>;
+  auto kern = fused_step_kernel<T, NW, G, PAGED>;
   const cudaError_t ce = configure_kernel((const void*)kern);
   if (ce != cudaSuccess) return ce;
   cudaLaunchConfig_t cfg = {};
@@ -1193,7 +1226,8 @@ struct PlanFn {
 template <typename T, int NW, int G>
 struct LaunchFn {
   static cudaError_t run(const Plan& pl, const hata_dims_t& d, const FusedParams& prm, cudaStream_t st) {
-    return launch_fused_t<T, NW, G>(pl, d, prm, st);
+    return prm.block_table ? launch_fused_t<T, NW, G, true>(pl, d, prm, st)
+                           : launch_fused_t<T, NW, G, false>(pl, d, prm, st);
   }
   static cudaError_t fail() { return cudaErrorNotSupported; }
 };
@@ -1235,8 +1269,8 @@ size_t fused_step_ws_bytes(const hata_dims_t&, int) { return 0; }
 
 cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K, const void* V,
                               const float* W, const float* Wk, uint32_t* codes, const int32_t* seq_lens, int k,
-                              float scale, void* out, uint32_t* qcode_out, int32_t* idx_out, char* ws,
-                              cudaStream_t st) {
+                              float scale, void* out, uint32_t* qcode_out, int32_t* idx_out,
+                              const PagedCache* pg, char* ws, cudaStream_t st) {
   const Plan pl = make_plan(d, k);
   if (!pl.ok) return cudaErrorNotSupported;
   FusedParams prm;
@@ -1262,6 +1296,10 @@ cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const voi
   prm.stages = pl.stages;
   prm.lay = pl.lay;
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.block_table = pg ? pg->block_table : nullptr;
+  prm.block_shift = pg ? pg->block_shift : 0;
+  prm.n_blocks = pg ? pg->n_blocks : 0;
+  prm.max_blocks = pg ? pg->max_blocks : 0;
   return dispatch<LaunchFn>(d, pl, d, prm, st);
 }
 

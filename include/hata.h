@@ -197,6 +197,30 @@ HATA_API hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* 
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The decode step over a paged cache (the block layout of vLLM PagedAttention,
+ * which the HashAttention summary lists among its foundations; a growing cache
+ * appends one token per step).  K_pool and V_pool are [n_blocks][Hkv][bs][d]
+ * (dims->dtype), codes_pool is [n_blocks][Hkv][bs][r/32] uint32, block_size bs is
+ * a power of two in [16, 65536].  Sequence b's logical token t lives in slot
+ * t mod bs of pool block block_table[b][t / bs]; block_table is device
+ * [B][ceil(max_seq / bs)] int32, with dims->max_seq the logical capacity of a
+ * sequence.  The new token's K/V row must already be in its slot, and its code is
+ * written there.  Queries are encoded with W_q and keys with W_k (pass the same
+ * matrix twice for HATA's single encoder).  Indices in idx_out are logical token
+ * indices; everything else is as in hata_decode_step.  A block number outside
+ * [0, n_blocks) is replaced by block 0 and flagged in the status word.  Returns
+ * HATA_ERR_UNSUPPORTED for shapes the fused kernel does not cover (G not in
+ * {1, 2, 4, 8}).  The prefill encode of a paged cache is hata_encode_append over
+ * the pool seen as a batch of blocks: dims with batch = n_blocks, max_seq = bs,
+ * x = K_pool, x_heads = Hkv, x_len = n_tok = codes_len = bs, seq_end = NULL.
+ */
+HATA_API hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, const void* K_pool,
+                                     const void* V_pool, const float* W_q, const float* W_k, uint32_t* codes_pool,
+                                     const int32_t* block_table, int block_size, int n_blocks,
+                                     const int32_t* seq_lens, int k, float scale, void* out, uint32_t* qcode_out,
+                                     int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dense flash-decode, the comparison baseline: exact attention of every query
  * head over all cached tokens (the dense attention that the "HATA" paper notes'
  * 实验 section times HATA against, at 32K-128K context):
