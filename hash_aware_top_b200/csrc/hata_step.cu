@@ -371,8 +371,9 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       for (int u4 = 0; u4 < 4; ++u4)
 #pragma unroll
         for (int a = 0; a < 8; ++a) wr[u4 * 8 + a] = Wsm[(s + 4 * a + 32 * u4) * R + j];
-#pragma unroll 1
-      for (int v = 0; v < nv_w; ++v) residue_sums(wr, v, s, j);
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+        if (v < nv_w) residue_sums(wr, v, s, j);
     }
     if (p.Wk && own_last) {  // block-uniform
       const float* Wkg = p.Wk + (size_t)g * D * R;
