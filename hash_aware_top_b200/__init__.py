@@ -27,6 +27,7 @@ __all__ = [
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_encode_append",
+    "hata_encode_read_status",
     "hata_hamming_scores",
     "hata_topk",
     "hata_topk_noalloc",
@@ -55,6 +56,7 @@ EXPORTED_SYMBOLS = (
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_encode_append",
+    "hata_encode_read_status",
     "hata_hamming_scores",
     "hata_topk",
     "hata_sparse_decode",
@@ -119,6 +121,7 @@ def _load():
         "hata_decode_step_qk": (I, [DP, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
         "hata_decode_step_paged": (I, [DP, P, P, P, P, P, P, P, I, I, P, I, F, P, P, P, P, S, P]),
         "hata_read_device_status": (I, [P, P, ctypes.POINTER(I)]),
+        "hata_encode_read_status": (I, [P, ctypes.POINTER(I)]),
         "hata_status_string": (ctypes.c_char_p, [I]),
         "hata_version": (I, []),
         "hata_decode_step_kernel_count": (I, [DP, I]),
@@ -358,6 +361,12 @@ def hata_decode_step_paged(dims: Dims, q, K_pool, V_pool, W_q, W_k, codes_pool, 
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step_paged")
+
+
+def hata_encode_read_status(stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(lib.hata_encode_read_status(_stream(stream), ctypes.byref(v)), "hata_encode_read_status")
+    return v.value
 
 
 def hata_read_device_status(ws, stream=None) -> int:

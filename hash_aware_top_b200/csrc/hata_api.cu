@@ -216,6 +216,14 @@ hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, con
   return e == cudaErrorNotSupported ? HATA_ERR_UNSUPPORTED : cuda_status(e);
 }
 
+hata_status_t hata_encode_read_status(void* stream, int* device_status) {
+  if (!device_status) return HATA_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  if (read_encode_status(static_cast<cudaStream_t>(stream), &v) != cudaSuccess) return HATA_ERR_CUDA;
+  *device_status = (int)v;
+  return HATA_OK;
+}
+
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {
   if (check_dims(dims) != HATA_OK || k < 1) return -1;
   return fused_step_applies(*dims, k) ? 1 : 6;

@@ -139,8 +139,9 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
                                                           W, codes, codes_len, hpg, d.hash_bits);
     return cudaGetLastError();
   }
-  if constexpr (sizeof(T) == 2) {  // bf16 keys: the tensor-core prefill (r <= 128)
-    const cudaError_t e = launch_encode_mma(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
+  if constexpr (sizeof(T) == 2) {  // bf16 keys: tensor-core prefill (r <= 128), tcgen05 first, then mma.sync
+    cudaError_t e = launch_encode_tc(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
+    if (e == cudaErrorNotSupported) e = launch_encode_mma(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
     if (e != cudaErrorNotSupported) return e;
   }
   const long long rows = (long long)hpg * n_tok;

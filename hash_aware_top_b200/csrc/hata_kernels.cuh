@@ -27,6 +27,12 @@ size_t fused_step_ws_bytes(const hata_dims_t& d, int k);
 cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
                               const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
                               cudaStream_t stream);
+// Prefill encode on tcgen05 tensor cores (bf16 keys, r <= 128; else cudaErrorNotSupported).
+cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
+                             const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                             cudaStream_t stream);
+// Read and clear the encode kernels' device status word (synchronises the stream).
+cudaError_t read_encode_status(cudaStream_t stream, uint32_t* status);
 size_t dense_ws_bytes(const hata_dims_t& d);
 cudaError_t launch_dense_decode(const hata_dims_t& d, const void* q, const void* K, const void* V,
                                 const int32_t* seq_lens, float scale, void* out, char* ws, cudaStream_t stream);

@@ -134,6 +134,12 @@ HATA_API hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x
                                  const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,
                                  void* stream);
 
+/* Read and clear the status word of the prefill encode kernels (synchronises the
+ * stream): HATA_ERR_TIMEOUT if a bounded wait of a hata_encode_append call on
+ * the tensor cores expired since the last read (its codes are then incomplete),
+ * else 0.  The word is one per device, in the library. */
+HATA_API hata_status_t hata_encode_read_status(void* stream, int* device_status);
+
 /*
  * Hamming scan with the GQA sum (Decode 阶段算法, Hamming and GQA steps;
  * 硬件高效优化, XOR + popc operator):

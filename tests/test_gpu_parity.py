@@ -45,6 +45,7 @@ def test_encode_prefill_and_queries(H, r, dtype):
     codes = dev_codes(np.full((2, 2, 1000, r // 32), sentinel, dtype=np.uint32))
     # prefill every slot below L_b: n_tok = max_seq ending at seq_lens
     H.hata_encode_append(d, K, 2, 1000, 1000, lens, W, codes, 1000)
+    assert H.hata_encode_read_status() == 0
     got = host_codes(codes)
     want, ys = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"], upto_last=False)
     for b in range(2):
@@ -61,6 +62,52 @@ def test_encode_prefill_and_queries(H, r, dtype):
         for h in range(8):
             c, y = oracle.encode(inp["q"][b, h], inp["W_H"][h // 4])
             assert_codes_match(gq[b, h], c, y, r)
+
+
+@pytest.mark.parametrize("r", [32, 64, 128])
+def test_encode_prefill_many_tiles_per_cta(H, r):
+    """A prefill long enough that every CTA of the tensor-core encode runs many
+    128-key tiles (its shared-memory stages and both accumulators wrap around
+    several times), with a ragged end."""
+    B, Hkv, L = 1, 8, 40000
+    wl = Workload("enc_long", B, 8, Hkv, 128, L, r, 16, "bf16", seq_len_range=(L - 77, L - 77))
+    inp = make_inputs(wl, seed=3, plant=False)
+    d = _dims(H, B, 8, Hkv, r, L, "bf16")
+    codes = dev_codes(np.zeros((B, Hkv, L, r // 32), dtype=np.uint32))
+    H.hata_encode_append(d, dev_float(inp["K"], "bf16"), Hkv, L, L, torch.from_numpy(inp["seq_lens"]).cuda(),
+                         torch.from_numpy(inp["W_H"]).cuda(), codes, L)
+    assert H.hata_encode_read_status() == 0
+    got = host_codes(codes)
+    want, ys = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"], upto_last=False)
+    Lb = int(inp["seq_lens"][0])
+    for g in range(Hkv):
+        assert_codes_match(got[0, g, :Lb], want[0, g, :Lb], ys[(0, g)], r)
+        assert np.all(got[0, g, Lb:] == 0)
+
+
+def test_encode_prefill_grouped_heads_window(H):
+    """The prefill form on query-like input: x_heads = Hq grouped on W_H[h // G],
+    a window of n_tok slots ending at seq_end, codes_len shorter than x_len."""
+    B, Hq, Hkv, xl, cl, r = 2, 8, 2, 700, 650, 128
+    rng = np.random.default_rng(5)
+    x = torch.tensor(rng.standard_normal((B, Hq, xl, 128), dtype=np.float32)).bfloat16()
+    W = (rng.standard_normal((Hkv, 128, r)) / math.sqrt(128)).astype(np.float32)
+    end = np.array([600, 690], dtype=np.int32)
+    n_tok = 333
+    d = _dims(H, B, Hq, Hkv, r, cl, "bf16")
+    sentinel = np.uint32(0x5A5A5A5A)
+    codes = dev_codes(np.full((B, Hq, cl, r // 32), sentinel, dtype=np.uint32))
+    H.hata_encode_append(d, x.cuda(), Hq, xl, n_tok, torch.from_numpy(end).cuda(), torch.from_numpy(W).cuda(),
+                         codes, cl)
+    assert H.hata_encode_read_status() == 0
+    got = host_codes(codes)
+    xf = x.float().numpy()
+    for b in range(B):
+        lo, hi = max(int(end[b]) - n_tok, 0), min(int(end[b]), cl)
+        for h in range(Hq):
+            c, y = oracle.encode(xf[b, h, lo:hi], W[h // (Hq // Hkv)])
+            assert_codes_match(got[b, h, lo:hi], c, y, r)
+            assert np.all(got[b, h, :lo] == sentinel) and np.all(got[b, h, hi:] == sentinel)
 
 
 def test_encode_append_single_slot(H):
