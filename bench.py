@@ -80,6 +80,15 @@ def recorded_traffic(workload_name):
     return int(fields["dram_bytes_per_launch"])
 
 
+def tensor_peak_bf16():
+    """Measured dense bf16 tensor throughput (TFLOP/s, burst) from MEASURED_PEAKS.json, or None."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -516,10 +525,17 @@ def run_gpu(args, wl):
     pre_ms = e0.elapsed_time(e1) / pre_reps
     n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
     pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + wl.hash_bits // 8)
-    prefill = {"kernel": "hata_encode_append (prefill form)", "us_per_call": pre_ms * 1e3, "keys": n_keys,
+    prefill = {"kernel": "hata_encode_append (prefill form; bf16 keys: tcgen05 tensor cores)",
+               "us_per_call": pre_ms * 1e3, "keys": n_keys,
                "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
                "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
                "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
+    if wl.dtype == "bf16" and wl.hash_bits <= 128:
+        # the tensor cores run W_H as three bf16 parts: 3x the algorithmic flops
+        prefill["mma_tflops"] = 3.0 * prefill["tflops"]
+        tpeak = tensor_peak_bf16()
+        if tpeak:
+            prefill["frac_of_tensor_peak"] = prefill["mma_tflops"] / tpeak
 
     peak, peak_kind = peak_hbm()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9

@@ -184,6 +184,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   constexpr int QV = G * D * ESZ / 16;            // ... of which the queries
   constexpr int EPV = 16 / ESZ;                   // elements per 16-byte vector
   constexpr int RPR = D * ESZ / 16;               // 16-byte pieces per K or V row
+  static_assert((2 * RPR) % 32 == 0, "a candidate's K and V pieces fill whole warps");
   constexpr int LT = 16;                          // threads per row in the logits
   constexpr int LE = D / LT;                      // elements per thread in the logits (8)
   constexpr int PVG = kFThreads / (D / 2);        // row groups in P.V (8): thread = (column pair, row group)
@@ -274,14 +275,16 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   // KV head g part holds bs consecutive slots.  A block number outside the pool
   // is flagged and replaced by block 0.
   const int32_t* btab = PAGED ? p.block_table + (size_t)b * p.max_blocks : nullptr;
+  auto phys_slot = [&](int pb, int t) -> size_t {  // (paged) slot of token t in pool block pb
+    if ((unsigned)pb >= (unsigned)p.n_blocks) {
+      set_status(p.status, HATA_ERR_INVALID_ARG);
+      pb = 0;
+    }
+    return (((size_t)pb * p.Hkv + g) << p.block_shift) | (size_t)(t & ((1 << p.block_shift) - 1));
+  };
   auto slot_of = [&](int t) -> size_t {
     if constexpr (PAGED) {
-      int pb = btab[t >> p.block_shift];
-      if ((unsigned)pb >= (unsigned)p.n_blocks) {
-        set_status(p.status, HATA_ERR_INVALID_ARG);
-        pb = 0;
-      }
-      return (((size_t)pb * p.Hkv + g) << p.block_shift) | (size_t)(t & ((1 << p.block_shift) - 1));
+      return phys_slot(btab[t >> p.block_shift], t);
     } else {
       return (size_t)u * p.max_seq + t;
     }
@@ -297,13 +300,27 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     lastv[s % kStages] = s;
     ptx::mbar_arrive_expect_tx(bar, bytes);
     if constexpr (PAGED) {
-      // one copy per block segment (segments start on 16-token boundaries: bs >= 16)
+      // one copy per block segment (segments start on 16-token boundaries: bs >= 16);
+      // up to 8 segments' block numbers are loaded together before their copies
       const int bsz = 1 << p.block_shift;
-      for (int x = 0; x < nb;) {
-        const int t = ts + x, seg = min(nb - x, bsz - (t & (bsz - 1)));
-        ptx::bulk_g2s(ring + (s % kStages) * kStageBytes + (size_t)x * NW * 4, p.codes + slot_of(t) * NW,
-                      (uint32_t)seg * NW * 4, bar, pol_stream);
-        x += seg;
+      for (int x0 = 0; x0 < nb;) {
+        int pbk[8], xs[8], sg[8], nseg = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (x0 < nb) {
+            const int t = ts + x0, seg = min(nb - x0, bsz - (t & (bsz - 1)));
+            pbk[k] = btab[t >> p.block_shift];
+            xs[k] = x0;
+            sg[k] = seg;
+            x0 += seg;
+            nseg = k + 1;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (k < nseg)
+            ptx::bulk_g2s(ring + (s % kStages) * kStageBytes + (size_t)xs[k] * NW * 4,
+                          p.codes + phys_slot(pbk[k], ts + xs[k]) * NW, (uint32_t)sg[k] * NW * 4, bar, pol_stream);
       }
     } else {
       if (bytes) ptx::bulk_g2s(ring + (s % kStages) * kStageBytes, cu + (size_t)ts * NW, bytes, bar, pol_stream);
@@ -724,13 +741,26 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     __syncwarp();
     // this warp's candidate rows: (candidate, 16-byte piece) pairs over the lanes
     const int q0 = min(wstart, GB), nq = min(wbase, GB) - q0;
+    if constexpr (PAGED) {
+      // 32 candidates at a time: lane l looks up candidate l's row, the pieces take it by shuffle
+      for (int c0 = 0; c0 < nq; c0 += 32) {  // warp-uniform
+        const int qc = min(32, nq - c0);
+        const unsigned long long myrow = lane < qc ? (unsigned long long)slot_of(cand[q0 + c0 + lane]) * D : 0ull;
+        for (int e = lane; e < qc * 2 * RPR; e += 32) {  // 2 * RPR is a multiple of 32: uniform trip count
+          const int qi = e / (2 * RPR), pc = e % (2 * RPR), q = q0 + c0 + qi;
+          const size_t row = (size_t)__shfl_sync(0xffffffffu, myrow, qi);
+          if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kg + row + pc * EPV);
+          else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vg + row + (pc - RPR) * EPV);
+        }
+      }
+    } else {
 #pragma unroll 2
-    for (int e = lane; e < nq * 2 * RPR; e += 32) {
-      const int q = q0 + e / (2 * RPR), pc = e % (2 * RPR);
-      const int t = cand[q];
-      const size_t row = slot_of(t) * D;
-      if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kg + row + pc * EPV);
-      else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vg + row + (pc - RPR) * EPV);
+      for (int e = lane; e < nq * 2 * RPR; e += 32) {
+        const int q = q0 + e / (2 * RPR), pc = e % (2 * RPR);
+        const size_t row = slot_of(cand[q]) * D;
+        if (pc < RPR) ptx::cp_async16(Kr + (size_t)q * D + pc * EPV, Kg + row + pc * EPV);
+        else ptx::cp_async16(Vr + (size_t)q * D + (pc - RPR) * EPV, Vg + row + (pc - RPR) * EPV);
+      }
     }
   }
   gather_commit();  // gather phase 0: the candidates' rows
