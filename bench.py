@@ -465,16 +465,32 @@ def run_gpu(args, wl):
                  "hata_speedup": d_ms / ms_per_step}
         del gd
 
-    # the same step over a paged cache: every layer's K, V and code buffers seen as
-    # pools of 256-token blocks, reached through a random (non-contiguous) block table
+    # the same step over a paged cache: every layer's K, V and codes are rearranged in
+    # place into pools of 256-token blocks placed by a random (non-contiguous) block
+    # table, so the paged step reads the same data and selects the same rows
     paged = None
     bs_p = 256
     if wl.max_seq % bs_p == 0 and H.hata_decode_step_kernel_count(dims, wl.k) == 1:
         max_blocks = wl.max_seq // bs_p
         n_blocks = wl.batch * max_blocks
         gen = torch.Generator().manual_seed(args.seed + 1)
-        btab = torch.randperm(n_blocks, generator=gen).to(torch.int32).reshape(wl.batch, max_blocks).to(dev)
+        perm = torch.randperm(n_blocks, generator=gen)
+        btab = perm.to(torch.int32).reshape(wl.batch, max_blocks).to(dev)
         pool = (n_blocks, wl.n_kv_heads, bs_p)
+        where = perm.to(dev)
+
+        def to_pool(t):  # [B][Hkv][Lmax][X] -> pool blocks, in place
+            X = t.shape[-1]
+            blocks = t.view(wl.batch, wl.n_kv_heads, max_blocks, bs_p, X).permute(0, 2, 1, 3, 4).reshape(
+                n_blocks, wl.n_kv_heads, bs_p, X)
+            out = torch.empty(blocks.shape, dtype=blocks.dtype, device=blocks.device)
+            out[where] = blocks
+            t.view(-1).copy_(out.view(-1))
+
+        for L in layers:
+            for name in ("K", "V", "codes"):
+                to_pool(L[name])
+        torch.cuda.synchronize()
 
         def paged_step(i):
             L = layers[i % R]
