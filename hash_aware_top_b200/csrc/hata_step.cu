@@ -54,6 +54,7 @@ constexpr int kStageBytes = 32768;
 constexpr int kTokCap = 65520;       // max tokens per CTA: u16 scores and u16 cumulative counts
 constexpr int kXS = 36;              // floats per residue row of an encoded vector (32 used, padded)
 constexpr int kMaxCS = 16;           // largest cluster
+constexpr int kPagedBt = 256;        // block-table entries of a CTA's slice kept in shared memory (paged cache)
 constexpr int kMaxGB = 256;          // largest gather batch (rows); below kFThreads: one candidate per thread
 constexpr int kOneCtaSmem = 116 * 1024;  // dynamic shared memory that keeps one CTA per SM
 constexpr uint32_t kWaitTries = 1u << 22;
@@ -221,6 +222,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
   __shared__ float redl[PVG * G];         // per-row-group probability sums
   __shared__ int s_nrow;
   __shared__ __align__(16) int hdr[kMaxCS * 4];  // per source CTA: range [lo, hi) of the histogram bins it sent
+  __shared__ int bt_s[PAGED ? kPagedBt : 1];     // (paged) block numbers of this CTA's slice, from block bt0
 
   const int u = blockIdx.x / CS;
   const int b = u / p.Hkv, g = u % p.Hkv;
@@ -282,9 +284,24 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
     }
     return (((size_t)pb * p.Hkv + g) << p.block_shift) | (size_t)(t & ((1 << p.block_shift) - 1));
   };
+  // (paged) the block numbers of this CTA's slice come from shared memory when the
+  // slice spans at most kPagedBt blocks, else from the table in global memory
+  const int bt0 = PAGED ? (t0 >> p.block_shift) : 0;
+  const int nbt = PAGED && t1 > t0 ? ((t1 - 1) >> p.block_shift) - bt0 + 1 : 0;
+  const bool bt_local = PAGED && nbt <= kPagedBt;
+  if constexpr (PAGED) {
+    if (bt_local) {
+      for (int i = tid; i < nbt; i += kFThreads) bt_s[i] = btab[bt0 + i];
+      __syncthreads();
+    }
+  }
+  auto block_of = [&](int t) -> int {  // (paged) pool block of token t; t in [t0, t1) when bt_local
+    const int i = t >> p.block_shift;
+    return bt_local && i - bt0 >= 0 && i - bt0 < nbt ? bt_s[i - bt0] : btab[i];
+  };
   auto slot_of = [&](int t) -> size_t {
     if constexpr (PAGED) {
-      return phys_slot(btab[t >> p.block_shift], t);
+      return phys_slot(block_of(t), t);
     } else {
       return (size_t)u * p.max_seq + t;
     }
@@ -309,7 +326,7 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
         for (int k = 0; k < 8; ++k) {
           if (x0 < nb) {
             const int t = ts + x0, seg = min(nb - x0, bsz - (t & (bsz - 1)));
-            pbk[k] = btab[t >> p.block_shift];
+            pbk[k] = block_of(t);
             xs[k] = x0;
             sg[k] = seg;
             x0 += seg;
@@ -1163,11 +1180,13 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
     pl.sel_cap = std::min(k, tok_cap);
     pl.nbins = G * d.hash_bits + 1;
     pl.stages = 0;
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) {
+    cudaFuncAttributes fa, fa_paged;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+        cudaFuncGetAttributes(&fa_paged, (const void*)fused_step_kernel<T, NW, G, true>) != cudaSuccess) {
       (void)cudaGetLastError();
       return best;
     }
+    fa.sharedSizeBytes = std::max(fa.sharedSizeBytes, fa_paged.sharedSizeBytes);  // one plan serves both
     for (int st = kMaxStages; st >= kMinStages; --st) {
       const size_t sm = smem_layout(G, NW, esize, tok_cap, pl.sel_cap, pl.nbins, CS, st).total;
       if (sm + fa.sharedSizeBytes <= 227 * 1024) {  // + static shared memory
