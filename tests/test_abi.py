@@ -100,6 +100,33 @@ def test_calls_reject_bad_arguments_before_launch(H):
     assert lib.hata_read_device_status(null, null, ctypes.byref(ctypes.c_int())) == 1
 
 
+def test_separate_encoder_and_paged_calls_reject_bad_arguments(H):
+    """hata_decode_step_qk, hata_decode_step_paged and hata_encode_read_status validate
+    on the host: missing or misaligned matrices and tables, block sizes that are not
+    a power of two in [16, 65536], an empty pool, a null status pointer."""
+    d = H.dims_for(1, 4, 1, 128, 128, 1024, "bf16")
+    P = ctypes.c_void_p
+    fake, odd, null = P(0x1000), P(0x1008), P(0)
+    lib = H.lib
+    f0 = ctypes.c_float(0.0)
+    # qk: W_k missing / misaligned
+    assert lib.hata_decode_step_qk(ctypes.byref(d), fake, fake, fake, fake, null, fake, fake, 4, f0, fake, null,
+                                   null, fake, 1 << 30, null) == 1
+    assert lib.hata_decode_step_qk(ctypes.byref(d), fake, fake, fake, fake, odd, fake, fake, 4, f0, fake, null,
+                                   null, fake, 1 << 30, null) == 1
+
+    def paged(block_table, bs, n_blocks, k=4):
+        return lib.hata_decode_step_paged(ctypes.byref(d), fake, fake, fake, fake, fake, fake, block_table, bs,
+                                          n_blocks, fake, k, f0, fake, null, null, fake, 1 << 30, null)
+
+    assert paged(null, 64, 16) == 1          # no block table
+    for bs in (0, 8, 15, 24, 100, 1 << 17):  # not a power of two in [16, 65536]
+        assert paged(fake, bs, 16) == 1, bs
+    assert paged(fake, 64, 0) == 1           # empty pool
+    assert paged(fake, 64, 16, k=0) == 1     # k < 1
+    assert lib.hata_encode_read_status(null, None) == 1
+
+
 def test_binding_refuses_cpu_tensors(H):
     import torch
 
