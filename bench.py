@@ -171,6 +171,23 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(value, dist, device):
+    """The largest value over all ranks (the duration of the slowest replica); `dist`
+    is torch.distributed when the process group is up, else None (one rank)."""
+    if dist is None:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, steps, seconds):
+    """Whole-job steps/s: every replica ran `steps` steps; the job took the slowest one's time."""
+    return world * steps / seconds
+
+
 def workload_config(wl, seq_lens, l2_note):
     return {
         "workload": wl.name,
@@ -382,16 +399,14 @@ def run_gpu(args, wl):
     # plausibility: the same graph timed with events recorded inside the replay stream's own order
     if ms / args.steps < 1e-4:
         raise RuntimeError(f"implausible step time {ms / args.steps * 1e3:.3f} us")
+    ms = max_over_ranks(ms, dist, dev)
     if dist:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     status = H.hata_read_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}: {H.hata_status_string(status)}")
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = job_throughput(world, args.steps, ms / 1e3)
 
     # end to end through the public call: pinned host inputs in, output read back, every step
     e2e_steps = min(args.steps, 300)
@@ -406,9 +421,12 @@ def run_gpu(args, wl):
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    t0 = time.perf_counter()
     kv_stage = torch.empty(kv_host.shape, dtype=kv_host.dtype, device=dev)
+    # timed on the device: events on the stream around the loop; every step waits for its
+    # result on the host, so the host side of each step lies inside the interval
+    e_e2e0, e_e2e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
+        e_e2e0.record(stream)
         for i in range(e2e_steps):
             L = layers[i % R]
             L["q"].copy_(q_host, non_blocking=True)
@@ -420,12 +438,10 @@ def run_gpu(args, wl):
             step(i)
             out_host.copy_(L["out"], non_blocking=True)
             stream.synchronize()
-    e2e_s = time.perf_counter() - t0
-    if dist:
-        t = torch.tensor([e2e_s], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_s = float(t.item())
-    e2e_value = world * e2e_steps / e2e_s
+        e_e2e1.record(stream)
+        e_e2e1.synchronize()
+    e2e_s = max_over_ranks(e_e2e0.elapsed_time(e_e2e1) / 1e3, dist, dev)
+    e2e_value = job_throughput(world, e2e_steps, e2e_s)
 
     # the dense flash-decode baseline on the same layer buffers (the comparison the pages report)
     dense = None
