@@ -12,7 +12,7 @@
 // product, so a code bit can differ from the exact sign only where |y| is within
 // fp32 rounding of zero.
 //
-// One CTA of four warps per SM, persistent over the 128-key tiles of one
+// One CTA of five warps per SM, persistent over the 128-key tiles of one
 // (batch, head):
 //   * W_H^T (three parts, r x 128 each) sits in shared memory in the K-major
 //     core-matrix layout the tensor core reads without swizzling: 8 rows x 16
@@ -23,15 +23,15 @@
 //     swizzle: the K-major layout with 1024-byte 8-row groups that the tensor
 //     core reads directly), S tiles in flight, each completing on its stage's
 //     mbarrier;
-//   * one thread issues the tile's MMAs (M = 128 keys, K = 16 each, kind::f16
-//     with bf16 inputs and fp32 accumulation; for r <= 64 one MMA of N = 3r per K
-//     step over the three stacked parts, for r = 128 three of N = r) into one of two TMEM
-//     accumulators, commits them to an mbarrier, and refills a stage as soon as
-//     the MMAs reading it are done;
-//   * the four warps read the previous tile's accumulator (warp w owns TMEM lanes
-//     32w .. 32w + 31, i.e. keys), turn 32 columns at a time into a code word,
-//     store each key's code as one vector and release the accumulator on a
-//     128-thread mbarrier.  No CTA-wide barrier inside the loop.
+//   * warp 4 (one lane) issues the tile's MMAs (M = 128 keys, K = 16 each,
+//     kind::f16 with bf16 inputs and fp32 accumulation; for r <= 64 one MMA of
+//     N = 3r per K step over the three stacked parts, for r = 128 three of N = r)
+//     into one of two TMEM accumulators, commits them to an mbarrier, and refills
+//     a stage as soon as the MMAs reading it are done;
+//   * warps 0-3 read each finished accumulator (warp w owns TMEM lanes
+//     32w .. 32w + 31, i.e. keys), add the parts, turn 32 columns at a time into
+//     a code word, store each key's code as one vector and release the
+//     accumulator on a 128-thread mbarrier.  No CTA-wide barrier inside the loop.
 // Every wait is bounded: on expiry the kernel records HATA_ERR_TIMEOUT in the
 // library's encode status word (hata_encode_read_status), stops issuing work,
 // waits (bounded) for the MMAs it issued, frees its TMEM and returns.

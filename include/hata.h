@@ -126,9 +126,12 @@ HATA_API hata_status_t hata_workspace_init(void* workspace, size_t workspace_byt
  * Typical uses: query codes (x = q, x_heads = Hq, x_len = codes_len = 1,
  * n_tok = 1, seq_end = NULL); appending the new key (x = K, x_heads = Hkv,
  * x_len = codes_len = max_seq, n_tok = 1, seq_end = seq_lens); prefill
- * (same with n_tok = max_seq).  The projection is fp32 FMA in a fixed order
- * (for n_tok <= 4 the same order as hata_decode_step, so both give the same
- * codes bit for bit).
+ * (same with n_tok = max_seq).  For n_tok <= 4 the projection is fp32 FMA in
+ * the same fixed order as hata_decode_step, so both give the same codes bit for
+ * bit.  The prefill form of bf16 keys with r <= 128 runs on the tensor cores
+ * with W_H split into three bf16 parts (exact products, fp32 accumulation in
+ * another order); other prefill forms are fp32 FMA.  Codes of the different
+ * forms can differ only where |x . W_H| is within fp32 rounding of zero.
  */
 HATA_API hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_heads, int x_len, int n_tok,
                                  const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,

@@ -16,6 +16,9 @@ Hash-Aware Top-k Attention for Scalable Large Model Inference", ACL 2025):
     (§Decode 阶段算法 and §关键发现 "GQA 兼容"); the aggregate is a sum;
   * top-k select, gather the chosen K/V rows, exact attention on them
     (§Decode 阶段算法; §整体框架 decode phase).
+The separate key encoder of decode_step (W_k) follows "HashAttention: Semantic
+Sparsity for Faster Inference" (AI summary, Approach: independent key and query
+mappings into Hamming space, pivotal tokens by XOR + popcount).
 
 Readings where the pages are silent (each is listed in the design notes):
   * bit j of a code is [y_j > 0] (y = x W_H); bit j lives in 32-bit word j // 32
