@@ -2,20 +2,21 @@
 // written straight into the code cache ("HATA" paper notes, 硬件高效优化:
 // projection -> sign -> bitpack -> cache update fused in one kernel).
 //
-// Two forms, chosen by the number of tokens per sequence:
+// Three forms, chosen by the number of tokens per sequence and the key type:
 //   * decode form (n_tok <= kDecodeTok): the few rows of a call (G query heads,
 //     or one new key per KV head) are latency-bound, so the work is spread over
 //     one CTA per (32-column word, KV group, batch).  Each CTA stages its rows
 //     and its 32 columns of W_H (transposed) in shared memory and every (row,
 //     column) projection is one warp_dot128 -- the same arithmetic as the fused
 //     decode step, so both paths produce identical codes.
-//   * prefill form, bf16 keys and r <= 128: the tensor-core kernel of
-//     hata_encode_mma.cu (W_H split in three bf16 parts, fp32 accumulation);
+//   * prefill form, bf16 keys and r <= 128: the tcgen05 tensor-core kernel of
+//     hata_encode_tc.cu (W_H split in three bf16 parts, fp32 accumulation), or
+//     the mma.sync kernel of hata_encode_mma.cu when no TMA tensor map can be made;
 //   * prefill form otherwise: each CTA owns one (batch, KV group) and a tile of 32 rows;
 //     thread (slice s, column j) accumulates y_j for rows s, s + NS, ... with
 //     fp32 FMAs in ascending i, reading W_H[g][i][j] coalesced along j; the sign
 //     bits of 32 consecutive columns are one warp ballot, i.e. one packed word.
-// The two forms round differently, so a key encoded by both can differ only in
+// The forms round differently, so a key encoded by two of them can differ only in
 // bits whose projection is within fp32 rounding of zero.
 #include "hata_kernels.cuh"
 

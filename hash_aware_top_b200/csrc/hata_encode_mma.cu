@@ -1,4 +1,6 @@
-// Prefill HashEncode on the tensor cores: y = x . W_H for every cached key,
+// Prefill HashEncode on the legacy tensor-core path (mma.sync), the fallback of
+// the tcgen05 kernel in hata_encode_tc.cu when no TMA tensor map can be made:
+// y = x . W_H for every cached key,
 // bit = [y > 0], LSB-first pack, written into the code cache ("HATA" paper notes,
 // 硬件高效优化: projection -> sign -> bitpack -> cache update in one kernel; this
 // is the one genuinely dense contraction of the method, [L x 128] x [128 x r]).
