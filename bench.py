@@ -188,7 +188,11 @@ def job_throughput(world, steps, seconds):
     return world * steps / seconds
 
 
-def workload_config(wl, seq_lens, l2_note):
+L2_NOTE = "inputs larger than L2: steps rotate over layer buffers holding more than 4x the L2 size"
+
+
+def workload_config(wl, seq_lens):
+    """The workload's identity, the same in both arms (arm-specific timing details go under "timing")."""
     return {
         "workload": wl.name,
         "batch": wl.batch,
@@ -200,7 +204,7 @@ def workload_config(wl, seq_lens, l2_note):
         "hash_bits": wl.hash_bits,
         "top_k": wl.k,
         "kv_dtype": wl.dtype,
-        "l2": l2_note,
+        "l2": L2_NOTE,
         "parallelism": "replicas",
     }
 
@@ -209,51 +213,98 @@ def workload_config(wl, seq_lens, l2_note):
 # reference arm: the CPU oracle on this host
 # ----------------------------------------------------------------------------
 
-def oracle_unit_runner(wl, inp):
-    """Returns (run(unit), n_units): run one (batch, KV head) unit of the decode step through the oracle."""
-    import oracle
-
-    G = wl.group
-    units = [(b, g) for b in range(wl.batch) for g in range(wl.n_kv_heads)]
-    prepared = {}
-
-    def prep(u):
-        b, g = units[u % len(units)]
-        if (b, g) not in prepared:
-            Lb = int(inp["seq_lens"][b])
-            K = inp["K"][b:b + 1, g:g + 1]
-            codes, _ = oracle.encode_cache(K, inp["W_H"][g:g + 1], np.array([Lb]))
-            prepared[(b, g)] = (inp["q"][b:b + 1, g * G:(g + 1) * G], K, inp["V"][b:b + 1, g:g + 1],
-                                inp["W_H"][g:g + 1], codes, np.array([Lb]))
-        return prepared[(b, g)]
-
-    def run(u):
-        q, K, V, W, codes, lens = prep(u)
-        t0 = time.perf_counter()
-        oracle.decode_step(q, K, V, W, codes, lens, wl.k)
-        return time.perf_counter() - t0
-
-    return run, prep, len(units)
+# The oracle's (batch, KV head) units of one decode step are independent, so the
+# all-core legs spread them over a process pool.  The pool is forked before any
+# CUDA call of this process (a fork after CUDA is initialised is unsafe), and its
+# workers read the inputs that the parent made (copy-on-write).
+_ORACLE_JOB = None  # (wl, inp, codes) for the pool's workers
+_LIMITS = None
 
 
-def cpu_baseline(wl, inp, budget_s=15.0, max_units=None):
+def _worker_init():
+    global _LIMITS
     from threadpoolctl import threadpool_limits
 
-    with threadpool_limits(1):
-        run, prep, n_units = oracle_unit_runner(wl, inp)
+    _LIMITS = threadpool_limits(1)  # one BLAS thread per worker process
+
+
+def _oracle_unit(u):
+    """One unit of the decode step through the oracle; returns its duration in seconds."""
+    import oracle
+
+    wl, inp, codes = _ORACLE_JOB
+    b, g = divmod(u % (wl.batch * wl.n_kv_heads), wl.n_kv_heads)
+    G = wl.group
+    Lb = np.array([int(inp["seq_lens"][b])])
+    t0 = time.perf_counter()
+    oracle.decode_step(inp["q"][b:b + 1, g * G:(g + 1) * G], inp["K"][b:b + 1, g:g + 1], inp["V"][b:b + 1, g:g + 1],
+                       inp["W_H"][g:g + 1], codes[b:b + 1, g:g + 1], Lb, wl.k)
+    return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+class OraclePool:
+    """The CPU oracle over whole decode steps on `cores` worker processes."""
+
+    def __init__(self, wl, inp, cores):
+        import multiprocessing
+
+        import oracle
+
+        global _ORACLE_JOB
+        codes, _ = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"])  # the cache before the step
+        _ORACLE_JOB = (wl, inp, codes)
+        self.units = wl.batch * wl.n_kv_heads
+        self.cores = cores
+        self.pool = multiprocessing.get_context("fork").Pool(cores, initializer=_worker_init)
+
+    def run_steps(self, n_steps):
+        """Wall-clock seconds for n_steps whole steps (all their units queued at once)."""
+        t0 = time.perf_counter()
+        self.pool.map(_oracle_unit, range(n_steps * self.units), chunksize=1)
+        return time.perf_counter() - t0
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def cpu_baseline(wl, inp, budget_s=12.0):
+    """The oracle on this host's cores, before any CUDA call: whole steps over all cores
+    (the reported value), plus one thread on a bounded sample of units."""
+    from threadpoolctl import threadpool_limits
+
+    cores = host_cores()
+    pool = OraclePool(wl, inp, cores)
+    try:
+        # one thread: units in order until the budget is spent
         elapsed, done = 0.0, 0
-        limit = n_units if max_units is None else min(max_units, n_units)
-        while done < limit and (elapsed < budget_s or done == 0):
-            prep(done)
-            elapsed += run(done)
-            done += 1
-    steps_per_s = (done / n_units) / elapsed
+        with threadpool_limits(1):
+            while done < pool.units and (elapsed < budget_s or done == 0):
+                elapsed += _oracle_unit(done)
+                done += 1
+        single = (done / pool.units) / elapsed
+        # all cores: enough whole steps for about budget_s of wall time
+        per_unit = elapsed / done
+        n_steps = max(1, min(200, math.ceil(budget_s * cores / (per_unit * pool.units))))
+        wall = pool.run_steps(n_steps)
+    finally:
+        pool.close()
     return {
-        "value": steps_per_s,
+        "value": n_steps / wall,
         "unit": "steps/s",
-        "cores": 1,
+        "cores": cores,
         "kind": "oracle",
-        "sample": f"{done} of {n_units} (batch, KV head) units of one decode step, float64 numpy, 1 thread",
+        "sample": f"{n_steps} whole decode steps ({n_steps * pool.units} (batch, KV head) units) over {cores} "
+                  "worker processes, one thread each, float64 numpy",
+        "single_thread": {"value": single, "unit": "steps/s", "cores": 1,
+                          "sample": f"{done} of {pool.units} units of one step, value scaled to whole steps"},
     }
 
 
@@ -262,19 +313,14 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     inp = make_inputs(wl, seed=args.seed)
-    from threadpoolctl import threadpool_limits
-
-    with threadpool_limits(1):
-        run, prep, n_units = oracle_unit_runner(wl, inp)
-        for u in range(args.warmup):
-            prep(u)
-            run(u)
-        times = []
-        for u in range(args.steps):
-            prep(u)
-            times.append(run(u))
-    total = sum(times)
-    value = (args.steps / n_units) / total
+    cores = host_cores()
+    pool = OraclePool(wl, inp, cores)
+    try:
+        pool.run_steps(args.warmup)
+        wall = pool.run_steps(args.steps)
+    finally:
+        pool.close()
+    value = args.steps / wall
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -283,17 +329,19 @@ def run_reference(args, wl):
         "n_gpus": args.gpus,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": 1e3 / value,
+        "ms_per_step": 1e3 * wall / args.steps,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": workload_config(wl, inp["seq_lens"], "host CPU"),
+        "config": workload_config(wl, inp["seq_lens"]),
+        "timing": {"arm": "CPU oracle, whole decode steps, wall clock",
+                   "units_per_step": wl.batch * wl.n_kv_heads, "worker_processes": cores},
         "cpu_baseline": {
-            "value": value, "unit": "steps/s", "cores": 1, "kind": "oracle",
-            "sample": f"each step = one of {n_units} (batch, KV head) units of one decode step; "
-                      "value scaled to whole steps",
+            "value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{args.steps} whole decode steps after {args.warmup} warm-up steps, every (batch, KV head) "
+                      f"unit queued on {cores} worker processes, one thread each",
         },
         "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -305,10 +353,120 @@ def run_reference(args, wl):
 # GPU arm
 # ----------------------------------------------------------------------------
 
-def run_gpu(args, wl):
+def graph_upload(g, stream):
+    """Upload an instantiated graph to the device before it is timed, so that the first
+    timed replay does not pay for it (driver call cuGraphUpload on the graph's exec handle)."""
+    import ctypes
+
+    try:
+        cuda = ctypes.CDLL("libcuda.so.1")
+        cuda.cuGraphUpload.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        rc = cuda.cuGraphUpload(ctypes.c_void_p(int(g.raw_cuda_graph_exec())), ctypes.c_void_p(stream.cuda_stream))
+        return rc == 0
+    except (OSError, AttributeError, RuntimeError):
+        return False
+
+
+def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
+    """Milliseconds for `steps` calls of step(i) replayed from CUDA graphs, after `warmup`
+    replayed steps: CUDA events on the launching stream, a synchronize (and a barrier
+    across ranks) on both sides."""
+    import contextlib
+
     import torch
 
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                step(i)
+        return g
+
+    with torch.cuda.stream(stream):
+        for i in range(3):  # eager calls before capture (first-launch setup)
+            step(i)
+    torch.cuda.synchronize()
+    chunk = min(steps, GRAPH_CHUNK)
+    g_chunk = capture(chunk)
+    rem = steps % chunk
+    g_rem = capture(rem) if rem else None
+    g_warm = capture(warmup)
+    for g in (g_chunk, g_rem, g_warm):
+        if g is not None:
+            graph_upload(g, stream)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):  # graph replays go to torch's current stream: the timed one
+        g_warm.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with (sampler or contextlib.nullcontext()), torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(steps // chunk):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+        ev1.synchronize()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if ms / steps < 1e-4:
+        raise RuntimeError(f"implausible step time {ms / steps * 1e3:.3f} us")
+    del g_chunk, g_rem, g_warm
+    return ms
+
+
+class LayerSet:
+    """R copies ("layers") of one workload's device buffers, so that consecutive steps read
+    different memory and the bytes touched per rotation exceed 4x the L2 size."""
+
+    def __init__(self, H, wl, inp, dev, layers=None):
+        import torch
+
+        self.wl, self.inp = wl, inp
+        self.tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        self.dims = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.hash_bits, wl.max_seq,
+                               wl.dtype)
+        self.step_bytes = algorithmic_bytes(wl, inp["seq_lens"])
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.R = max(2, math.ceil(4 * l2 / self.step_bytes)) if layers is None else layers
+        self.l2 = l2
+
+        def to_dev(a):
+            return torch.from_numpy(a).to(dev).to(self.tdt)
+
+        base = {"q": to_dev(inp["q"]), "K": to_dev(inp["K"]), "V": to_dev(inp["V"]),
+                "W": torch.from_numpy(inp["W_H"]).to(dev), "lens": torch.from_numpy(inp["seq_lens"]).to(dev)}
+        self.ws = torch.empty(H.hata_workspace_size(self.dims, wl.k), dtype=torch.uint8, device=dev)
+        H.hata_workspace_init(self.ws)
+        # prefill: encode every cached key through the library
+        codes0 = torch.zeros((wl.batch, wl.n_kv_heads, wl.max_seq, wl.words), dtype=torch.int32, device=dev)
+        H.hata_encode_append(self.dims, base["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, base["lens"], base["W"],
+                             codes0, wl.max_seq, self.ws)
+        self.layers = []
+        for i in range(self.R):
+            lay = {n: (t if i == 0 else t.clone()) for n, t in base.items()}
+            lay["codes"] = codes0 if i == 0 else codes0.clone()
+            lay["out"] = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=self.tdt, device=dev)
+            self.layers.append(lay)
+        torch.cuda.synchronize()
+
+    def timing_note(self):
+        return {"layer_buffers": self.R, "mb_touched_per_rotation": round(self.R * self.step_bytes / 1e6),
+                "l2_mb": round(self.l2 / 1e6)}
+
+
+def run_gpu(args, wl):
     world, rank, local = dist_env()
+    inp = make_inputs(wl, seed=args.seed)
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, inp)  # before the first CUDA call of this process (forked pool)
+
+    import torch
+
     torch.cuda.set_device(local)
     dist = None
     if world > 1:
@@ -322,83 +480,17 @@ def run_gpu(args, wl):
     import hash_aware_top_b200 as H
 
     dev = torch.device("cuda", local)
-    inp = make_inputs(wl, seed=args.seed)
-    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-    dims = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.hash_bits, wl.max_seq, wl.dtype)
-    step_bytes = algorithmic_bytes(wl, inp["seq_lens"])
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    R = max(2, math.ceil(4 * l2 / step_bytes)) if args.layers is None else args.layers
-
-    def to_dev(a):
-        return torch.from_numpy(a).to(dev).to(tdt)
-
-    base = {
-        "q": to_dev(inp["q"]), "K": to_dev(inp["K"]), "V": to_dev(inp["V"]),
-        "W": torch.from_numpy(inp["W_H"]).to(dev),
-        "lens": torch.from_numpy(inp["seq_lens"]).to(dev),
-    }
-    ws = torch.empty(H.hata_workspace_size(dims, wl.k), dtype=torch.uint8, device=dev)
-    H.hata_workspace_init(ws)
-    # prefill: encode every cached key through the library
-    codes0 = torch.zeros((wl.batch, wl.n_kv_heads, wl.max_seq, wl.words), dtype=torch.int32, device=dev)
-    H.hata_encode_append(dims, base["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, base["lens"], base["W"], codes0,
-                         wl.max_seq)
-    layers = []
-    for i in range(R):
-        lay = {n: (t if i == 0 else t.clone()) for n, t in base.items()}
-        lay["codes"] = codes0 if i == 0 else codes0.clone()
-        lay["out"] = torch.empty((wl.batch, wl.n_q_heads, wl.head_dim), dtype=tdt, device=dev)
-        layers.append(lay)
-    torch.cuda.synchronize()
-
     stream = torch.cuda.Stream(device=dev)
+    ls = LayerSet(H, wl, inp, dev, args.layers)
+    dims, R, layers, ws, step_bytes = ls.dims, ls.R, ls.layers, ls.ws, ls.step_bytes
 
     def step(i):
         L = layers[i % R]
         H.hata_decode_step(dims, L["q"], L["K"], L["V"], L["W"], L["codes"], L["lens"], wl.k, 0.0, L["out"], None,
                            None, ws, stream)
 
-    def capture(n, first):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                step(first + i)
-        return g
-
-    with torch.cuda.stream(stream):
-        for i in range(3):  # eager calls before capture (first-launch setup)
-            step(i)
-    torch.cuda.synchronize()
-    chunk = min(args.steps, GRAPH_CHUNK)
-    g_chunk = capture(chunk, 0)
-    rem = args.steps % chunk
-    g_rem = capture(rem, 0) if rem else None
-    g_warm = capture(args.warmup, 0) if args.warmup else None
-    torch.cuda.synchronize()
-
-    # graph replays are launched on torch's current stream: make it the stream the events are recorded on
-    with torch.cuda.stream(stream):
-        if g_warm is not None:
-            g_warm.replay()
-    torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
-    with sampler, torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(args.steps // chunk):
-            g_chunk.replay()
-        if g_rem is not None:
-            g_rem.replay()
-        ev1.record(stream)
-        ev1.synchronize()
-    torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    # plausibility: the same graph timed with events recorded inside the replay stream's own order
-    if ms / args.steps < 1e-4:
-        raise RuntimeError(f"implausible step time {ms / args.steps * 1e3:.3f} us")
+    ms = graph_time(step, args.steps, args.warmup, stream, dist, sampler)
     ms = max_over_ranks(ms, dist, dev)
     if dist:
         dist.barrier()
@@ -407,7 +499,6 @@ def run_gpu(args, wl):
         raise RuntimeError(f"device status {status}: {H.hata_status_string(status)}")
     ms_per_step = ms / args.steps
     value = job_throughput(world, args.steps, ms / 1e3)
-
     # end to end through the public call: pinned host inputs in, output read back, every step
     e2e_steps = min(args.steps, 300)
     L0 = layers[0]
@@ -453,40 +544,51 @@ def run_gpu(args, wl):
             H.hata_dense_decode(dims, L["q"], L["K"], L["V"], L["lens"], 0.0, L["out"], dws, stream)
 
         d_steps = min(args.steps, 2000)
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                dense_step(i)
-        torch.cuda.synchronize()
-        gd = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gd, stream=stream):
-            for i in range(min(d_steps, GRAPH_CHUNK)):
-                dense_step(i)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            gd.replay()  # warm-up
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            reps = max(1, d_steps // min(d_steps, GRAPH_CHUNK))
-            for _ in range(reps):
-                gd.replay()
-            e1.record(stream)
-            e1.synchronize()
-        d_ms = e0.elapsed_time(e1) / (reps * min(d_steps, GRAPH_CHUNK))
+        d_ms = graph_time(dense_step, d_steps, args.warmup, stream) / d_steps
         d_bytes = sum(2 * int(Lb) * wl.n_kv_heads * wl.head_dim * 2 for Lb in inp["seq_lens"]) + \
             2 * wl.batch * wl.n_q_heads * wl.head_dim * 2
-        dense = {"kernel": "hata_dense_decode (dense flash-decode, bf16 tensor-core tiles)",
+        dense = {"kernel": "hata_dense_decode (dense flash-decode, bf16 tensor-core tiles)", "steps": d_steps,
                  "us_per_step": d_ms * 1e3, "bytes_per_step": d_bytes,
                  "achieved_gbs": d_bytes / (d_ms * 1e-3) / 1e9,
                  "hata_speedup": d_ms / ms_per_step}
-        del gd
+
+    # prefill encode (hata_encode_append over every cached key of every layer buffer)
+    pre_reps = max(2, min(R, 8))
+    with torch.cuda.stream(stream):
+        H.hata_encode_append(dims, layers[0]["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, layers[0]["lens"],
+                             layers[0]["W"], layers[0]["codes"], wl.max_seq, ws, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(pre_reps):
+            L = layers[i % R]
+            H.hata_encode_append(dims, L["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L["lens"], L["W"], L["codes"],
+                                 wl.max_seq, ws, stream)
+        e1.record(stream)
+        e1.synchronize()
+    pre_ms = e0.elapsed_time(e1) / pre_reps
+    n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
+    pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + wl.hash_bits // 8)
+    prefill = {"kernel": "hata_encode_append (prefill form; bf16 keys: tcgen05 tensor cores)",
+               "us_per_call": pre_ms * 1e3, "keys": n_keys,
+               "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
+               "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
+               "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
+    if wl.dtype == "bf16" and wl.hash_bits <= 128:
+        # the tensor cores run W_H as three bf16 parts: 3x the algorithmic flops
+        prefill["mma_tflops"] = 3.0 * prefill["tflops"]
+        tpeak = tensor_peak_bf16()
+        if tpeak:
+            prefill["frac_of_tensor_peak"] = prefill["mma_tflops"] / tpeak
+    if H.hata_read_device_status(ws) != 0:
+        raise RuntimeError("device status set by the prefill encode")
 
     # the same step over a paged cache: every layer's K, V and codes are rearranged in
     # place into pools of 256-token blocks placed by a random (non-contiguous) block
     # table, so the paged step reads the same data and selects the same rows
     paged = None
     bs_p = 256
-    if wl.max_seq % bs_p == 0 and H.hata_decode_step_kernel_count(dims, wl.k) == 1:
+    if wl.max_seq % bs_p == 0 and H.hata_decode_step_kernel_count(dims, wl.k) >= 1:
         max_blocks = wl.max_seq // bs_p
         n_blocks = wl.batch * max_blocks
         gen = torch.Generator().manual_seed(args.seed + 1)
@@ -515,65 +617,44 @@ def run_gpu(args, wl):
                                      0.0, L["out"], None, None, ws, stream)
 
         p_steps = min(args.steps, 2000)
-        with torch.cuda.stream(stream):
-            for i in range(3):
-                paged_step(i)
-        torch.cuda.synchronize()
-        gp = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gp, stream=stream):
-            for i in range(min(p_steps, GRAPH_CHUNK)):
-                paged_step(i)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(stream):
-            gp.replay()  # warm-up
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            reps = max(1, p_steps // min(p_steps, GRAPH_CHUNK))
-            for _ in range(reps):
-                gp.replay()
-            e1.record(stream)
-            e1.synchronize()
-        p_ms = e0.elapsed_time(e1) / (reps * min(p_steps, GRAPH_CHUNK))
-        paged = {"kernel": "hata_decode_step_paged (256-token blocks, random block table)",
+        p_ms = graph_time(paged_step, p_steps, args.warmup, stream) / p_steps
+        paged = {"kernel": "hata_decode_step_paged (256-token blocks, random block table)", "steps": p_steps,
                  "us_per_step": p_ms * 1e3, "achieved_gbs": step_bytes / (p_ms * 1e-3) / 1e9,
                  "vs_unpaged": ms_per_step / p_ms}
-        del gp
-
-    # prefill encode (hata_encode_append over every cached key of every layer buffer)
-    pre_reps = max(2, min(R, 8))
-    with torch.cuda.stream(stream):
-        H.hata_encode_append(dims, layers[0]["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, layers[0]["lens"],
-                             layers[0]["W"], layers[0]["codes"], wl.max_seq, stream)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(pre_reps):
-            L = layers[i % R]
-            H.hata_encode_append(dims, L["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L["lens"], L["W"], L["codes"],
-                                 wl.max_seq, stream)
-        e1.record(stream)
-        e1.synchronize()
-    pre_ms = e0.elapsed_time(e1) / pre_reps
-    n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
-    pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + wl.hash_bits // 8)
-    prefill = {"kernel": "hata_encode_append (prefill form; bf16 keys: tcgen05 tensor cores)",
-               "us_per_call": pre_ms * 1e3, "keys": n_keys,
-               "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
-               "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
-               "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
-    if wl.dtype == "bf16" and wl.hash_bits <= 128:
-        # the tensor cores run W_H as three bf16 parts: 3x the algorithmic flops
-        prefill["mma_tflops"] = 3.0 * prefill["tflops"]
-        tpeak = tensor_peak_bf16()
-        if tpeak:
-            prefill["frac_of_tensor_peak"] = prefill["mma_tflops"] / tpeak
+    timing = ls.timing_note()
+    del ls, layers
+    torch.cuda.empty_cache()
 
     peak, peak_kind = peak_hbm()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     prefill["frac_of_peak"] = prefill["achieved_gbs"] / peak
     if dense is not None:
         dense["frac_of_peak"] = dense["achieved_gbs"] / peak
+
+    # the other context lengths the metric names (32K-128K): the same step, timed the same way
+    workloads = {}
+    for name in (args.also or []):
+        if name == wl.name:
+            continue
+        wl2 = WORKLOADS[name]
+        ls2 = LayerSet(H, wl2, make_inputs(wl2, seed=args.seed), dev)
+
+        def step2(i, ls2=ls2):
+            L = ls2.layers[i % ls2.R]
+            H.hata_decode_step(ls2.dims, L["q"], L["K"], L["V"], L["W"], L["codes"], L["lens"], wl2.k, 0.0,
+                               L["out"], None, None, ls2.ws, stream)
+
+        n2 = min(args.steps, 2000)
+        ms2 = graph_time(step2, n2, args.warmup, stream) / n2
+        if H.hata_read_device_status(ls2.ws) != 0:
+            raise RuntimeError(f"device status set on workload {name}")
+        gbs2 = ls2.step_bytes / (ms2 * 1e-3) / 1e9
+        workloads[name] = {"steps": n2, "us_per_step": ms2 * 1e3, "steps_per_s": 1e3 / ms2,
+                           "algorithmic_bytes_per_step": ls2.step_bytes, "achieved_gbs": gbs2,
+                           "frac": gbs2 / peak, **ls2.timing_note()}
+        del ls2
+        torch.cuda.empty_cache()
+
     line = {
         "metric": METRIC,
         "value": value,
@@ -587,10 +668,8 @@ def run_gpu(args, wl):
         "vs_baseline": None,
         "dtype": wl.dtype,
         "data": "synthetic",
-        "config": workload_config(
-            wl, inp["seq_lens"],
-            f"inputs larger than L2: steps rotate over {R} layer buffers, {R * step_bytes / 1e6:.0f} MB touched "
-            f"per rotation vs {l2 / 1e6:.0f} MB L2"),
+        "config": workload_config(wl, inp["seq_lens"]),
+        "timing": timing,
         "roofline": {
             "bound": "hbm",
             "kernel": "hata_decode_step (whole step)",
@@ -605,13 +684,14 @@ def run_gpu(args, wl):
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
         "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
+        "workloads": workloads,
         "dense_baseline": dense,
         "paged_step": paged,
         "prefill_encode": prefill,
         "clocks": sampler.summary(),
     }
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(wl, inp)
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -630,7 +710,11 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=None, help="layer buffers to rotate over (default: > 4x L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--also", nargs="*", default=None,
+                    help="other workloads timed in the same run (default: llama8b_32k beside the 128K headline)")
     args = ap.parse_args(argv)
+    if args.also is None:
+        args.also = ["llama8b_32k"] if args.workload == "llama8b_128k" else []
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     wl = WORKLOADS[args.workload]

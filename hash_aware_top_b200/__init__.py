@@ -27,7 +27,6 @@ __all__ = [
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_encode_append",
-    "hata_encode_read_status",
     "hata_hamming_scores",
     "hata_topk",
     "hata_topk_noalloc",
@@ -56,7 +55,6 @@ EXPORTED_SYMBOLS = (
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_encode_append",
-    "hata_encode_read_status",
     "hata_hamming_scores",
     "hata_topk",
     "hata_sparse_decode",
@@ -113,7 +111,7 @@ def _load():
     sig = {
         "hata_workspace_size": (I, [DP, I, ctypes.POINTER(S)]),
         "hata_workspace_init": (I, [P, S, P]),
-        "hata_encode_append": (I, [DP, P, I, I, I, P, P, P, I, P]),
+        "hata_encode_append": (I, [DP, P, I, I, I, P, P, P, I, P, S, P]),
         "hata_hamming_scores": (I, [DP, P, P, P, P, P]),
         "hata_topk": (I, [DP, P, P, I, P, P, P, S, P]),
         "hata_sparse_decode": (I, [DP, P, P, P, P, I, F, P, P, S, P]),
@@ -121,7 +119,6 @@ def _load():
         "hata_decode_step_qk": (I, [DP, P, P, P, P, P, P, P, I, F, P, P, P, P, S, P]),
         "hata_decode_step_paged": (I, [DP, P, P, P, P, P, P, P, I, I, P, I, F, P, P, P, P, S, P]),
         "hata_read_device_status": (I, [P, P, ctypes.POINTER(I)]),
-        "hata_encode_read_status": (I, [P, ctypes.POINTER(I)]),
         "hata_status_string": (ctypes.c_char_p, [I]),
         "hata_version": (I, []),
         "hata_decode_step_kernel_count": (I, [DP, I]),
@@ -206,8 +203,11 @@ def hata_workspace_init(ws: torch.Tensor, stream=None):
            "hata_workspace_init")
 
 
-def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len, stream=None):
-    """x holds [B][x_heads][x_len][d] elements and codes [B][x_heads][codes_len][r/32] words (any view)."""
+def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len, ws, stream=None):
+    """x holds [B][x_heads][x_len][d] elements and codes [B][x_heads][codes_len][r/32] words (any view).
+
+    ws is a uint8 device workspace (at least 16 bytes; a decode-step workspace serves) whose status word
+    receives device-side errors; read it with hata_read_device_status."""
     d = dims
     _check(
         lib.hata_encode_append(
@@ -217,7 +217,7 @@ def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes
             _ptr(seq_end, "seq_end", (d.batch,), torch.int32, optional=True),
             _ptr(W_H, "W_H", (d.n_kv_heads, d.head_dim, d.hash_bits), torch.float32),
             _ptr(codes, "codes", dtype=_codes_dtype(codes), numel=d.batch * x_heads * codes_len * d.words),
-            int(codes_len), _stream(stream)),
+            int(codes_len), _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_encode_append")
 
 
@@ -361,12 +361,6 @@ def hata_decode_step_paged(dims: Dims, q, K_pool, V_pool, W_q, W_k, codes_pool, 
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step_paged")
-
-
-def hata_encode_read_status(stream=None) -> int:
-    v = ctypes.c_int(0)
-    _check(lib.hata_encode_read_status(_stream(stream), ctypes.byref(v)), "hata_encode_read_status")
-    return v.value
 
 
 def hata_read_device_status(ws, stream=None) -> int:

@@ -12,22 +12,6 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-hata_status_t check_dims(const hata_dims_t* d) {
-  if (!d) return HATA_ERR_INVALID_ARG;
-  if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->max_seq < 1 || d->head_dim < 1 ||
-      d->hash_bits < 1)
-    return HATA_ERR_INVALID_ARG;
-  if (d->n_q_heads % d->n_kv_heads) return HATA_ERR_INVALID_ARG;
-  if (d->dtype != HATA_F32 && d->dtype != HATA_BF16) return HATA_ERR_INVALID_ARG;
-  if (d->flags & ~HATA_FLAG_EARLY_PREFETCH) return HATA_ERR_INVALID_ARG;
-  if (d->head_dim != kHeadDim) return HATA_ERR_UNSUPPORTED;
-  if (d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
-    return HATA_ERR_UNSUPPORTED;
-  const long long G = d->n_q_heads / d->n_kv_heads;
-  if (G > 16 || G * d->hash_bits + 1 > kMaxBins) return HATA_ERR_UNSUPPORTED;
-  return HATA_OK;
-}
-
 hata_status_t cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return HATA_OK;
   return HATA_ERR_CUDA;
@@ -75,15 +59,16 @@ hata_status_t hata_workspace_init(void* ws, size_t bytes, void* stream) {
 
 hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_heads, int x_len, int n_tok,
                                  const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,
-                                 void* stream) {
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   hata_status_t s = check_dims(dims);
   if (s != HATA_OK) return s;
   if (!x || !W_H || !codes || !aligned16(x) || !aligned16(W_H) || !aligned16(codes)) return HATA_ERR_INVALID_ARG;
   if (x_heads < 1 || x_heads % dims->n_kv_heads || x_len < 1 || codes_len < 1 || n_tok < 0)
     return HATA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes) return HATA_ERR_WORKSPACE;
   if (n_tok == 0) return HATA_OK;
   return cuda_status(launch_encode(*dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len,
-                                   static_cast<cudaStream_t>(stream)));
+                                   static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream)));
 }
 
 hata_status_t hata_hamming_scores(const hata_dims_t* dims, const uint32_t* qcode, const uint32_t* codes,
@@ -169,8 +154,11 @@ hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const 
   uint32_t* qc = qcode_out ? qcode_out : reinterpret_cast<uint32_t*>(ws + L.qcode);
   int32_t* ix = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   int32_t* sc = reinterpret_cast<int32_t*>(ws + L.scores);
-  if ((e = launch_encode(d, q, d.n_q_heads, 1, 1, nullptr, W_q, qc, 1, st)) != cudaSuccess) return cuda_status(e);
-  if ((e = launch_encode(d, K, d.n_kv_heads, d.max_seq, 1, seq_lens, W_k, codes, d.max_seq, st)) != cudaSuccess)
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  if ((e = launch_encode(d, q, d.n_q_heads, 1, 1, nullptr, W_q, qc, 1, status, st)) != cudaSuccess)
+    return cuda_status(e);
+  if ((e = launch_encode(d, K, d.n_kv_heads, d.max_seq, 1, seq_lens, W_k, codes, d.max_seq, status, st)) !=
+      cudaSuccess)
     return cuda_status(e);
   if ((e = launch_hamming(d, qc, codes, seq_lens, sc, st)) != cudaSuccess) return cuda_status(e);
   if ((e = launch_topk(d, L, sc, seq_lens, k, ix, nullptr, ws, st)) != cudaSuccess) return cuda_status(e);
@@ -214,14 +202,6 @@ hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, con
                                           qcode_out, idx_out, &pg, static_cast<char*>(workspace),
                                           static_cast<cudaStream_t>(stream));
   return e == cudaErrorNotSupported ? HATA_ERR_UNSUPPORTED : cuda_status(e);
-}
-
-hata_status_t hata_encode_read_status(void* stream, int* device_status) {
-  if (!device_status) return HATA_ERR_INVALID_ARG;
-  uint32_t v = 0;
-  if (read_encode_status(static_cast<cudaStream_t>(stream), &v) != cudaSuccess) return HATA_ERR_CUDA;
-  *device_status = (int)v;
-  return HATA_OK;
 }
 
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {

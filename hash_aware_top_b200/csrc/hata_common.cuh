@@ -14,8 +14,26 @@ constexpr int kTopkChunk = 4096;     // tokens per top-k chunk in the granular p
 constexpr int kSparseRows = 32;      // gathered rows per CTA in the granular sparse decode
 constexpr int kMaxBins = 8193;       // G * r + 1 histogram bins supported
 constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 16;  // smallest buffer that can hold a device status word
 
 __host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Validation of the problem shape shared by every entry point (host side).
+inline hata_status_t check_dims(const hata_dims_t* d) {
+  if (!d) return HATA_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->max_seq < 1 || d->head_dim < 1 ||
+      d->hash_bits < 1)
+    return HATA_ERR_INVALID_ARG;
+  if (d->n_q_heads % d->n_kv_heads) return HATA_ERR_INVALID_ARG;
+  if (d->dtype != HATA_F32 && d->dtype != HATA_BF16) return HATA_ERR_INVALID_ARG;
+  if (d->flags & ~HATA_FLAG_EARLY_PREFETCH) return HATA_ERR_INVALID_ARG;
+  if (d->head_dim != kHeadDim) return HATA_ERR_UNSUPPORTED;
+  if (d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
+    return HATA_ERR_UNSUPPORTED;
+  const long long G = d->n_q_heads / d->n_kv_heads;
+  if (G > 16 || G * d->hash_bits + 1 > kMaxBins) return HATA_ERR_UNSUPPORTED;
+  return HATA_OK;
+}
 
 // Workspace regions (byte offsets).  One layout serves every call for given dims and k.
 struct WsLayout {

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kEncThreads)
 
 template <typename T>
 cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok, const int32_t* seq_end,
-                     const float* W, uint32_t* codes, int codes_len, cudaStream_t st) {
+                     const float* W, uint32_t* codes, int codes_len, uint32_t* status, cudaStream_t st) {
   const int hpg = x_heads / d.n_kv_heads;
   if (n_tok <= kDecodeTok) {
     const int nbz = (hpg * n_tok + kDecRows - 1) / kDecRows;
@@ -141,7 +141,7 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
     return cudaGetLastError();
   }
   if constexpr (sizeof(T) == 2) {  // bf16 keys: tensor-core prefill (r <= 128), tcgen05 first, then mma.sync
-    cudaError_t e = launch_encode_tc(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
+    cudaError_t e = launch_encode_tc(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, status, st);
     if (e == cudaErrorNotSupported) e = launch_encode_mma(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, st);
     if (e != cudaErrorNotSupported) return e;
   }
@@ -161,11 +161,11 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
 }  // namespace
 
 cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
-                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len, uint32_t* status,
                           cudaStream_t stream) {
   if (d.dtype == HATA_BF16)
-    return launch_t<__nv_bfloat16>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, stream);
-  return launch_t<float>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, stream);
+    return launch_t<__nv_bfloat16>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, status, stream);
+  return launch_t<float>(d, x, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, status, stream);
 }
 
 }  // namespace hata

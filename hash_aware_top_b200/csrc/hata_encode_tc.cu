@@ -33,18 +33,19 @@
 //     a code word, store each key's code as one vector and release the
 //     accumulator on a 128-thread mbarrier.  No CTA-wide barrier inside the loop.
 // Every wait is bounded: on expiry the kernel records HATA_ERR_TIMEOUT in the
-// library's encode status word (hata_encode_read_status), stops issuing work,
-// waits (bounded) for the MMAs it issued, frees its TMEM and returns.
+// caller's status word (the workspace passed to hata_encode_append), stops
+// issuing work, waits (bounded) for the MMAs it issued, frees its TMEM and
+// returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "hata_kernels.cuh"
 
 namespace hata {
-
-__device__ uint32_t g_encode_status;
 
 namespace {
 
@@ -171,7 +172,7 @@ template <int R>
 __global__ void __launch_bounds__(kTcThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap xmap, int x_heads, int x_len, int n_tok,
                      const int32_t* __restrict__ seq_end, const float* __restrict__ W, uint32_t* __restrict__ codes,
-                     int codes_len, int hpg) {
+                     int codes_len, int hpg, uint32_t* status) {
   constexpr int D = kHeadDim;
   constexpr int NWd = R / 32;
   constexpr int S = tc_stages(R);
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
     if (abort_s) return false;
     if (tc_wait(bar, parity)) return true;
-    if (!abort_s) atomicExch(&g_encode_status, (uint32_t)HATA_ERR_TIMEOUT);
+    if (!abort_s) set_status(status, HATA_ERR_TIMEOUT);
     abort_s = 1;
     return false;
   };
@@ -349,22 +350,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// Per device: the SM count and the shared-memory attributes of the three
+// instantiations, set once under a mutex.  A failed attribute call is returned
+// (the caller then uses another encode kernel).
+cudaError_t tc_device_setup(int* sms_out) {
+  static std::mutex mu;
+  static std::map<int, std::pair<cudaError_t, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = done.find(dev);
+  if (it == done.end()) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(encode_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(32));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(encode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(64));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(encode_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(128));
+    if (e != cudaSuccess) (void)cudaGetLastError();
+    it = done.emplace(dev, std::make_pair(e, std::max(sms, 1))).first;
+  }
+  *sms_out = it->second.second;
+  return it->second.first;
+}
+
 }  // namespace
 
 cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
                              const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
-                             cudaStream_t st) {
+                             uint32_t* status, cudaStream_t st) {
   if (d.dtype != HATA_BF16 || d.hash_bits > 128) return cudaErrorNotSupported;
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms < 1) sms = 1;
-    cudaFuncSetAttribute(encode_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(32));
-    cudaFuncSetAttribute(encode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(64));
-    cudaFuncSetAttribute(encode_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, tc_smem(128));
-  }
+  int sms = 0;
+  if (tc_device_setup(&sms) != cudaSuccess) return cudaErrorNotSupported;
   const int hpg = x_heads / d.n_kv_heads;
   const long long heads = (long long)d.batch * x_heads;
   const long long tiles = (n_tok + kTcTile - 1) / kTcTile;
@@ -376,18 +396,18 @@ cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, i
   const cuuint64_t gstride[1] = {(cuuint64_t)kHeadDim * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)kTcTile};
   const cuuint32_t estride[2] = {1, 1};
-  // the driver's tensor-map encoder, looked up through the runtime (no link-time driver dependency)
-  static PFN_cuTensorMapEncodeTiled encode_tiled = nullptr;
-  if (!encode_tiled) {
+  // the driver's tensor-map encoder, looked up once through the runtime (no link-time driver dependency)
+  static const PFN_cuTensorMapEncodeTiled encode_tiled = []() -> PFN_cuTensorMapEncodeTiled {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn) {
+        q != cudaDriverEntryPointSuccess) {
       (void)cudaGetLastError();
-      return cudaErrorNotSupported;
+      return nullptr;
     }
-    encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
-  }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+  }();
+  if (!encode_tiled) return cudaErrorNotSupported;
   if (encode_tiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -398,30 +418,20 @@ cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, i
   switch (d.hash_bits) {
     case 32:
       encode_tc_kernel<32><<<grid, kTcThreads, tc_smem(32), st>>>(xmap, x_heads, x_len, n_tok, seq_end, W, codes,
-                                                                  codes_len, hpg);
+                                                                  codes_len, hpg, status);
       break;
     case 64:
       encode_tc_kernel<64><<<grid, kTcThreads, tc_smem(64), st>>>(xmap, x_heads, x_len, n_tok, seq_end, W, codes,
-                                                                  codes_len, hpg);
+                                                                  codes_len, hpg, status);
       break;
     case 128:
       encode_tc_kernel<128><<<grid, kTcThreads, tc_smem(128), st>>>(xmap, x_heads, x_len, n_tok, seq_end, W, codes,
-                                                                    codes_len, hpg);
+                                                                    codes_len, hpg, status);
       break;
     default:
       return cudaErrorNotSupported;
   }
   return cudaGetLastError();
-}
-
-cudaError_t read_encode_status(cudaStream_t st, uint32_t* out) {
-  cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_encode_status, sizeof(uint32_t), 0, cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  const uint32_t zero = 0u;
-  if (e == cudaSuccess)
-    e = cudaMemcpyToSymbolAsync(g_encode_status, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
-  return e;
 }
 
 }  // namespace hata

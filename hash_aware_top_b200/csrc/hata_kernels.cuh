@@ -6,8 +6,9 @@
 
 namespace hata {
 
+// status: the caller's device status word (a bounded wait that runs out is recorded there)
 cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
-                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
+                          const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len, uint32_t* status,
                           cudaStream_t stream);
 
 cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,
@@ -30,9 +31,7 @@ cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, 
 // Prefill encode on tcgen05 tensor cores (bf16 keys, r <= 128; else cudaErrorNotSupported).
 cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
                              const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
-                             cudaStream_t stream);
-// Read and clear the encode kernels' device status word (synchronises the stream).
-cudaError_t read_encode_status(cudaStream_t stream, uint32_t* status);
+                             uint32_t* status, cudaStream_t stream);
 size_t dense_ws_bytes(const hata_dims_t& d);
 cudaError_t launch_dense_decode(const hata_dims_t& d, const void* q, const void* K, const void* V,
                                 const int32_t* seq_lens, float scale, void* out, char* ws, cudaStream_t stream);

@@ -81,15 +81,8 @@ using namespace hata;
 
 extern "C" hata_status_t hata_topk_noalloc(const hata_dims_t* dims, const int32_t* scores, const int32_t* seq_lens,
                                            int k, int32_t* idx, int32_t* n_sel, void* stream) {
-  if (!dims || dims->batch < 1 || dims->n_q_heads < 1 || dims->n_kv_heads < 1 || dims->max_seq < 1 ||
-      dims->n_q_heads % dims->n_kv_heads || (dims->dtype != HATA_F32 && dims->dtype != HATA_BF16) ||
-      (dims->flags & ~HATA_FLAG_EARLY_PREFETCH))
-    return HATA_ERR_INVALID_ARG;
-  if (dims->head_dim != kHeadDim ||
-      (dims->hash_bits != 32 && dims->hash_bits != 64 && dims->hash_bits != 128 && dims->hash_bits != 256))
-    return HATA_ERR_UNSUPPORTED;
-  const long long G = dims->n_q_heads / dims->n_kv_heads;
-  if (G > 16 || G * dims->hash_bits + 1 > kMaxBins) return HATA_ERR_UNSUPPORTED;
+  const hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
   if (!scores || !seq_lens || !idx || k < 1) return HATA_ERR_INVALID_ARG;
   const WsLayout L = topk_layout(*dims);
   if (L.total > kNoAllocScratchBytes) return HATA_ERR_WORKSPACE;  // too large for the built-in scratch

@@ -492,7 +492,10 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       __syncwarp();
       if (lane == 0) {
         // counters never reset: the k-th use of buffer s % kStages ends at count k * kNWarp
-        if (rel_s >= 0 && rel_old == ((rel_s / kStages) + 1) * kNWarp - 1 && rel_s + kStages < nst) {
+        // no refill once a wait has expired: the copies left in flight are then exactly
+        // the ones lastv records, which the drain before exit waits for
+        if (rel_s >= 0 && rel_old == ((rel_s / kStages) + 1) * kNWarp - 1 && rel_s + kStages < nst &&
+            !stat[ST_ABORT]) {
           ptx::fence_proxy_async_smem();
           issue(rel_s + kStages);
         }
@@ -1085,11 +1088,15 @@ __global__ void __launch_bounds__(kFThreads, 1) fused_step_kernel(const FusedPar
       static_cast<T*>(p.out)[((size_t)b * p.Hq + (size_t)g * G + h) * D + (e % D)] = from_f32<T>(l > 0.f ? o / l : 0.f);
     }
   }
-  if (stat[ST_ABORT] && tid == 0) {
-    // give outstanding bulk copies one more bounded chance to land before exit
-    for (int bi = 0; bi < kStages; ++bi)
-      if (lastv[bi] >= 0) ptx::mbar_wait_bounded(&mbar[bi], (uint32_t)(lastv[bi] / kStages) & 1u, kWaitTries);
-    ptx::mbar_wait_bounded(&mbar[kMaxStages + 1], 0u, kWaitTries);  // the W_H copy
+  if (stat[ST_ABORT]) {
+    // nothing may land in shared memory after the CTA exits: every thread waits for its
+    // own row gathers, and thread 0 gives the bulk copies one more bounded chance
+    ptx::cp_async_wait_all();
+    if (tid == 0) {
+      for (int bi = 0; bi < kStages; ++bi)
+        if (lastv[bi] >= 0) ptx::mbar_wait_bounded(&mbar[bi], (uint32_t)(lastv[bi] / kStages) & 1u, kWaitTries);
+      ptx::mbar_wait_bounded(&mbar[kMaxStages + 1], 0u, kWaitTries);  // the W_H copy
+    }
   }
 }
 

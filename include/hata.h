@@ -30,8 +30,9 @@
  *
  * Conventions for every call:
  *   - All tensor arguments are DEVICE pointers owned by the caller.  The library
- *     allocates no device memory and keeps no global mutable state; scratch
- *     space is a caller-provided workspace (hata_workspace_size).
+ *     allocates no device memory.  Scratch space and the device status word are
+ *     a caller-provided workspace (hata_workspace_size); the one exception is
+ *     hata_topk_noalloc, whose scratch is a fixed array inside the library.
  *   - Every call only enqueues work on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream) and never synchronises, except
  *     hata_read_device_status.
@@ -132,16 +133,17 @@ HATA_API hata_status_t hata_workspace_init(void* workspace, size_t workspace_byt
  * with W_H split into three bf16 parts (exact products, fp32 accumulation in
  * another order); other prefill forms are fp32 FMA.  Codes of the different
  * forms can differ only where |x . W_H| is within fp32 rounding of zero.
+ *   workspace  device, 16-byte aligned, at least 16 bytes (any workspace from
+ *              hata_workspace_size qualifies, and can be shared with the other
+ *              calls on the same stream): only its status word is used.  If a
+ *              bounded wait of the tensor-core kernel runs out, HATA_ERR_TIMEOUT
+ *              is recorded there (the codes are then incomplete); read it with
+ *              hata_read_device_status.  Missing or too small:
+ *              HATA_ERR_WORKSPACE.
  */
 HATA_API hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_heads, int x_len, int n_tok,
                                  const int32_t* seq_end, const float* W_H, uint32_t* codes, int codes_len,
-                                 void* stream);
-
-/* Read and clear the status word of the prefill encode kernels (synchronises the
- * stream): HATA_ERR_TIMEOUT if a bounded wait of a hata_encode_append call on
- * the tensor cores expired since the last read (its codes are then incomplete),
- * else 0.  The word is one per device, in the library. */
-HATA_API hata_status_t hata_encode_read_status(void* stream, int* device_status);
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Hamming scan with the GQA sum (Decode 阶段算法, Hamming and GQA steps;

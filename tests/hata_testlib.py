@@ -61,3 +61,58 @@ def max_abs(a, b) -> float:
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def run_step(H, wl, inp, codes0, ws=None, with_debug=True, flags=0):
+    """One hata_decode_step through the C ABI on the workload's inputs, with the cache holding codes0."""
+    d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype, flags)
+    ws = ws if ws is not None else new_workspace(d, wl.k)
+    codes = dev_codes(codes0)
+    out = torch.full((wl.batch, wl.n_q_heads, 128), float("nan"), dtype=d.torch_dtype, device="cuda")
+    qcode = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda") if with_debug else None
+    idx = torch.full((wl.batch, wl.n_kv_heads, wl.k), -99, dtype=torch.int32, device="cuda") if with_debug else None
+    H.hata_decode_step(d, dev_float(inp["q"], wl.dtype), dev_float(inp["K"], wl.dtype), dev_float(inp["V"], wl.dtype),
+                       torch.from_numpy(inp["W_H"]).cuda(), codes, torch.from_numpy(inp["seq_lens"]).cuda(), wl.k,
+                       0.0, out, qcode, idx, ws)
+    torch.cuda.synchronize()
+    return {
+        "codes": host_codes(codes),
+        "out": out.float().cpu().numpy(),
+        "qcode": host_codes(qcode) if with_debug else None,
+        "idx": idx.cpu().numpy() if with_debug else None,
+        "ws": ws,
+    }
+
+
+def check_step(wl, inp, codes0, got, W_k=None):
+    """Compare one decode step with the oracle.  Where the GPU's fp32 projection
+    lands on the other side of zero inside the exemption band, the downstream
+    results are checked for validity against the codes the GPU chose.  W_k: a
+    separate key encoder (codes0 then holds keys encoded with it)."""
+    ref = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes0, inp["seq_lens"], wl.k, W_k=W_k)
+    G, r = wl.group, wl.hash_bits
+    flips = assert_codes_match(got["qcode"], ref["qcode"], ref["y_q"], r)
+    for b in range(wl.batch):
+        Lb = int(inp["seq_lens"][b])
+        for g in range(wl.n_kv_heads):
+            flips += assert_codes_match(got["codes"][b, g, Lb - 1], ref["codes"][b, g, Lb - 1], ref["y_k"][b, g], r)
+            assert np.array_equal(got["codes"][b, g, :Lb - 1], codes0[b, g, :Lb - 1])
+    tol = TOL[wl.dtype]
+    for b in range(wl.batch):
+        Lb = int(inp["seq_lens"][b])
+        for g in range(wl.n_kv_heads):
+            hs = slice(g * G, (g + 1) * G)
+            if flips == 0:
+                want_idx = ref["idx"][b, g]
+                want_out = ref["out"][b, hs]
+            else:  # validity: the oracle's own steps applied to the codes the GPU chose
+                D = oracle.gqa_scores(got["qcode"][b, hs], got["codes"][b, g, :Lb], r)
+                S = oracle.topk_select(D, wl.k)
+                want_idx = np.full(wl.k, -1)
+                want_idx[:len(S)] = S
+                want_out = oracle.sparse_attention(inp["q"][b, hs], inp["K"][b, g], inp["V"][b, g], S,
+                                                   1 / math.sqrt(128))
+            assert np.array_equal(got["idx"][b, g], want_idx), (b, g)
+            err = max_abs(got["out"][b, hs], want_out)
+            assert err <= tol, (b, g, err)
+    return ref, flips

@@ -77,7 +77,11 @@ def test_calls_reject_bad_arguments_before_launch(H):
     null = P(0)
     lib = H.lib
     # null pointers
-    assert lib.hata_encode_append(ctypes.byref(d), null, 1, 64, 1, null, fake, fake, 64, null) == 1
+    assert lib.hata_encode_append(ctypes.byref(d), null, 1, 64, 1, null, fake, fake, 64, fake, 16, null) == 1
+    # the encode's status workspace: missing, misaligned or smaller than one status word
+    assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, null, 16, null) == 5
+    assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, P(0x1008), 16, null) == 5
+    assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, fake, 8, null) == 5
     assert lib.hata_hamming_scores(ctypes.byref(d), fake, fake, null, fake, null) == 1
     # k < 1
     assert lib.hata_topk(ctypes.byref(d), fake, fake, 0, fake, null, fake, 1 << 20, null) == 1
@@ -94,16 +98,16 @@ def test_calls_reject_bad_arguments_before_launch(H):
                                   fake, 1 << 30, null) == 1
     # x_heads not a multiple of Hkv, unsupported dims
     d2 = H.dims_for(1, 4, 2, 128, 128, 64, "bf16")
-    assert lib.hata_encode_append(ctypes.byref(d2), fake, 3, 64, 1, null, fake, fake, 64, null) == 1
+    assert lib.hata_encode_append(ctypes.byref(d2), fake, 3, 64, 1, null, fake, fake, 64, fake, 16, null) == 1
     d3 = H.dims_for(1, 4, 1, 128, 100, 64, "bf16")
     assert lib.hata_hamming_scores(ctypes.byref(d3), fake, fake, fake, fake, null) == 2
     assert lib.hata_read_device_status(null, null, ctypes.byref(ctypes.c_int())) == 1
 
 
 def test_separate_encoder_and_paged_calls_reject_bad_arguments(H):
-    """hata_decode_step_qk, hata_decode_step_paged and hata_encode_read_status validate
-    on the host: missing or misaligned matrices and tables, block sizes that are not
-    a power of two in [16, 65536], an empty pool, a null status pointer."""
+    """hata_decode_step_qk and hata_decode_step_paged validate on the host: missing or
+    misaligned matrices and tables, block sizes that are not a power of two in
+    [16, 65536], an empty pool."""
     d = H.dims_for(1, 4, 1, 128, 128, 1024, "bf16")
     P = ctypes.c_void_p
     fake, odd, null = P(0x1000), P(0x1008), P(0)
@@ -124,7 +128,6 @@ def test_separate_encoder_and_paged_calls_reject_bad_arguments(H):
         assert paged(fake, bs, 16) == 1, bs
     assert paged(fake, 64, 0) == 1           # empty pool
     assert paged(fake, 64, 16, k=0) == 1     # k < 1
-    assert lib.hata_encode_read_status(null, None) == 1
 
 
 def test_binding_refuses_cpu_tensors(H):

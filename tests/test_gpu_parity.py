@@ -9,8 +9,8 @@ import pytest
 import oracle
 from hata_inputs import Workload, make_inputs, random_codes, random_indices, random_scores
 
-from hata_testlib import (TOL, assert_codes_match, default_scale, dev_codes, dev_float, host_codes, max_abs,
-                          new_workspace)
+from hata_testlib import (TOL, assert_codes_match, check_step, default_scale, dev_codes, dev_float, host_codes,
+                          max_abs, new_workspace, run_step)
 
 pytestmark = pytest.mark.gpu
 
@@ -44,8 +44,9 @@ def test_encode_prefill_and_queries(H, r, dtype):
     sentinel = np.uint32(0xA5A5A5A5)
     codes = dev_codes(np.full((2, 2, 1000, r // 32), sentinel, dtype=np.uint32))
     # prefill every slot below L_b: n_tok = max_seq ending at seq_lens
-    H.hata_encode_append(d, K, 2, 1000, 1000, lens, W, codes, 1000)
-    assert H.hata_encode_read_status() == 0
+    ws = new_workspace(d, 16)
+    H.hata_encode_append(d, K, 2, 1000, 1000, lens, W, codes, 1000, ws)
+    assert H.hata_read_device_status(ws) == 0
     got = host_codes(codes)
     want, ys = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"], upto_last=False)
     for b in range(2):
@@ -56,7 +57,7 @@ def test_encode_prefill_and_queries(H, r, dtype):
     # queries: x_len = codes_len = 1, heads grouped on W_H[h // G]
     q = dev_float(inp["q"], dtype)
     qc = dev_codes(np.zeros((2, 8, r // 32), dtype=np.uint32))
-    H.hata_encode_append(d, q, 8, 1, 1, None, W, qc, 1)
+    H.hata_encode_append(d, q, 8, 1, 1, None, W, qc, 1, ws)
     gq = host_codes(qc)
     for b in range(2):
         for h in range(8):
@@ -74,9 +75,10 @@ def test_encode_prefill_many_tiles_per_cta(H, r):
     inp = make_inputs(wl, seed=3, plant=False)
     d = _dims(H, B, 8, Hkv, r, L, "bf16")
     codes = dev_codes(np.zeros((B, Hkv, L, r // 32), dtype=np.uint32))
+    ws = new_workspace(d, 16)
     H.hata_encode_append(d, dev_float(inp["K"], "bf16"), Hkv, L, L, torch.from_numpy(inp["seq_lens"]).cuda(),
-                         torch.from_numpy(inp["W_H"]).cuda(), codes, L)
-    assert H.hata_encode_read_status() == 0
+                         torch.from_numpy(inp["W_H"]).cuda(), codes, L, ws)
+    assert H.hata_read_device_status(ws) == 0
     got = host_codes(codes)
     want, ys = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"], upto_last=False)
     Lb = int(inp["seq_lens"][0])
@@ -97,9 +99,10 @@ def test_encode_prefill_grouped_heads_window(H):
     d = _dims(H, B, Hq, Hkv, r, cl, "bf16")
     sentinel = np.uint32(0x5A5A5A5A)
     codes = dev_codes(np.full((B, Hq, cl, r // 32), sentinel, dtype=np.uint32))
+    ws = new_workspace(d, 16)
     H.hata_encode_append(d, x.cuda(), Hq, xl, n_tok, torch.from_numpy(end).cuda(), torch.from_numpy(W).cuda(),
-                         codes, cl)
-    assert H.hata_encode_read_status() == 0
+                         codes, cl, ws)
+    assert H.hata_read_device_status(ws) == 0
     got = host_codes(codes)
     xf = x.float().numpy()
     for b in range(B):
@@ -117,8 +120,10 @@ def test_encode_append_single_slot(H):
     d = _dims(H, 3, 4, 4, 128, 300, "bf16")
     codes0 = random_codes((3, 4, 300), 128, seed=5)
     codes = dev_codes(codes0)
+    ws = new_workspace(d, 16)
     H.hata_encode_append(d, dev_float(inp["K"], "bf16"), 4, 300, 1, torch.from_numpy(inp["seq_lens"]).cuda(),
-                         torch.from_numpy(inp["W_H"]).cuda(), codes, 300)
+                         torch.from_numpy(inp["W_H"]).cuda(), codes, 300, ws)
+    assert H.hata_read_device_status(ws) == 0
     got = host_codes(codes)
     for b in range(3):
         Lb = int(inp["seq_lens"][b])
@@ -301,60 +306,6 @@ STEP_CASES = {
 }
 
 
-def run_step(H, wl, inp, codes0, ws=None, with_debug=True):
-    d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype)
-    ws = ws if ws is not None else new_workspace(d, wl.k)
-    codes = dev_codes(codes0)
-    out = torch.full((wl.batch, wl.n_q_heads, 128), float("nan"), dtype=d.torch_dtype, device="cuda")
-    qcode = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda") if with_debug else None
-    idx = torch.full((wl.batch, wl.n_kv_heads, wl.k), -99, dtype=torch.int32, device="cuda") if with_debug else None
-    H.hata_decode_step(d, dev_float(inp["q"], wl.dtype), dev_float(inp["K"], wl.dtype), dev_float(inp["V"], wl.dtype),
-                       torch.from_numpy(inp["W_H"]).cuda(), codes, torch.from_numpy(inp["seq_lens"]).cuda(), wl.k,
-                       0.0, out, qcode, idx, ws)
-    torch.cuda.synchronize()
-    return {
-        "codes": host_codes(codes),
-        "out": out.float().cpu().numpy(),
-        "qcode": host_codes(qcode) if with_debug else None,
-        "idx": idx.cpu().numpy() if with_debug else None,
-        "ws": ws,
-    }
-
-
-def check_step(wl, inp, codes0, got, W_k=None):
-    """Compare one decode step with the oracle.  Where the GPU's fp32 projection
-    lands on the other side of zero inside the exemption band, the downstream
-    results are checked for validity against the codes the GPU chose.  W_k: a
-    separate key encoder (codes0 then holds keys encoded with it)."""
-    ref = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], codes0, inp["seq_lens"], wl.k, W_k=W_k)
-    G, r = wl.group, wl.hash_bits
-    flips = assert_codes_match(got["qcode"], ref["qcode"], ref["y_q"], r)
-    for b in range(wl.batch):
-        Lb = int(inp["seq_lens"][b])
-        for g in range(wl.n_kv_heads):
-            flips += assert_codes_match(got["codes"][b, g, Lb - 1], ref["codes"][b, g, Lb - 1], ref["y_k"][b, g], r)
-            assert np.array_equal(got["codes"][b, g, :Lb - 1], codes0[b, g, :Lb - 1])
-    tol = TOL[wl.dtype]
-    for b in range(wl.batch):
-        Lb = int(inp["seq_lens"][b])
-        for g in range(wl.n_kv_heads):
-            hs = slice(g * G, (g + 1) * G)
-            if flips == 0:
-                want_idx = ref["idx"][b, g]
-                want_out = ref["out"][b, hs]
-            else:  # validity: the oracle's own steps applied to the codes the GPU chose
-                D = oracle.gqa_scores(got["qcode"][b, hs], got["codes"][b, g, :Lb], r)
-                S = oracle.topk_select(D, wl.k)
-                want_idx = np.full(wl.k, -1)
-                want_idx[:len(S)] = S
-                want_out = oracle.sparse_attention(inp["q"][b, hs], inp["K"][b, g], inp["V"][b, g], S,
-                                                   1 / math.sqrt(128))
-            assert np.array_equal(got["idx"][b, g], want_idx), (b, g)
-            err = max_abs(got["out"][b, hs], want_out)
-            assert err <= tol, (b, g, err)
-    return ref, flips
-
-
 @pytest.mark.parametrize("name", list(STEP_CASES))
 def test_decode_step(H, name):
     wl = STEP_CASES[name]
@@ -378,8 +329,8 @@ def test_decode_step_equals_granular_chain(H):
     lens = torch.from_numpy(inp["seq_lens"]).cuda()
     codes = dev_codes(codes0)
     qc = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda")
-    H.hata_encode_append(d, q, wl.n_q_heads, 1, 1, None, W, qc, 1)
-    H.hata_encode_append(d, K, wl.n_kv_heads, wl.max_seq, 1, lens, W, codes, wl.max_seq)
+    H.hata_encode_append(d, q, wl.n_q_heads, 1, 1, None, W, qc, 1, ws)
+    H.hata_encode_append(d, K, wl.n_kv_heads, wl.max_seq, 1, lens, W, codes, wl.max_seq, ws)
     sc = torch.empty((wl.batch, wl.n_kv_heads, wl.max_seq), dtype=torch.int32, device="cuda")
     H.hata_hamming_scores(d, qc, codes, lens, sc)
     idx = torch.empty((wl.batch, wl.n_kv_heads, wl.k), dtype=torch.int32, device="cuda")

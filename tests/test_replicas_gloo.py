@@ -99,3 +99,17 @@ def test_reference_arm_json_contract():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["e2e"]["value"] == line["value"]
+
+
+def test_cpu_baseline_uses_every_host_core():
+    """The benchmark's CPU baseline times whole decode steps of the oracle on every core
+    this process may run on, and a bounded one-thread sample beside it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from hata_inputs import WORKLOADS, make_inputs
+
+    wl = WORKLOADS["tiny_f32_4k"]
+    cb = bench.cpu_baseline(wl, make_inputs(wl, seed=0), budget_s=0.5)
+    assert cb["kind"] == "oracle" and cb["unit"] == "steps/s" and cb["value"] > 0
+    assert cb["cores"] == bench.host_cores()
+    assert cb["single_thread"]["cores"] == 1 and cb["single_thread"]["value"] > 0
