@@ -50,6 +50,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhata.so"
 HATA_OK, HATA_ERR_INVALID_ARG, HATA_ERR_UNSUPPORTED, HATA_ERR_CUDA, HATA_ERR_TIMEOUT, HATA_ERR_WORKSPACE = range(6)
 HATA_F32, HATA_BF16 = 0, 1
 HATA_FLAG_EARLY_PREFETCH = 1
+HATA_FLAG_TEST_EXPIRE_WAIT = 2  # test hook: the step's first bounded wait runs out (see include/hata.h)
 
 EXPORTED_SYMBOLS = (
     "hata_workspace_size",

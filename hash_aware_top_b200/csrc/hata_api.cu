@@ -1,6 +1,7 @@
 // extern "C" entry points of libhata: argument validation, workspace carving,
 // launches.  Nothing here allocates device memory or synchronises (except
 // hata_read_device_status).
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 
@@ -17,7 +18,9 @@ hata_status_t cuda_status(cudaError_t e) {
   return HATA_ERR_CUDA;
 }
 
-WsLayout layout_for(const hata_dims_t& d, int k) { return make_layout(d, k, fused_step_ws_bytes(d, k)); }
+WsLayout layout_for(const hata_dims_t& d, int k) {
+  return make_layout(d, k, std::max(fused_step_ws_bytes(d, k), split_step_ws_bytes(d, k)));
+}
 
 hata_status_t check_ws(const hata_dims_t& d, int k, const void* ws, size_t bytes, WsLayout* L) {
   *L = layout_for(d, k);
@@ -145,8 +148,12 @@ hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
-  cudaError_t e = launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out,
+  cudaError_t e = launch_split_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out,
                                     nullptr, ws, st);
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+  if (dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT) return HATA_ERR_UNSUPPORTED;  // the hook exists in the split step only
+  e = launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, nullptr, ws,
+                        st);
   if (e != cudaErrorNotSupported) return cuda_status(e);
 
   // Chain of the granular kernels (shapes the fused kernel does not cover).
@@ -198,14 +205,19 @@ hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, con
   while ((1 << pg.block_shift) < block_size) ++pg.block_shift;
   pg.n_blocks = n_blocks;
   pg.max_blocks = (dims->max_seq + block_size - 1) / block_size;
-  const cudaError_t e = launch_fused_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out,
-                                          qcode_out, idx_out, &pg, static_cast<char*>(workspace),
-                                          static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_split_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out,
+                                    qcode_out, idx_out, &pg, static_cast<char*>(workspace),
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+  if (dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT) return HATA_ERR_UNSUPPORTED;
+  e = launch_fused_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out, qcode_out, idx_out,
+                        &pg, static_cast<char*>(workspace), static_cast<cudaStream_t>(stream));
   return e == cudaErrorNotSupported ? HATA_ERR_UNSUPPORTED : cuda_status(e);
 }
 
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {
   if (check_dims(dims) != HATA_OK || k < 1) return -1;
+  if (split_step_applies(*dims, k)) return 2;
   return fused_step_applies(*dims, k) ? 1 : 6;
 }
 

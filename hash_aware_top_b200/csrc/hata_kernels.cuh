@@ -50,4 +50,12 @@ cudaError_t launch_fused_step(const hata_dims_t& d, const WsLayout& L, const voi
                               const int32_t* seq_lens, int k, float scale, void* out, uint32_t* qcode_out,
                               int32_t* idx_out, const PagedCache* pg, char* ws, cudaStream_t stream);
 
+// Decode step as a scan kernel over all SMs plus a per-unit tail kernel (hata_fused.cu).
+bool split_step_applies(const hata_dims_t& d, int k);
+size_t split_step_ws_bytes(const hata_dims_t& d, int k);
+cudaError_t launch_split_step(const hata_dims_t& d, const WsLayout& L, const void* q, const void* K,
+                              const void* V, const float* W, const float* Wk, uint32_t* codes,
+                              const int32_t* seq_lens, int k, float scale, void* out, uint32_t* qcode_out,
+                              int32_t* idx_out, const PagedCache* pg, char* ws, cudaStream_t stream);
+
 }  // namespace hata

@@ -104,6 +104,15 @@ typedef struct {
  * encode of the same cache. */
 #define HATA_FLAG_EARLY_PREFETCH 1
 
+/* Test hook for the timeout path of hata_decode_step (and its _qk and _paged
+ * forms): the call's first bounded device-side wait is made on a barrier that
+ * nothing completes, with a short limit, so it runs out; the call then records
+ * HATA_ERR_TIMEOUT in the workspace's status word, skips its remaining work
+ * without touching memory outside its arguments, and its outputs are
+ * undefined.  Never set it outside tests; after it, re-initialise the
+ * workspace (hata_workspace_init). */
+#define HATA_FLAG_TEST_EXPIRE_WAIT 2
+
 /* Bytes of workspace that every call below needs for these dims and budget k
  * (one size serves all calls).  Returns HATA_OK and writes *bytes. */
 HATA_API hata_status_t hata_workspace_size(const hata_dims_t* dims, int k, size_t* bytes);

@@ -403,5 +403,41 @@ def test_decode_step_flags_length_beyond_cache(H):
 
 
 def test_kernel_count_reports_fused_and_chain(H):
-    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 1
+    # scan kernel + tail kernel, or the chain of six granular launches (G = 3)
+    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 2
     assert H.hata_decode_step_kernel_count(H.dims_for(1, 6, 2, 128, 128, 3000, "bf16"), 100) == 6
+
+
+def _custom_step(H, wl, seed, codes0):
+    inp = make_inputs(wl, seed=seed, plant=False)
+    got = run_step(H, wl, inp, codes0)
+    check_step(wl, inp, codes0, got)
+    assert H.hata_read_device_status(got["ws"]) == 0
+
+
+def test_decode_step_heavy_ties(H):
+    """Every cached code equal: all but the new token tie.  The earliest chunks' candidate
+    lists cannot hold their tie quota, so the tail kernel rescores them from the cache."""
+    wl = Workload("ties", 2, 8, 2, 128, 20000, 128, 600, "bf16", seq_len_range=(15000, 20000))
+    codes0 = np.repeat(random_codes((1, 1, 1), 128, seed=3), 2 * 2 * 20000, axis=0).reshape(2, 2, 20000, 4)
+    _custom_step(H, wl, 21, codes0)
+
+
+def test_decode_step_selection_in_one_chunk(H):
+    """The k nearest codes all sit in the first 2,000 slots (a copy of the group's first
+    query code with a few random bits flipped), so one chunk holds the whole selection and
+    its list stops short of the threshold."""
+    wl = Workload("clustered", 1, 16, 4, 128, 60000, 128, 700, "bf16")
+    inp = make_inputs(wl, seed=23, plant=False)
+    qcode = oracle.decode_step(inp["q"], inp["K"], inp["V"], inp["W_H"], np.zeros((1, 4, 60000, 4), np.uint32),
+                               inp["seq_lens"], 1)["qcode"]
+    codes0 = random_codes((1, 4, 60000), 128, seed=5)
+    rng = np.random.default_rng(29)
+    for g in range(4):
+        near = np.repeat(qcode[0, 4 * g][None, :], 2000, axis=0)
+        flips = np.zeros((2000, 4), np.uint32)
+        for t in range(2000):  # 1-20 random bit flips per slot: many distinct low scores
+            for bit in rng.choice(128, size=int(rng.integers(1, 21)), replace=False):
+                flips[t, bit // 32] |= np.uint32(1) << np.uint32(bit % 32)
+        codes0[0, g, :2000] = near ^ flips
+    _custom_step(H, wl, 23, codes0)
