@@ -51,6 +51,7 @@ HATA_OK, HATA_ERR_INVALID_ARG, HATA_ERR_UNSUPPORTED, HATA_ERR_CUDA, HATA_ERR_TIM
 HATA_F32, HATA_BF16 = 0, 1
 HATA_FLAG_EARLY_PREFETCH = 1
 HATA_FLAG_TEST_EXPIRE_WAIT = 2  # test hook: the step's first bounded wait runs out (see include/hata.h)
+HATA_FLAG_ALL_SM_SCAN = 4  # the all-SM form of the decode step for any shape it covers
 
 EXPORTED_SYMBOLS = (
     "hata_workspace_size",

@@ -22,6 +22,17 @@ WsLayout layout_for(const hata_dims_t& d, int k) {
   return make_layout(d, k, std::max(fused_step_ws_bytes(d, k), split_step_ws_bytes(d, k)));
 }
 
+// The fused form of a decode step (both give the same results).  Measured on B200 at
+// the benchmark workloads: the single-launch cluster form is faster while the units
+// are few (8 units at 32K-128K, one unit, 32 units of r = 32 codes), the all-SM form
+// with many units (128 ragged units) and on a paged cache (its per-segment copies are
+// issued from several lanes at once).
+bool use_all_sm(const hata_dims_t& d, int k, bool paged) {
+  if (!split_step_applies(d, k)) return false;
+  if (d.flags & (HATA_FLAG_ALL_SM_SCAN | HATA_FLAG_TEST_EXPIRE_WAIT)) return true;
+  return paged || (long long)d.batch * d.n_kv_heads >= 64 || !fused_step_applies(d, k);
+}
+
 hata_status_t check_ws(const hata_dims_t& d, int k, const void* ws, size_t bytes, WsLayout* L) {
   *L = layout_for(d, k);
   if (!ws || !aligned16(ws)) return HATA_ERR_WORKSPACE;
@@ -148,13 +159,15 @@ hata_status_t hata_decode_step_qk(const hata_dims_t* dims, const void* q, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
 
-  cudaError_t e = launch_split_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out,
-                                    nullptr, ws, st);
+  cudaError_t e = cudaErrorNotSupported;
+  if (use_all_sm(*dims, k, false))
+    e = launch_split_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, nullptr,
+                          ws, st);
+  else if (!(dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT))  // the test hook exists in the all-SM form only
+    e = launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, nullptr,
+                          ws, st);
   if (e != cudaErrorNotSupported) return cuda_status(e);
-  if (dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT) return HATA_ERR_UNSUPPORTED;  // the hook exists in the split step only
-  e = launch_fused_step(*dims, L, q, K, V, W_q, W_k, codes, seq_lens, k, scale, out, qcode_out, idx_out, nullptr, ws,
-                        st);
-  if (e != cudaErrorNotSupported) return cuda_status(e);
+  if (dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT) return HATA_ERR_UNSUPPORTED;
 
   // Chain of the granular kernels (shapes the fused kernel does not cover).
   const hata_dims_t& d = *dims;
@@ -205,9 +218,10 @@ hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, con
   while ((1 << pg.block_shift) < block_size) ++pg.block_shift;
   pg.n_blocks = n_blocks;
   pg.max_blocks = (dims->max_seq + block_size - 1) / block_size;
-  cudaError_t e = launch_split_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out,
-                                    qcode_out, idx_out, &pg, static_cast<char*>(workspace),
-                                    static_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaErrorNotSupported;
+  if (use_all_sm(*dims, k, true))
+    e = launch_split_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out, qcode_out,
+                          idx_out, &pg, static_cast<char*>(workspace), static_cast<cudaStream_t>(stream));
   if (e != cudaErrorNotSupported) return cuda_status(e);
   if (dims->flags & HATA_FLAG_TEST_EXPIRE_WAIT) return HATA_ERR_UNSUPPORTED;
   e = launch_fused_step(*dims, L, q, K_pool, V_pool, W_q, W_k, codes_pool, seq_lens, k, scale, out, qcode_out, idx_out,
@@ -217,7 +231,7 @@ hata_status_t hata_decode_step_paged(const hata_dims_t* dims, const void* q, con
 
 int hata_decode_step_kernel_count(const hata_dims_t* dims, int k) {
   if (check_dims(dims) != HATA_OK || k < 1) return -1;
-  if (split_step_applies(*dims, k)) return 2;
+  if (use_all_sm(*dims, k, false)) return 3;
   return fused_step_applies(*dims, k) ? 1 : 6;
 }
 

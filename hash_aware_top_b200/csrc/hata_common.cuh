@@ -26,7 +26,8 @@ inline hata_status_t check_dims(const hata_dims_t* d) {
     return HATA_ERR_INVALID_ARG;
   if (d->n_q_heads % d->n_kv_heads) return HATA_ERR_INVALID_ARG;
   if (d->dtype != HATA_F32 && d->dtype != HATA_BF16) return HATA_ERR_INVALID_ARG;
-  if (d->flags & ~(HATA_FLAG_EARLY_PREFETCH | HATA_FLAG_TEST_EXPIRE_WAIT)) return HATA_ERR_INVALID_ARG;
+  if (d->flags & ~(HATA_FLAG_EARLY_PREFETCH | HATA_FLAG_TEST_EXPIRE_WAIT | HATA_FLAG_ALL_SM_SCAN))
+    return HATA_ERR_INVALID_ARG;
   if (d->head_dim != kHeadDim) return HATA_ERR_UNSUPPORTED;
   if (d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
     return HATA_ERR_UNSUPPORTED;

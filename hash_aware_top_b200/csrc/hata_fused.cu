@@ -51,7 +51,9 @@ namespace hata {
 namespace {
 
 constexpr int kSThreads = 512;                  // scan CTA
+constexpr int kSWarp = kSThreads / 32;
 constexpr int kTThreads = 512;                  // tail CTA
+constexpr int kEThreads = 128;                  // encode CTA: 4 residues x the 32 columns of one code word
 constexpr int kNWarp = 512 / 32;
 constexpr int kRingBytes = 131072;              // one chunk's codes, all in flight at once
 constexpr int kPieceBytes = 16384;              // one mbarrier per piece
@@ -73,6 +75,7 @@ constexpr uint32_t kAbortBit = 0x80000000u;     // chunk record header: the scan
 struct StepGeom {
   int C, P, cap, nbp;
   uint32_t slot_bytes, cum_off, cand_off;
+  uint32_t hist_bytes, unit_bytes;  // unit region: histogram [nbp] u32, then P chunk records
 };
 
 struct StepParams {
@@ -103,21 +106,19 @@ __host__ __device__ constexpr int nbins_padded(int G, int R) { return (G * R + 1
 // Dynamic shared memory of the scan kernel: ring | scores (aliased by the encode's
 // residue sums) | histogram | fp32 encode inputs | mbarriers.
 struct ScanSmem {
-  int ring, D, hist, xr, mbar, total;
+  int ring, D, hist, mbar, total;
 };
 __host__ __device__ constexpr int round16(int x) { return (x + 15) / 16 * 16; }
 __host__ __device__ inline ScanSmem scan_smem(int G, int NW) {
-  const int R = NW * 32, NV = G + 1;
+  const int R = NW * 32;
   const int cmax = kRingBytes / (NW * 4);
   const int nbp = nbins_padded(G, R);
   const int bpt = (nbp + kSThreads - 1) / kSThreads;
   ScanSmem s{};
   s.ring = 0;
   s.D = kRingBytes;
-  const int dbytes = round16(cmax * 2 + 32) > NV * 4 * R * 4 ? round16(cmax * 2 + 32) : NV * 4 * R * 4;
-  s.hist = s.D + dbytes;
-  s.xr = s.hist + bpt * kSThreads * 4;
-  s.mbar = round16(s.xr + NV * 4 * kXS * 4);
+  s.hist = s.D + round16(cmax * 2 + 32);
+  s.mbar = s.hist + bpt * kSThreads * 4;
   s.total = s.mbar + (kMaxPieces + 1) * 8;
   return s;
 }
@@ -134,9 +135,9 @@ __host__ __device__ inline TailSmem tail_smem(int G, int NW, int esize, const St
     o = round16(o + bytes);
     return r;
   };
-  s.rec = take(geo.P * (int)geo.slot_bytes);
-  // the K rows' buffer also holds the P.V partial sums [row groups][G][d] fp32
-  s.Kr = take(std::max(GB * kHeadDim * esize, (kTThreads / (kHeadDim / 2)) * G * kHeadDim * 4));
+  s.rec = take((int)geo.unit_bytes);
+  // the K rows' buffer also holds the warps' attention partials [warps][G][d + 2] fp32
+  s.Kr = take(std::max(GB * kHeadDim * esize, (kTThreads / 32) * G * (kHeadDim + 2) * 4));
   s.Vr = take(GB * kHeadDim * esize);
   s.lg = take(G * GB * 4);
   s.rowtok = take(GB * 4);
@@ -201,56 +202,150 @@ __device__ __forceinline__ size_t token_slot(const StepParams& p, int b, int g, 
 __device__ __forceinline__ int clamp_seq(int L, int max_seq) { return L < 0 ? 0 : (L > max_seq ? max_seq : L); }
 
 // ---------------------------------------------------------------------------
+// encode kernel: the G query codes and the new key's code of every unit, one code
+// word (32 columns of W_H) per CTA
+// ---------------------------------------------------------------------------
+template <typename T, int NW, int G, bool PAGED>
+__global__ void __launch_bounds__(kEThreads) step_encode_kernel(const StepParams p) {
+  constexpr int D = kHeadDim;
+  constexpr int ESZ = (int)sizeof(T);
+  constexpr int R = NW * 32;
+  constexpr int NV = G + 1;                  // G queries + new key
+  constexpr int XV = NV * D * ESZ / 16;      // 16-byte vectors of q + new key
+  constexpr int QV = G * D * ESZ / 16;
+  constexpr int EPV = 16 / ESZ;
+  static_assert(kEThreads == 128, "4 residues x 32 columns");
+  __shared__ __align__(16) float xr[NV * 4 * kXS];
+  __shared__ float sb[NV * 4 * 32];
+
+  // CTA (unit, code word jw): thread (residue s, column 32 jw + lane)
+  const int tid = threadIdx.x, lane = tid & 31, s = tid >> 5;
+  const int u = blockIdx.x / NW, jw = blockIdx.x % NW;
+  const int b = u / p.Hkv, g = u % p.Hkv;
+  const int jc = jw * 32 + lane;
+  const bool early = (p.flags & HATA_FLAG_EARLY_PREFETCH) != 0;
+  // W_H rows s + 4a + 32u4 of column jc: y_jc of warp_dot128 is (S_0 + S_2) + (S_1 + S_3)
+  // with S_s this thread's residue sum
+  auto load_w = [&](const float* Wm, float (&w)[32]) {
+    const float* Wg = Wm + (size_t)g * D * R + jc;
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4)
+#pragma unroll
+      for (int a = 0; a < 8; ++a) w[u4 * 8 + a] = __ldg(Wg + (size_t)(s + 4 * a + 32 * u4) * R);
+  };
+  float wq[32];
+  if (early) {
+    ptx::pdl_launch_dependents();  // the scan kernel may prefetch codes during the preceding kernel
+    load_w(p.Wq, wq);              // the preceding kernel writes no W_H then
+  }
+  ptx::pdl_wait();  // q and the new K row come from the preceding kernel
+  if (!early) {
+    ptx::pdl_launch_dependents();  // the preceding kernel is complete: the scan kernel may read the cache
+    load_w(p.Wq, wq);
+  }
+  const int L = clamp_seq(p.seq_lens[b], p.max_seq);
+  const int nv = L > 0 ? NV : G;
+  const T* qg = static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D;
+  const T* kn = static_cast<const T*>(p.K) + (L > 0 ? token_slot<PAGED>(p, b, g, L - 1) : 0) * D;
+  for (int t = tid; t < (L > 0 ? XV : QV); t += kEThreads) {
+    const uint4 xv = t < QV ? reinterpret_cast<const uint4*>(qg)[t] : reinterpret_cast<const uint4*>(kn)[t - QV];
+    float xe[EPV];
+    Vec16<T>::convert(xv, xe);
+    const int v = t * EPV / D;
+#pragma unroll
+    for (int e = 0; e < EPV; ++e) {
+      const int i = (t * EPV + e) % D;
+      xr[(v * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)] = xe[e];
+    }
+  }
+  __syncthreads();
+  auto residue_sum = [&](const float (&w)[32], int v) {
+    const float* xs_ = xr + (v * 4 + s) * kXS;
+    float P_[8];
+#pragma unroll
+    for (int u4 = 0; u4 < 4; ++u4) {
+      const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
+      const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
+      const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int a = 0; a < 8; ++a) P_[a] = u4 == 0 ? xx[a] * w[u4 * 8 + a] : fmaf(xx[a], w[u4 * 8 + a], P_[a]);
+    }
+    const float q0 = P_[0] + P_[4], q1 = P_[1] + P_[5], q2 = P_[2] + P_[6], q3 = P_[3] + P_[7];
+    sb[(v * 4 + s) * 32 + lane] = (q0 + q2) + (q1 + q3);
+  };
+#pragma unroll
+  for (int v = 0; v < G; ++v) residue_sum(wq, v);
+  if (L > 0) {
+    if (p.Wk == nullptr) {
+      residue_sum(wq, G);
+    } else {
+      float wk[32];
+      load_w(p.Wk, wk);
+      residue_sum(wk, G);
+    }
+  }
+  __syncthreads();
+  if (s == 0) {
+    for (int v = 0; v < nv; ++v) {
+      const float* sv = sb + v * 4 * 32;
+      const float y = (sv[lane] + sv[2 * 32 + lane]) + (sv[32 + lane] + sv[3 * 32 + lane]);
+      const unsigned bits = __ballot_sync(0xffffffffu, y > 0.f);
+      if (lane == 0) {
+        if (v < G) {
+          const size_t o = ((size_t)b * p.Hq + (size_t)g * G + v) * NW + jw;
+          p.qcode_ws[o] = bits;
+          if (p.qcode_out) p.qcode_out[o] = bits;
+        } else {
+          p.codes[token_slot<PAGED>(p, b, g, L - 1) * NW + jw] = bits;  // the cache update
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // scan kernel
 // ---------------------------------------------------------------------------
 template <typename T, int NW, int G, bool PAGED>
 __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
-  constexpr int D = kHeadDim;
-  constexpr int ESZ = (int)sizeof(T);
   constexpr int R = NW * 32;
-  constexpr int NV = G + 1;                  // encoded vectors: G queries + new key
   constexpr int NB = G * R + 1;              // score values
   constexpr int NBP = nbins_padded(G, R);
   constexpr int BPT = (NBP + kSThreads - 1) / kSThreads;
-  constexpr int XV = NV * D * ESZ / 16;      // 16-byte vectors of q + new key
-  constexpr int QV = G * D * ESZ / 16;
-  constexpr int EPV = 16 / ESZ;
   constexpr int PT = kPieceBytes / (NW * 4);  // tokens per piece
-  constexpr int TPP = PT / kSThreads;         // tokens per thread per piece
+  constexpr int TPP = (PT + kSThreads - 1) / kSThreads;  // tokens per thread per piece
   constexpr int BULK_Q = NW >= 4 ? 1 : 4 / NW;  // tokens per 16 bytes
-  static_assert(PT % kSThreads == 0, "whole tokens per thread per piece");
-  static_assert(XV <= kSThreads, "one vector of q / new key per thread");
+  static_assert(kMaxPieces <= 32, "one lane of warp 0 per piece");
   const ScanSmem S = scan_smem(G, NW);
   unsigned char* ring = smem + S.ring;
+  uint32_t* lst = reinterpret_cast<uint32_t*>(smem + S.ring);  // the token-ordered list (the ring is free by then)
   uint16_t* Ds = reinterpret_cast<uint16_t*>(smem + S.D);
-  float* sb = reinterpret_cast<float*>(smem + S.D);  // [NV][4][R] residue sums (before the scores exist)
-  int* hist = reinterpret_cast<int*>(smem + S.hist);
-  float* xr = reinterpret_cast<float*>(smem + S.xr);
+  int* hist = reinterpret_cast<int*>(smem + S.hist);  // counts, then each bin's exclusive prefix
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + S.mbar);  // pieces, then one nothing completes
   __shared__ int s_pre[kMaxB + 1];  // first chunk of batch b: Hkv * sum_{b' < b} ceil(L_b' / C)
   __shared__ int s_len[kMaxB];
-  __shared__ int warp_sums[kNWarp];
-  __shared__ __align__(16) uint32_t qc[NV * NW];
+  __shared__ int warp_sums[kSWarp];
+  __shared__ __align__(16) uint32_t qc[(G + 1) * NW];  // the unit's query codes, then the new key's code
   __shared__ int s_abort, s_Bc, s_below;
   __shared__ int s_blk[PAGED ? kMaxChunkBlocks : 1];  // (paged) pool block of each block the chunk spans
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const StepGeom& geo = p.geo;
   const int C = geo.C;
-  const bool early = (p.flags & HATA_FLAG_EARLY_PREFETCH) != 0;
   const bool test_expire = (p.flags & HATA_FLAG_TEST_EXPIRE_WAIT) != 0;
-  (void)lane;
-  (void)warp;
 
   if (tid == 0) {
-    for (int i = 0; i <= kMaxPieces; ++i) ptx::mbar_init(&mbar[i], 1);
+    for (int i = 0; i < kMaxPieces + 1; ++i) ptx::mbar_init(&mbar[i], 1);
     ptx::fence_mbarrier_init();
     s_abort = 0;
   }
-  if (!early) ptx::pdl_wait();
-  ptx::pdl_launch_dependents();
-  bool waited = !early;
+  // This kernel starts once the encode kernel has passed its own wait on the
+  // preceding kernel (or, with early prefetch, at once): seq_lens and the cached
+  // codes of slots [0, L - 1) are final, so they are read before this kernel waits
+  // for the encode kernel; the query codes, the new key's code and every write come
+  // after that wait.
+  bool waited = false;
 
   // ---- chunk map: batch b holds Hkv * ceil(L_b / C) chunks, units b-major ----------
   {
@@ -261,9 +356,9 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
       int L = 0;
       if (b < p.B) {
         const int raw = p.seq_lens[b];
-        if (raw > p.max_seq && blockIdx.x == 0) set_status(p.status, HATA_ERR_INVALID_ARG);
         L = clamp_seq(raw, p.max_seq);
         s_len[b] = L;
+        if (raw > p.max_seq) s_len[b] = -L - 1;  // flagged once the writes may start
       }
       cnt[e] = p.Hkv * ((L + C - 1) / C);
     }
@@ -278,7 +373,8 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
   const uint64_t pol_stream = ptx::policy_evict_first();
   int enc_u = -1;         // unit whose query codes qc holds
   uint32_t par = 0u;      // bit pc: parity of the phase piece barrier pc completes next
-  int last_np = 0, done_np = 0;  // thread 0: pieces issued for the latest chunk, and waited for
+  int last_np = 0;        // pieces issued for the latest chunk (drained on abort)
+  uint32_t waited_mask = 0u;  // pieces of the latest chunk this thread has waited for
 
   for (int c = blockIdx.x; c < nchunks; c += gridDim.x) {
     // ---- locate the chunk: batch (largest b with s_pre[b] <= c), unit, index ---------
@@ -288,34 +384,35 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
       if (s_pre[mid] <= c) lo = mid;
       else hi = mid - 1;
     }
-    const int b = lo, L = s_len[b];
+    const int b = lo, Ls = s_len[b], L = Ls < 0 ? -Ls - 1 : Ls;
     const int Pb = (L + C - 1) / C;
     const int loc = c - s_pre[b], g = loc / Pb, j = loc % Pb;
     const int u = b * p.Hkv + g;
     const int t0 = j * C, t1 = min(L, t0 + C), len = t1 - t0;
     const int np = (len + PT - 1) / PT;
-    unsigned char* rec = p.rec + (size_t)(u * geo.P + j) * geo.slot_bytes;
+    unsigned char* urec = p.rec + (size_t)u * geo.unit_bytes;  // unit histogram, then the chunk records
+    unsigned char* rec = urec + geo.hist_bytes + (size_t)j * geo.slot_bytes;
     int32_t* rhdr = reinterpret_cast<int32_t*>(rec);
     const bool aborted_before = s_abort != 0;
+    const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
 
-    // ---- 1. the chunk's codes into the ring ------------------------------------------
+    // ---- 1. the chunk's codes into the ring: lane pc of warp 0 issues piece pc -------
     if constexpr (PAGED) {
       if (!aborted_before) {  // block-uniform: the chunk's block numbers, read in parallel
         const int blk0 = t0 >> p.block_shift, nblk = ((t1 - 1) >> p.block_shift) - blk0 + 1;
         for (int i = tid; i < nblk; i += kSThreads) {
           int pb = p.block_table[(size_t)b * p.max_blocks + blk0 + i];
-          if ((unsigned)pb >= (unsigned)p.n_blocks) {
-            set_status(p.status, HATA_ERR_INVALID_ARG);
-            pb = 0;
-          }
+          if ((unsigned)pb >= (unsigned)p.n_blocks) pb = -1;  // flagged below, block 0 used
           s_blk[i] = pb;
         }
         __syncthreads();
       }
     }
-    if (tid == 0 && !aborted_before) {
-      ptx::fence_proxy_async_smem();  // this CTA's earlier generic reads of the ring come first
-      for (int pc = 0; pc < np; ++pc) {
+    if (warp == 0 && !aborted_before) {
+      if (lane == 0) ptx::fence_proxy_async_smem();  // this CTA's earlier generic reads of the ring come first
+      __syncwarp();
+      const int pc = lane;
+      if (pc < np) {
         const int ts = t0 + pc * PT, nt = min(PT, t1 - ts);
         const int nb = nt / BULK_Q * BULK_Q;  // tokens the copy moves (whole 16-byte units)
         ptx::mbar_arrive_expect_tx(&mbar[pc], (uint32_t)nb * NW * 4);
@@ -324,7 +421,7 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
           const int bsz = 1 << p.block_shift, blk0 = t0 >> p.block_shift;
           for (int x0 = 0; x0 < nb;) {
             const int t = ts + x0, seg = min(nb - x0, bsz - (t & (bsz - 1)));
-            const size_t slot = (((size_t)s_blk[(t >> p.block_shift) - blk0] * p.Hkv + g) << p.block_shift) |
+            const size_t slot = (((size_t)max(0, s_blk[(t >> p.block_shift) - blk0]) * p.Hkv + g) << p.block_shift) |
                                 (size_t)(t & (bsz - 1));
             ptx::bulk_g2s(ring + pc * kPieceBytes + (size_t)x0 * NW * 4, p.codes + slot * NW, (uint32_t)seg * NW * 4,
                           &mbar[pc], pol_stream);
@@ -336,99 +433,32 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
                           (uint32_t)nb * NW * 4, &mbar[pc], pol_stream);
         }
       }
-      last_np = np;
-      done_np = 0;
     }
+    last_np = aborted_before ? last_np : np;
+    waited_mask = aborted_before ? waited_mask : 0u;
 
-    // ---- 2. encode the queries (and the new key) -------------------------------------
-    const bool own_last = L > 0 && t0 <= L - 1 && L - 1 < t1;
-    if (!aborted_before && (u != enc_u || own_last)) {
-      // thread item (residue s, column jc) keeps its 32 W values in registers: y_jc of
-      // warp_dot128 is (S_0 + S_2) + (S_1 + S_3) with S_s the residue-s partial sums
-      float wr[32];
-      const float* Wg = p.Wq + (size_t)g * D * R;
-      auto load_w = [&](const float* Wm, int itm, float (&w)[32]) {
-        const int s = (itm >> 5) & 3, jc = (itm >> 7) * 32 + (itm & 31);
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4)
-#pragma unroll
-          for (int a = 0; a < 8; ++a) w[u4 * 8 + a] = __ldg(Wm + (size_t)(s + 4 * a + 32 * u4) * R + jc);
-      };
-      if (tid < 4 * R) load_w(Wg, tid, wr);  // W_H does not depend on the preceding kernel
-      if (!waited) {
-        ptx::pdl_wait();  // q and the new key row come from the preceding kernel
-        waited = true;
-      }
-      const int nvec = own_last ? XV : QV;
-      if (tid < nvec) {
-        uint4 xv;
-        if (tid < QV) {
-          xv = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) + ((size_t)b * p.Hq + (size_t)g * G) * D)[tid];
-        } else {
-          const T* kn = static_cast<const T*>(p.K) + token_slot<PAGED>(p, b, g, L - 1) * D;
-          xv = reinterpret_cast<const uint4*>(kn)[tid - QV];
-        }
-        float xe[EPV];
-        Vec16<T>::convert(xv, xe);
-        const int v = tid * EPV / D;
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) {
-          const int i = (tid * EPV + e) % D;
-          xr[(v * 4 + (i & 3)) * kXS + (i >> 5) * 8 + ((i >> 2) & 7)] = xe[e];
-        }
-      }
-      for (int v = tid; v < BPT * kSThreads; v += kSThreads) hist[v] = 0;
-      __syncthreads();
-      auto residue_sums = [&](const float (&w)[32], int v, int itm) {
-        const int s = (itm >> 5) & 3, jc = (itm >> 7) * 32 + (itm & 31);
-        const float* xs_ = xr + (v * 4 + s) * kXS;
-        float P_[8];
-#pragma unroll
-        for (int u4 = 0; u4 < 4; ++u4) {
-          const float4 x0 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[0];
-          const float4 x1 = reinterpret_cast<const float4*>(xs_ + u4 * 8)[1];
-          const float xx[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-          for (int a = 0; a < 8; ++a) P_[a] = u4 == 0 ? xx[a] * w[u4 * 8 + a] : fmaf(xx[a], w[u4 * 8 + a], P_[a]);
-        }
-        const float q0 = P_[0] + P_[4], q1 = P_[1] + P_[5], q2 = P_[2] + P_[6], q3 = P_[3] + P_[7];
-        sb[(v * 4 + s) * R + jc] = (q0 + q2) + (q1 + q3);
-      };
-      const bool key_from_wq = own_last && p.Wk == nullptr;
-      for (int itm = tid; itm < 4 * R; itm += kSThreads) {
-        if (itm != tid) load_w(Wg, itm, wr);
-#pragma unroll
-        for (int v = 0; v < G; ++v) residue_sums(wr, v, itm);
-        if (key_from_wq) residue_sums(wr, G, itm);
-      }
-      if (own_last && p.Wk != nullptr) {  // block-uniform
-        const float* Wkg = p.Wk + (size_t)g * D * R;
-        for (int itm = tid; itm < 4 * R; itm += kSThreads) {
-          load_w(Wkg, itm, wr);
-          residue_sums(wr, G, itm);
-        }
-      }
-      __syncthreads();
-      const int nv_enc = own_last ? NV : G;
-      for (int pi = warp; pi < nv_enc * NW; pi += kNWarp) {  // one code word per warp item
-        const int v = pi / NW, jw = pi % NW, jc = jw * 32 + lane;
-        const float* sv = sb + v * 4 * R;
-        const float y = (sv[jc] + sv[2 * R + jc]) + (sv[R + jc] + sv[3 * R + jc]);
-        const unsigned bits = __ballot_sync(0xffffffffu, y > 0.f);
-        if (lane == 0) qc[v * NW + jw] = bits;
-      }
-      __syncthreads();
-      enc_u = u;
-      if (j == 0 && tid < G * NW) {
-        const size_t o = ((size_t)b * p.Hq + (size_t)g * G) * NW + tid;
-        p.qcode_ws[o] = qc[tid];
-        if (p.qcode_out) p.qcode_out[o] = qc[tid];
-      }
-      if (own_last && tid < NW) p.codes[token_slot<PAGED>(p, b, g, L - 1) * NW + tid] = qc[G * NW + tid];
-    } else {
-      for (int v = tid; v < BPT * kSThreads; v += kSThreads) hist[v] = 0;
-      __syncthreads();
+    // ---- 2. the query codes (and the new key's code) from the encode kernel ---------
+    if (!waited) {
+      ptx::pdl_wait();  // the encode kernel is complete (and so is the kernel before it)
+      ptx::pdl_launch_dependents();  // the tail kernel may read q and seq_lens before its own wait
+      waited = true;
+      if (blockIdx.x == 0 && tid < p.B && s_len[tid] < 0) set_status(p.status, HATA_ERR_INVALID_ARG);
     }
+    if constexpr (PAGED) {
+      if (!aborted_before) {
+        const int blk0 = t0 >> p.block_shift, nblk = ((t1 - 1) >> p.block_shift) - blk0 + 1;
+        for (int i = tid; i < nblk; i += kSThreads)
+          if (s_blk[i] < 0) set_status(p.status, HATA_ERR_INVALID_ARG);
+      }
+    }
+    if (!aborted_before && (u != enc_u || own_last)) {
+      if (tid < G * NW) qc[tid] = p.qcode_ws[((size_t)b * p.Hq + (size_t)g * G) * NW + tid];
+      if (own_last && tid >= G * NW && tid < (G + 1) * NW)
+        qc[tid] = p.codes[token_slot<PAGED>(p, b, g, L - 1) * NW + (tid - G * NW)];
+      enc_u = u;
+    }
+    for (int v = tid; v < BPT * kSThreads; v += kSThreads) hist[v] = 0;
+    __syncthreads();
 
     // ---- 3. scores + histogram ------------------------------------------------------
     if (!aborted_before) {
@@ -446,7 +476,7 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
           break;
         }
         par ^= 1u << pc;
-        if (tid == 0) done_np = pc + 1;
+        waited_mask |= 1u << pc;
         const int base = pc * PT, nt = min(PT, len - base), nb = nt / BULK_Q * BULK_Q;
         const uint32_t* buf = reinterpret_cast<const uint32_t*>(ring + pc * kPieceBytes);
         uint32_t kw[TPP][NW];
@@ -486,7 +516,8 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
         }
       }
       __syncthreads();
-      // the ring held the old code of slot L - 1 (or part of the new one): rescore it
+      // the ring may hold the old code of slot L - 1 (the encode kernel writes the new
+      // one while the copies run): rescore it with the new code
       if (own_last && tid == 0 && !s_abort) {
         uint32_t keyc[NW];
 #pragma unroll
@@ -506,7 +537,7 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
       __syncthreads();
     }
 
-    // ---- 4. chunk record: cumulative histogram, bound, candidate list ----------------
+    // ---- 4. chunk record: cumulative histogram, bound, candidates sorted by score ----
     if (s_abort) {  // block-uniform (read after a barrier)
       if (tid == 0) {
         rhdr[0] = 0;
@@ -522,6 +553,7 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
     const int want = want_l < geo.cap ? (int)want_l : geo.cap;
     {
       uint16_t* rcum = reinterpret_cast<uint16_t*>(rec + geo.cum_off);
+      uint32_t* uhist = reinterpret_cast<uint32_t*>(urec);
       int hv[BPT], local = 0;
 #pragma unroll
       for (int i = 0; i < BPT; ++i) {
@@ -534,7 +566,11 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
       for (int i = 0; i < BPT; ++i) {
         const int v = tid * BPT + i, before = run;
         run += hv[i];
-        if (v < NBP) rcum[v] = (uint16_t)run;
+        hist[v] = before;  // exclusive prefix: the first sorted position of score v
+        if (v < NBP) {
+          rcum[v] = (uint16_t)run;
+          if (hv[i]) atomicAdd(&uhist[v], (uint32_t)hv[i]);  // the unit's histogram
+        }
         if (before <= want && run > want) {  // the unique first bin whose count passes want
           s_Bc = v;
           s_below = before;
@@ -542,49 +578,70 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
       }
     }
     __syncthreads();
+    const int Bc = s_Bc, below = s_below;
+    const int tie_listed = Bc < NB ? want - below : 0;
+    const int nlisted = below + tie_listed;
     {
-      const int Bc = s_Bc, below = s_below;
-      const int tie_listed = Bc < NB ? want - below : 0;
-      uint32_t* rcand = reinterpret_cast<uint32_t*>(rec + geo.cand_off);
+      // token-ordered list (into the ring, free now): every score below Bc, and the
+      // first tie_listed scores equal to Bc.  Each thread flags its 16 consecutive
+      // scores as bit masks, one block scan places them.
       int lp_carry = 0, ep_carry = 0;
       for (int base = 0; base < len; base += 16 * kSThreads) {  // block-uniform trip count
         const int a = base + tid * 16;
-        uint16_t dv[16];
-        {
-          uint4 v0 = make_uint4(0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu), v1 = v0;
-          if (a < len) {  // a < len: both 16-byte loads stay inside the padded scores
-            v0 = reinterpret_cast<const uint4*>(Ds + a)[0];
-            v1 = reinterpret_cast<const uint4*>(Ds + a)[1];
-          }
-          const uint16_t* h0 = reinterpret_cast<const uint16_t*>(&v0);
-          const uint16_t* h1 = reinterpret_cast<const uint16_t*>(&v1);
+        uint32_t mlt = 0u, meq = 0u;
+        if (a < len) {  // a < len: both 16-byte loads stay inside the padded scores
+          const uint4 v0 = reinterpret_cast<const uint4*>(Ds + a)[0];
+          const uint4 v1 = reinterpret_cast<const uint4*>(Ds + a)[1];
+          const uint32_t w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            dv[i] = a + i < len ? h0[i] : (uint16_t)0xffffu;
-            dv[8 + i] = a + 8 + i < len ? h1[i] : (uint16_t)0xffffu;
+            const int d0 = (int)(w8[i] & 0xffffu), d1 = (int)(w8[i] >> 16);
+            mlt |= (d0 < Bc ? 1u : 0u) << (2 * i) | (d1 < Bc ? 1u : 0u) << (2 * i + 1);
+            meq |= (d0 == Bc ? 1u : 0u) << (2 * i) | (d1 == Bc ? 1u : 0u) << (2 * i + 1);
           }
         }
-        int lt = 0, eq = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          lt += (int)dv[i] < Bc;
-          eq += (int)dv[i] == Bc;
-        }
         int tot;
-        const int pre = block_exclusive_scan<kSThreads>(lt | (eq << 16), warp_sums, &tot);
+        const int pre = block_exclusive_scan<kSThreads>(__popc(mlt) | (__popc(meq) << 16), warp_sums, &tot);
         int lp = lp_carry + (pre & 0xffff), ep = ep_carry + (pre >> 16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int d = dv[i];
-          if (d < Bc || (d == Bc && ep < tie_listed)) rcand[lp + min(ep, tie_listed)] = ((uint32_t)d << 16) | (uint32_t)(a + i);
-          lp += d < Bc;
-          ep += d == Bc;
+        uint32_t mm = mlt | meq;
+        while (mm) {  // the thread's flagged scores, in token order
+          const int i = __ffs(mm) - 1;
+          mm &= mm - 1u;
+          const int m_lt = __popc(mlt & ((1u << i) - 1u)), m_eq = __popc(meq & ((1u << i) - 1u));
+          const int lpi = lp + m_lt, epi = ep + m_eq;
+          const bool is_lt = (mlt >> i) & 1u;
+          if (is_lt || epi < tie_listed)
+            lst[lpi + min(epi, tie_listed)] = ((uint32_t)(is_lt ? 0 : 1) << 31) | (uint32_t)(a + i);
         }
         lp_carry += tot & 0xffff;
         ep_carry += tot >> 16;
       }
+    }
+    __syncthreads();
+    {
+      // sorted by score, equal scores in token order: each listed token first takes a
+      // slot of its score's bin (any order), then its rank inside the bin by token index
+      // (bins are small); the bin starts at the count of lower scores (hist, exclusive)
+      uint32_t* rcand = reinterpret_cast<uint32_t*>(rec + geo.cand_off);
+      uint32_t* tmp = lst + geo.cap;                         // bin slots: offsets, unordered in a bin
+      int* fill = reinterpret_cast<int*>(tmp + geo.cap);     // next free slot of each bin
+      for (int v = tid; v < NBP; v += kSThreads) fill[v] = hist[v];
+      __syncthreads();
+      for (int e = tid; e < nlisted; e += kSThreads) {
+        const uint32_t ent = lst[e];
+        const int off = (int)(ent & 0xffffu), d = (ent >> 31) ? Bc : (int)Ds[off];
+        tmp[atomicAdd(&fill[d], 1)] = ((uint32_t)d << 16) | (uint32_t)off;
+      }
+      __syncthreads();
+      for (int e = tid; e < nlisted; e += kSThreads) {
+        const uint32_t me = tmp[e];
+        const int d = (int)(me >> 16), b0 = hist[d], b1 = fill[d];
+        int rk = 0;
+        for (int x = b0; x < b1; ++x) rk += tmp[x] < me;  // same score: compares the offsets
+        rcand[b0 + rk] = me;
+      }
       if (tid == 0) {
-        rhdr[0] = below + tie_listed;
+        rhdr[0] = nlisted;
         rhdr[1] = Bc;
         rhdr[2] = tie_listed;
         rhdr[3] = len;
@@ -593,9 +650,67 @@ __global__ void __launch_bounds__(kSThreads, 1) step_scan_kernel(const StepParam
     __syncthreads();  // the ring, scores and histogram are free for the next chunk
   }
 
+  if (!waited) ptx::pdl_launch_dependents();  // (no chunk here)
   if (s_abort && tid == 0) {
-    // let the copies of the latest chunk that nobody waited for land (bounded) before exit
-    for (int pc = done_np; pc < last_np; ++pc) ptx::mbar_wait_bounded(&mbar[pc], (par >> pc) & 1u, kWaitTries);
+    // let the copies of the latest chunk that this thread did not wait for land (bounded)
+    for (int pc = 0; pc < last_np; ++pc)
+      if (!((waited_mask >> pc) & 1u)) ptx::mbar_wait_bounded(&mbar[pc], (par >> pc) & 1u, kWaitTries);
+  }
+}
+
+// Selected tokens of a chunk whose candidate list stops short of the threshold T:
+// every token scoring below T, then the first q scoring T, in token order, found by
+// rescoring the chunk's codes from the cache (block-wide; 16 consecutive tokens a
+// thread per pass, scored four at a time, once to count and once to place, which keeps
+// the registers of this rare path low).  The token of selected rank rk in [lo, hi) goes
+// to out[rk].
+template <int NW, int G, bool PAGED>
+__device__ __forceinline__ void rescore_chunk(const StepParams& p, int b, int g, int t0c, int lenc, int Tt, int q,
+                                              int lo, int hi, int* out, const uint32_t* qcs, int* warp_sums) {
+  const int tid = threadIdx.x;
+  GroupQuery<NW, G> gq;
+  gq.init(qcs);
+  auto score_at = [&](int t) {  // score of chunk token t, or INT_MAX past the chunk
+    if (t >= lenc) return INT_MAX;
+    uint32_t kw[NW];
+    load_code<NW>(p.codes + token_slot<PAGED>(p, b, g, t0c + t) * NW, kw);
+    return gq.score(kw, qcs, G);
+  };
+  int lp_carry = 0, ep_carry = 0;
+  for (int base = 0; base < lenc; base += 16 * kTThreads) {
+    const int a = base + tid * 16;
+    int lt = 0, eq = 0;
+#pragma unroll 1
+    for (int i0 = 0; i0 < 16; i0 += 4) {
+      int dv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dv[i] = score_at(a + i0 + i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lt += dv[i] < Tt;
+        eq += dv[i] == Tt;
+      }
+    }
+    int tot;
+    const int pre = block_exclusive_scan<kTThreads>(lt | (eq << 16), warp_sums, &tot);
+    int lp = lp_carry + (pre & 0xffff), ep = ep_carry + (pre >> 16);
+#pragma unroll 1
+    for (int i0 = 0; i0 < 16; i0 += 4) {
+      int dv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dv[i] = score_at(a + i0 + i);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (dv[i] < Tt || (dv[i] == Tt && ep < q)) {
+          const int rk = lp + min(ep, q);
+          if (rk >= lo && rk < hi) out[rk] = t0c + a + i0 + i;
+        }
+        lp += dv[i] < Tt;
+        ep += dv[i] == Tt;
+      }
+    }
+    lp_carry += tot & 0xffff;
+    ep_carry += tot >> 16;
   }
 }
 
@@ -610,11 +725,11 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   constexpr int R = NW * 32;
   constexpr int NB = G * R + 1;
   constexpr int NBP = nbins_padded(G, R);
+  constexpr int BPT = (NBP + kTThreads - 1) / kTThreads;
   constexpr int EPV = 16 / ESZ;
   constexpr int RPR = D * ESZ / 16;          // 16-byte pieces per K or V row
-  constexpr int LT = 16;                     // threads per row in the logits
-  constexpr int LE = D / LT;                 // elements per thread in the logits
-  constexpr int PVG = kTThreads / (D / 2);   // row groups in P.V
+  constexpr int CPL = D / 32;                // columns of a row per lane in the attention
+  constexpr int RPW = G <= 2 ? 4 : (G == 4 ? 2 : 1);  // rows a warp takes at once (register budget)
   constexpr int OPT = (G * D + kTThreads - 1) / kTThreads;
   static_assert((2 * RPR) % 32 == 0, "a row's K and V pieces fill whole warps");
 
@@ -624,7 +739,7 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   const StepGeom& geo = p.geo;
   const int GB = p.GB;
   const TailSmem S = tail_smem(G, NW, ESZ, geo, GB, CS);
-  unsigned char* recs = smem + S.rec;
+  unsigned char* urec = smem + S.rec;  // the unit's histogram, then its chunk records
   T* Kr = reinterpret_cast<T*>(smem + S.Kr);
   T* Vr = reinterpret_cast<T*>(smem + S.Vr);
   float* lg = reinterpret_cast<float*>(smem + S.lg);
@@ -636,18 +751,20 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   uint32_t* qcs = reinterpret_cast<uint32_t*>(smem + S.qcs);
   uint64_t* mb = reinterpret_cast<uint64_t*>(smem + S.mbar);  // [0] records copy, [1] row gathers
   __shared__ int warp_sums[kNWarp];
-  __shared__ int s_T, s_below_all, s_abort;
-  __shared__ int bmaxi[G];
-  __shared__ float redl[PVG * G];
+  __shared__ int s_T, s_below, s_abort, s_uncovered;
   __shared__ float part[G * 2];
 
   const int u = blockIdx.x / CS;
   const int b = u / p.Hkv, g = u % p.Hkv;
+  const uint32_t* uh = reinterpret_cast<const uint32_t*>(urec);
+  auto rec = [&](int c) { return urec + geo.hist_bytes + (size_t)c * geo.slot_bytes; };
+  auto hdr = [&](int c) { return reinterpret_cast<const int32_t*>(rec(c)); };
+  auto cum = [&](int c) { return reinterpret_cast<const uint16_t*>(rec(c) + geo.cum_off); };
+  auto cand = [&](int c) { return reinterpret_cast<const uint32_t*>(rec(c) + geo.cand_off); };
 
+  // Before the wait: the scan kernel passed its own wait before it let this kernel
+  // start, so seq_lens and q are final; only its records are not.
   ptx::cluster_arrive_relaxed();  // completed by the wait before the first remote store
-  ptx::pdl_wait();                // the scan kernel's records are complete and visible
-  ptx::pdl_launch_dependents();
-
   const int L = clamp_seq(p.seq_lens[b], p.max_seq);
   const int n = min(p.k, L);
   const int Pb = (L + geo.C - 1) / geo.C;
@@ -656,86 +773,78 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
     ptx::mbar_init(&mb[1], kTThreads);
     ptx::fence_mbarrier_init();
     s_abort = 0;
-    s_T = NB - 1;
-    if (Pb > 0) {
-      const uint32_t bytes = (uint32_t)Pb * geo.slot_bytes;
-      ptx::mbar_arrive_expect_tx(&mb[0], bytes);
-      ptx::bulk_g2s(recs, p.rec + (size_t)u * geo.P * geo.slot_bytes, bytes, &mb[0], ptx::policy_evict_first());
-    }
   }
   for (int e = tid; e < G * D; e += kTThreads)
     xp[e] = to_f32<T>(static_cast<const T*>(p.q)[((size_t)b * p.Hq + (size_t)g * G) * D + e]);
-  if (tid < G * NW) qcs[tid] = p.qcode_ws[((size_t)b * p.Hq + (size_t)g * G) * NW + tid];
   if (tid < G) {
     part[2 * tid] = -INFINITY;
     part[2 * tid + 1] = 0.f;
-    bmaxi[tid] = ord_of(-INFINITY);
   }
+  ptx::pdl_wait();  // the scan kernel's records are complete and visible
+  ptx::pdl_launch_dependents();
+  if (tid == 0 && Pb > 0) {
+    const uint32_t bytes = geo.hist_bytes + (uint32_t)Pb * geo.slot_bytes;
+    ptx::mbar_arrive_expect_tx(&mb[0], bytes);
+    ptx::bulk_g2s(urec, p.rec + (size_t)u * geo.unit_bytes, bytes, &mb[0], ptx::policy_evict_first());
+  }
+  if (tid < G * NW) qcs[tid] = p.qcode_ws[((size_t)b * p.Hq + (size_t)g * G) * NW + tid];
   __syncthreads();  // the barrier initialisation is visible before anyone waits on it
   if (Pb > 0 && !ptx::mbar_wait_spin(&mb[0], 0u, kWaitTries)) {
     set_status(p.status, HATA_ERR_TIMEOUT);
     s_abort = 1;
   }
   __syncthreads();
-  auto hdr = [&](int c) { return reinterpret_cast<const int32_t*>(recs + (size_t)c * geo.slot_bytes); };
-  auto cum = [&](int c) { return reinterpret_cast<const uint16_t*>(recs + (size_t)c * geo.slot_bytes + geo.cum_off); };
-  auto cand = [&](int c) { return reinterpret_cast<const uint32_t*>(recs + (size_t)c * geo.slot_bytes + geo.cand_off); };
   if (!s_abort)
     for (int c = tid; c < Pb; c += kTThreads)
       if ((uint32_t)hdr(c)[3] & kAbortBit) s_abort = 1;  // the scan gave up (its status is set)
+  if (tid == 0) {
+    s_T = NB - 1;
+    s_below = 0;
+    s_uncovered = 0;
+  }
   __syncthreads();
   const bool active = !s_abort && n > 0;
 
-  // ---- 5. threshold T, tie quota m, each chunk's share of the selection -------------
+  // ---- 5. threshold T (one scan of the unit histogram), each chunk's share ---------
   if (active) {
-    int best = INT_MAX;
-    for (int v8 = tid; v8 < NBP / 8; v8 += kTThreads) {
-      int tot[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int c = 0; c < Pb; ++c) {
-        const uint4 w = reinterpret_cast<const uint4*>(cum(c))[v8];
-        tot[0] += (int)(w.x & 0xffffu); tot[1] += (int)(w.x >> 16);
-        tot[2] += (int)(w.y & 0xffffu); tot[3] += (int)(w.y >> 16);
-        tot[4] += (int)(w.z & 0xffffu); tot[5] += (int)(w.z >> 16);
-        tot[6] += (int)(w.w & 0xffffu); tot[7] += (int)(w.w >> 16);
-      }
+    int hv[BPT], local = 0;
 #pragma unroll
-      for (int e = 7; e >= 0; --e)
-        if (tot[e] >= n) best = v8 * 8 + e;
-      if (best != INT_MAX) break;  // later groups of this thread are higher
+    for (int i = 0; i < BPT; ++i) {
+      const int v = tid * BPT + i;
+      hv[i] = v < NBP ? (int)uh[v] : 0;
+      local += hv[i];
     }
-    if (best != INT_MAX) atomicMin(&s_T, best);
+    int total;
+    int run = block_exclusive_scan<kTThreads>(local, warp_sums, &total);
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int v = tid * BPT + i, before = run;
+      run += hv[i];
+      if (before < n && run >= n && v < NB) {  // the unique first score whose count reaches n
+        s_T = v;
+        s_below = before;
+      }
+    }
   }
   __syncthreads();
   const int Tt = s_T;
   if (active && warp == 0) {
-    // per chunk (lane c of each 32-chunk group): counts below T and at T, then prefix sums
-    int below_all = 0;
-    for (int c0 = 0; c0 < Pb; c0 += 32) {
-      const int c = c0 + lane;
-      int bl = 0, te = 0;
-      if (c < Pb) {
-        bl = Tt > 0 ? (int)cum(c)[Tt - 1] : 0;
-        te = (int)cum(c)[Tt] - bl;
-      }
-      below_all += __reduce_add_sync(0xffffffffu, bl);
-    }
-    const int m = n - below_all;  // ties at T that are selected
+    const int m = n - s_below;  // ties at T that are selected
     int tie_run = 0, sel_run = 0;
-    for (int c0 = 0; c0 < Pb; c0 += 32) {
+    for (int c0 = 0; c0 < Pb; c0 += 32) {  // lane c of each 32-chunk group
       const int c = c0 + lane;
       int bl = 0, te = 0;
       if (c < Pb) {
         bl = Tt > 0 ? (int)cum(c)[Tt - 1] : 0;
         te = (int)cum(c)[Tt] - bl;
       }
-      int ti = te;  // inclusive scan of the ties
+      int ti = te;  // inclusive scans of the ties and of the selected counts
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, ti, o);
         if (lane >= o) ti += y;
       }
-      const int ties_before = tie_run + ti - te;
-      const int q = max(0, min(m - ties_before, te));
+      const int q = max(0, min(m - (tie_run + ti - te), te));
       const int sel = bl + q;
       int si = sel;
 #pragma unroll
@@ -744,6 +853,8 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
         if (lane >= o) si += y;
       }
       if (c < Pb) {
+        // the list (sorted by score, ties in token order) holds the selection as its
+        // first sel entries when T < Bc, or when T == Bc and the quota fits the ties listed
         const int32_t* h = hdr(c);
         const int Bc = h[1], tl = h[2];
         const bool covered = Tt < Bc || (Tt == Bc && q <= tl);
@@ -751,6 +862,7 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
         sst[4 * c + 1] = sel;
         sst[4 * c + 2] = q;
         sst[4 * c + 3] = covered ? 1 : 0;
+        if (!covered && sel > 0) s_uncovered = 1;
       }
       tie_run += __shfl_sync(0xffffffffu, ti, 31);
       sel_run += __shfl_sync(0xffffffffu, si, 31);
@@ -765,94 +877,72 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   float oacc[OPT];
 #pragma unroll
   for (int q = 0; q < OPT; ++q) oacc[q] = 0.f;
+  // Flash decode per warp: warp w takes rows w, w + 16, ... of every batch (RPW at a
+  // time), keeping per head a running maximum and sum (warp-uniform) and the weighted
+  // sum of V for the lane's columns CPL lane .. CPL lane + CPL - 1.  Exp2 domain: the
+  // logits are scaled by scale * log2(e).
+  float wm[G], wsum[G], wo[G][CPL], xq[G][CPL];
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    wm[h] = -INFINITY;
+    wsum[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) wo[h][e] = 0.f;
+  }
   uint32_t gphase = 0;
   const T* Kg = static_cast<const T*>(p.K);
   const T* Vg = static_cast<const T*>(p.V);
+  // a row index outside [0, L) is never expected: it is flagged and row 0 used instead
+  auto checked = [&](int t) {
+    if ((unsigned)t >= (unsigned)L) {
+      set_status(p.status, HATA_ERR_INVALID_ARG);
+      t = 0;
+    }
+    return t;
+  };
   for (int cur = r0; cur < r1; cur += GB) {  // block-uniform
     const int end = min(r1, cur + GB), nr = end - cur;
-    // rows of the ranks [cur, end): covered chunks from their lists (one warp per chunk)
-    for (int c = warp; c < Pb; c += kNWarp) {
-      const int sb0 = sst[4 * c], sel = sst[4 * c + 1], q = sst[4 * c + 2];
-      if (!sst[4 * c + 3] || sb0 + sel <= cur || sb0 >= end) continue;  // warp-uniform
-      const int lo = max(0, cur - sb0), hi = min(sel, end - sb0);
-      const int nl = min(hdr(c)[0], geo.cap);
-      const uint32_t* lst = cand(c);
-      const int t0c = c * geo.C;
-      const unsigned lm = (1u << lane) - 1u;
-      int lt_run = 0, eq_run = 0;
-      for (int e0 = 0; e0 < nl; e0 += 32) {
-        const int e = e0 + lane;
-        const uint32_t ent = e < nl ? lst[e] : 0xffffffffu;
-        const int d = (int)(ent >> 16);
-        const bool lt = e < nl && d < Tt, eq = e < nl && d == Tt;
-        const unsigned blt = __ballot_sync(0xffffffffu, lt), beq = __ballot_sync(0xffffffffu, eq);
-        const int ltpre = lt_run + __popc(blt & lm), eqpre = eq_run + __popc(beq & lm);
-        const int rk = ltpre + min(eqpre, q);
-        if ((lt || (eq && eqpre < q)) && rk >= lo && rk < hi) rowtok[sb0 + rk - cur] = t0c + (int)(ent & 0xffffu);
-        lt_run += __popc(blt);
-        eq_run += __popc(beq);
-        if (lt_run + min(eq_run, q) >= hi) break;  // warp-uniform
-      }
-    }
-    // chunks whose list stops short of T: rescore from the cache (block-wide, in order)
-    for (int c = 0; c < Pb; ++c) {
+    // chunks whose list stops short of T: rescore from the cache (block-wide, in token order)
+    for (int c = 0; s_uncovered && c < Pb; ++c) {
       const int sb0 = sst[4 * c], sel = sst[4 * c + 1], q = sst[4 * c + 2];
       if (sst[4 * c + 3] || sb0 + sel <= cur || sb0 >= end) continue;  // block-uniform
-      const int lo = max(0, cur - sb0), hi = min(sel, end - sb0);
-      const int t0c = c * geo.C, lenc = min(geo.C, L - t0c);
-      GroupQuery<NW, G> gq;
-      gq.init(qcs);
-      int lp_carry = 0, ep_carry = 0;
-      for (int base = 0; base < lenc; base += 16 * kTThreads) {
-        const int a = base + tid * 16;
-        int dv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          dv[i] = INT_MAX;
-          if (a + i < lenc) {
-            uint32_t kw[NW];
-            load_code<NW>(p.codes + token_slot<PAGED>(p, b, g, t0c + a + i) * NW, kw);
-            dv[i] = gq.score(kw, qcs, G);
-          }
-        }
-        int lt = 0, eq = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          lt += dv[i] < Tt;
-          eq += dv[i] == Tt;
-        }
-        int tot;
-        const int pre = block_exclusive_scan<kTThreads>(lt | (eq << 16), warp_sums, &tot);
-        int lp = lp_carry + (pre & 0xffff), ep = ep_carry + (pre >> 16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (dv[i] < Tt || (dv[i] == Tt && ep < q)) {
-            const int rk = lp + min(ep, q);
-            if (rk >= lo && rk < hi) rowtok[sb0 + rk - cur] = t0c + a + i;
-          }
-          lp += dv[i] < Tt;
-          ep += dv[i] == Tt;
-        }
-        lp_carry += tot & 0xffff;
-        ep_carry += tot >> 16;
+      rescore_chunk<NW, G, PAGED>(p, b, g, c * geo.C, min(geo.C, L - c * geo.C), Tt, q, max(0, cur - sb0),
+                                  min(sel, end - sb0), rowtok + sb0 - cur, qcs, warp_sums);
+    }
+    // covered chunks: rank rk of chunk c is entry rk - sb0 of its sorted list
+    for (int i = tid; i < nr; i += kTThreads) {
+      const int rk = cur + i;
+      int c = 0;  // the chunk holding selected rank rk (chunks of an empty share are skipped)
+      for (int x = 1; x < Pb; ++x)
+        if (sst[4 * x] <= rk) c = x;
+      if (sst[4 * c + 3]) {
+        const uint32_t ent = cand(c)[min(rk - sst[4 * c], geo.cap - 1)];
+        rowtok[i] = c * geo.C + (int)(ent & 0xffffu);
       }
     }
     __syncthreads();
-    // indices (ascending: ranks follow token order) and the row gathers
-    // a row index outside [0, L) is never expected: it is flagged and row 0 used instead
-    auto checked = [&](int t) {
-      if ((unsigned)t >= (unsigned)L) {
-        set_status(p.status, HATA_ERR_INVALID_ARG);
-        t = 0;
-      }
-      return t;
-    };
-    if (ix || PAGED) {
+    // indices in ascending token order (selected ranks of a chunk follow its tokens)
+    if (ix) {
       for (int i = tid; i < nr; i += kTThreads) {
-        if (ix) ix[cur + i] = rowtok[i];
-        if constexpr (PAGED) rowslot[i] = (long long)token_slot<true>(p, b, g, checked(rowtok[i]));
+        const int rk = cur + i;
+        int c = 0;
+        for (int x = 1; x < Pb; ++x)
+          if (sst[4 * x] <= rk) c = x;
+        int pos = rk;
+        if (sst[4 * c + 3]) {  // a sorted list: the rank among the chunk's selected tokens by token index
+          const uint32_t* lst = cand(c);
+          const int sel = min(sst[4 * c + 1], geo.cap), me = rk - sst[4 * c];
+          const uint32_t mo = lst[min(me, geo.cap - 1)] & 0xffffu;
+          int before = 0;
+          for (int e = 0; e < sel; ++e) before += (lst[e] & 0xffffu) < mo;
+          pos = sst[4 * c] + before;
+        }
+        ix[pos] = rowtok[i];
       }
-      if constexpr (PAGED) __syncthreads();
+    }
+    if constexpr (PAGED) {
+      for (int i = tid; i < nr; i += kTThreads) rowslot[i] = (long long)token_slot<true>(p, b, g, checked(rowtok[i]));
+      __syncthreads();
     }
     for (int e = tid; e < nr * 2 * RPR; e += kTThreads) {
       const int r = e / (2 * RPR), w = e % (2 * RPR);
@@ -872,129 +962,108 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
     __syncthreads();
     if (s_abort) break;  // block-uniform (read after the barrier)
 
-    // logits (exp2 domain): 16 threads per row, 8 elements each, every head at once
-    {
-      const int sgi = lane % LT;
-      float xq[G][LE];
+    if (cur == r0) {  // the lane's slice of the queries (xp is ready long before)
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int e = 0; e < LE; ++e) xq[h][e] = xp[h * D + sgi * LE + e];
-      float mx[G];
+        for (int e = 0; e < CPL; ++e) xq[h][e] = xp[h * D + CPL * lane + e];
+    }
+    for (int rb = warp; rb < nr; rb += RPW * kNWarp) {  // warp-uniform
+      float lgt[RPW][G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
-      for (int rb = warp * (32 / LT); rb < nr; rb += kNWarp * (32 / LT)) {  // warp-uniform
-        const int r = rb + lane / LT;
-        const bool valid = r < nr;
-        const int rr = valid ? r : 0;
-        float kv[LE];
-#pragma unroll
-        for (int v = 0; v < LE / EPV; ++v) {
-          float t8[EPV];
-          Vec16<T>::convert(*reinterpret_cast<const uint4*>(Kr + (size_t)rr * D + sgi * LE + v * EPV), t8);
-#pragma unroll
-          for (int e = 0; e < EPV; ++e) kv[v * EPV + e] = t8[e];
+      for (int i = 0; i < RPW; ++i) {
+        const int r = min(rb + i * kNWarp, nr - 1);
+        float kv[CPL];
+        if constexpr (ESZ == 2) {
+          const uint2 w2 = *reinterpret_cast<const uint2*>(Kr + (size_t)r * D + CPL * lane);
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.y));
+          kv[0] = f0.x; kv[1] = f0.y; kv[2] = f1.x; kv[3] = f1.y;
+        } else {
+          const float4 f = *reinterpret_cast<const float4*>(Kr + (size_t)r * D + CPL * lane);
+          kv[0] = f.x; kv[1] = f.y; kv[2] = f.z; kv[3] = f.w;
         }
-        float acc[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float a = xq[h][0] * kv[0];
 #pragma unroll
-          for (int e = 1; e < LE; ++e) a = fmaf(xq[h][e], kv[e], a);
-          acc[h] = a;
+          for (int e = 1; e < CPL; ++e) a = fmaf(xq[h][e], kv[e], a);
+          lgt[i][h] = a;
         }
+      }
 #pragma unroll
-        for (int o = 1; o < LT; o <<= 1)
+      for (int o = 16; o; o >>= 1)
 #pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-        if (valid && sgi == 0) {
+        for (int i = 0; i < RPW; ++i)
+#pragma unroll
+          for (int h = 0; h < G; ++h) lgt[i][h] += __shfl_xor_sync(0xffffffffu, lgt[i][h], o);
+#pragma unroll
+      for (int i = 0; i < RPW; ++i) {
+        const int r = rb + i * kNWarp;
+        if (r < nr) {  // warp-uniform
+          float vv[CPL];
+          if constexpr (ESZ == 2) {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(Vr + (size_t)r * D + CPL * lane);
+            const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.x));
+            const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.y));
+            vv[0] = f0.x; vv[1] = f0.y; vv[2] = f1.x; vv[3] = f1.y;
+          } else {
+            const float4 f = *reinterpret_cast<const float4*>(Vr + (size_t)r * D + CPL * lane);
+            vv[0] = f.x; vv[1] = f.y; vv[2] = f.z; vv[3] = f.w;
+          }
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float lv = acc[h] * p.scale_log2;
-            lg[h * GB + r] = lv;
-            mx[h] = fmaxf(mx[h], lv);
+            const float l = lgt[i][h] * p.scale_log2;
+            const float mn = fmaxf(wm[h], l);
+            const float alpha = exp2f(wm[h] - mn);  // 0 while the maximum is -inf
+            const float pr = exp2f(l - mn);
+            wsum[h] = fmaf(wsum[h], alpha, pr);
+#pragma unroll
+            for (int e = 0; e < CPL; ++e) wo[h][e] = fmaf(wo[h][e], alpha, pr * vv[e]);
+            wm[h] = mn;
           }
         }
       }
+    }
+    __syncthreads();  // every warp is done with the K and V rows of this batch
+  }
+  // combine the warps' partials through shared memory (the K rows' buffer, free now)
+  {
+    constexpr int WS = D + 2;  // per warp and head: the D columns, then the maximum and sum
+    float* wbuf = reinterpret_cast<float*>(Kr);  // [kNWarp][G][WS]
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], LT));
-        if (lane == 0 && mx[h] != -INFINITY) atomicMax(&bmaxi[h], ord_of(mx[h]));
+    for (int h = 0; h < G; ++h) {
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) wbuf[(warp * G + h) * WS + CPL * lane + e] = wo[h][e];
+      if (lane == 0) {
+        wbuf[(warp * G + h) * WS + D] = wm[h];
+        wbuf[(warp * G + h) * WS + D + 1] = wsum[h];
       }
     }
     __syncthreads();
-    // softmax against the running maximum, then P.V: thread (column pair cp, row
-    // group rg) sums rows rg, rg + PVG, ...; the PVG partial sums meet in shared
-    // memory (the K rows' buffer, free once the logits are done)
-    for (int e = tid; e < G * nr; e += kTThreads) {
-      const int h = e / nr, i = e - h * nr;
-      const float mn = fmaxf(part[2 * h], float_of_ord(bmaxi[h]));
-      lg[h * GB + i] = exp2f(lg[h * GB + i] - mn);
-    }
-    __syncthreads();
-    {
-      const int cp = tid % (D / 2), rg = tid / (D / 2);
-      float pacc[G][2], lsum[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
-#pragma unroll 4
-      for (int r = rg; r < nr; r += PVG) {
-        float v0, v1;
-        if constexpr (ESZ == 2) {
-          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * D)[cp]);
-          v0 = f.x;
-          v1 = f.y;
-        } else {
-          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * D)[cp];
-          v0 = f.x;
-          v1 = f.y;
+    for (int q = 0; q < OPT; ++q) {
+      const int e = tid + q * kTThreads;
+      if (e < G * D) {
+        const int h = e / D, col = e % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kNWarp; ++w) M = fmaxf(M, wbuf[(w * G + h) * WS + D]);
+        float l = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kNWarp; ++w) {
+            const float sc = exp2f(wbuf[(w * G + h) * WS + D] - M);
+            l = fmaf(wbuf[(w * G + h) * WS + D + 1], sc, l);
+            o = fmaf(wbuf[(w * G + h) * WS + col], sc, o);
+          }
         }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float pr_ = lg[h * GB + r];
-          pacc[h][0] = fmaf(pr_, v0, pacc[h][0]);
-          pacc[h][1] = fmaf(pr_, v1, pacc[h][1]);
-          lsum[h] += pr_;
+        oacc[q] = o;
+        if (col == 0) {
+          part[2 * h] = M;
+          part[2 * h + 1] = l;
         }
       }
-      float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
-      if (cp == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) redl[rg * G + h] = lsum[h];
-    }
-    __syncthreads();
-    {
-      const float* red = reinterpret_cast<const float*>(Kr);
-#pragma unroll
-      for (int q = 0; q < OPT; ++q) {
-        const int e = tid + q * kTThreads;
-        if (e < G * D) {
-          const int h = e / D, i = e % D;
-          const float m_old = part[2 * h];
-          const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
-          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
-          float sum = 0.f;
-#pragma unroll
-          for (int jg = 0; jg < PVG; ++jg) sum += red[((size_t)jg * G + h) * D + i];
-          oacc[q] = fmaf(oacc[q], alpha, sum);
-        }
-      }
-    }
-    __syncthreads();  // every thread has read the running maxima and the partial sums
-    if (tid < G) {
-      const int h = tid;
-      const float m_old = part[2 * h];
-      const float mn = fmaxf(m_old, float_of_ord(bmaxi[h]));
-      const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
-      float ls = 0.f;
-#pragma unroll
-      for (int jg = 0; jg < PVG; ++jg) ls += redl[jg * G + h];
-      part[2 * h + 1] = part[2 * h + 1] * alpha + ls;
-      part[2 * h] = mn;
-      bmaxi[h] = ord_of(-INFINITY);
     }
     __syncthreads();
   }
@@ -1025,22 +1094,33 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
     if (s_abort) v = (w & 1) ? 0.f : -INFINITY;
     ptx::st_dsmem_f32(ptx::dsmem_addr(&mslot[rank * stride + w], owner), v);
   }
-  ptx::cluster_sync();  // every CTA holds the partials of its columns
+  ptx::cluster_sync();  // every CTA holds the partials of its columns; every records copy has landed
+  if (rank == 0 && Pb > 0)  // the unit's histogram starts at zero for the next call
+    for (int v = tid; v < NBP; v += kTThreads) reinterpret_cast<uint32_t*>(p.rec + (size_t)u * geo.unit_bytes)[v] = 0u;
   for (int col = tid; col < mc; col += kTThreads) {
     const int e = rank * mc + col;
     if (e < G * D) {
       const int h = e / D;
+      // every source's (max, sum, column) first, then the log-sum-exp merge (no branches,
+      // so the loads of all sources are in flight together)
+      float mv[kMaxCS], lv[kMaxCS], ov[kMaxCS];
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) {
+        const int cc = min(c, CS - 1);
+        mv[c] = c < CS ? mslot[cc * stride + 2 * h] : -INFINITY;
+        lv[c] = mslot[cc * stride + 2 * h + 1];
+        ov[c] = mslot[cc * stride + 2 * G + col];
+      }
       float M = -INFINITY;
-      for (int c = 0; c < CS; ++c) M = fmaxf(M, mslot[c * stride + 2 * h]);
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) M = fmaxf(M, mv[c]);
       float l = 0.f, o = 0.f;
-      if (M != -INFINITY)
-        for (int c = 0; c < CS; ++c) {
-          const float mv = mslot[c * stride + 2 * h];
-          if (mv == -INFINITY) continue;
-          const float w = exp2f(mv - M);
-          l = fmaf(mslot[c * stride + 2 * h + 1], w, l);
-          o = fmaf(mslot[c * stride + 2 * G + col], w, o);
-        }
+#pragma unroll
+      for (int c = 0; c < kMaxCS; ++c) {
+        const float w = mv[c] == -INFINITY ? 0.f : exp2f(mv[c] - M);
+        l = fmaf(lv[c], w, l);
+        o = fmaf(ov[c], w, o);
+      }
       static_cast<T*>(p.out)[((size_t)b * p.Hq + (size_t)g * G + h) * D + (e % D)] =
           from_f32<T>(l > 0.f ? o / l : 0.f);
     }
@@ -1100,6 +1180,9 @@ cudaError_t configure(const void* kern, int* max_dyn) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     }
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    // every kernel of the step asks for the largest shared-memory carveout, so an SM that
+    // runs one of them can take a CTA of the next one without reconfiguring
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) (void)cudaGetLastError();
     it = done.emplace(std::make_pair(kern, dev), std::make_pair(e, dyn)).first;
   }
@@ -1149,8 +1232,9 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
   const int cmax = kRingBytes / (NW * 4);
   // chunk slots per unit: spread the units over every SM, chunks of at least kMinChunk
   // tokens and at most one ring
+  const long long scan_sms = sms;  // the encode CTAs are small enough to share SMs with the scan
   long long P = (d.max_seq + cmax - 1) / cmax;
-  if (U < sms) P = std::max<long long>(P, sms / U);
+  if (U < scan_sms) P = std::max<long long>(P, scan_sms / U);
   P = std::min<long long>(P, std::max<long long>(1, (d.max_seq + kMinChunk - 1) / kMinChunk));
   P = std::max<long long>(P, (d.max_seq + cmax - 1) / cmax);
   long long C = ((d.max_seq + P - 1) / P + 15) / 16 * 16;
@@ -1159,14 +1243,19 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
   StepGeom geo{};
   geo.C = (int)C;
   geo.P = (int)P;
-  geo.cap = (int)((std::min<long long>(C, (long long)k + 64) + 3) / 4 * 4);
   geo.nbp = nbins_padded(G, R);
+  // list capacity: the tokens a chunk can list (a list stopping short of the threshold
+  // is rescored in the tail); the scan sorts it in its ring: two lists and a bin counter each
+  geo.cap = (int)((std::min<long long>(C, (long long)k + 64) + 3) / 4 * 4);
+  geo.cap = std::min(geo.cap, (kRingBytes - geo.nbp * 4) / 8 / 4 * 4);
   geo.cum_off = 16;
   geo.cand_off = (uint32_t)(16 + geo.nbp * 2);
   geo.slot_bytes = (uint32_t)(geo.cand_off + geo.cap * 4);
-  if (U * P > 0x7fffffffLL / geo.slot_bytes) return pl;
+  geo.hist_bytes = (uint32_t)(geo.nbp * 4);
+  geo.unit_bytes = geo.hist_bytes + (uint32_t)P * geo.slot_bytes;
+  if ((long long)P * geo.slot_bytes > 0x7fffffffLL || U > 0x7fffffffLL / geo.unit_bytes) return pl;
   pl.geo = geo;
-  pl.scan_grid = (int)std::min<long long>(U * P, sms);
+  pl.scan_grid = (int)std::min<long long>(U * P, scan_sms);
   pl.scan_smem = (size_t)scan_smem(G, NW).total;
   int dyn_scan = 0, dyn_scan_p = 0, dyn_tail = 0, dyn_tail_p = 0;
   if (configure((const void*)step_scan_kernel<T, NW, G, false>, &dyn_scan) != cudaSuccess ||
@@ -1201,7 +1290,7 @@ Plan make_plan_t(const hata_dims_t& d, int k) {
   pl.CS = bestCS;
   pl.GB = bestGB;
   pl.tail_smem = best_smem;
-  pl.ws_bytes = align_up((size_t)U * P * geo.slot_bytes, kAlign) + align_up((size_t)d.batch * d.n_q_heads * NW * 4, kAlign);
+  pl.ws_bytes = align_up((size_t)U * geo.unit_bytes, kAlign) + align_up((size_t)d.batch * d.n_q_heads * NW * 4, kAlign);
   pl.ok = true;
   return pl;
 }
@@ -1242,21 +1331,30 @@ struct PlanFn {
 
 template <typename T, int NW, int G, bool PAGED>
 cudaError_t launch_t(const Plan& pl, const hata_dims_t& d, const StepParams& prm, cudaStream_t st) {
+  auto enc = step_encode_kernel<T, NW, G, PAGED>;
   auto scan = step_scan_kernel<T, NW, G, PAGED>;
   auto tail = step_tail_kernel<T, NW, G, PAGED>;
-  cudaError_t e = configure((const void*)scan, nullptr);
+  cudaError_t e = configure((const void*)enc, nullptr);
+  if (e == cudaSuccess) e = configure((const void*)scan, nullptr);
   if (e == cudaSuccess) e = configure((const void*)tail, nullptr);
   if (e != cudaSuccess) return e;
+  // all three are launched with programmatic dependent launch: each may start while
+  // the kernel before it runs and waits (griddepcontrol.wait) before using its results
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)pl.scan_grid, 1, 1);
-  cfg.blockDim = dim3(kSThreads, 1, 1);
-  cfg.dynamicSmemBytes = pl.scan_smem;
+  cfg.gridDim = dim3((unsigned)(d.batch * d.n_kv_heads * NW), 1, 1);
+  cfg.blockDim = dim3(kEThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, enc, prm);
+  if (e != cudaSuccess) return e;
+  cfg.gridDim = dim3((unsigned)pl.scan_grid, 1, 1);
+  cfg.blockDim = dim3(kSThreads, 1, 1);
+  cfg.dynamicSmemBytes = pl.scan_smem;
   e = cudaLaunchKernelEx(&cfg, scan, prm);
   if (e != cudaSuccess) return e;
   at[1].id = cudaLaunchAttributeClusterDimension;
@@ -1334,8 +1432,8 @@ cudaError_t launch_split_step(const hata_dims_t& d, const WsLayout& L, const voi
   prm.idx_out = idx_out;
   prm.status = reinterpret_cast<uint32_t*>(ws + L.status);
   prm.rec = reinterpret_cast<unsigned char*>(ws + L.fused);
-  prm.qcode_ws = reinterpret_cast<uint32_t*>(ws + L.fused + align_up((size_t)d.batch * d.n_kv_heads * pl.geo.P *
-                                                                        pl.geo.slot_bytes, kAlign));
+  prm.qcode_ws = reinterpret_cast<uint32_t*>(ws + L.fused + align_up((size_t)d.batch * d.n_kv_heads *
+                                                                        pl.geo.unit_bytes, kAlign));
   prm.B = d.batch;
   prm.Hq = d.n_q_heads;
   prm.Hkv = d.n_kv_heads;

@@ -113,6 +113,15 @@ typedef struct {
  * workspace (hata_workspace_init). */
 #define HATA_FLAG_TEST_EXPIRE_WAIT 2
 
+/* The decode step has two fused forms with identical results.  The cluster form
+ * (one launch; a thread-block cluster of up to 16 SMs per (batch, KV head) unit,
+ * every exchange on chip) is used while the units are few.  The all-SM form (an
+ * encode kernel, a scan kernel that spreads every unit's cache over all SMs, and
+ * a tail kernel with one cluster per unit, chained by programmatic dependent
+ * launch) is used for 64 or more units and for paged caches.  This flag selects
+ * the all-SM form for any shape it covers. */
+#define HATA_FLAG_ALL_SM_SCAN 4
+
 /* Bytes of workspace that every call below needs for these dims and budget k
  * (one size serves all calls).  Returns HATA_OK and writes *bytes. */
 HATA_API hata_status_t hata_workspace_size(const hata_dims_t* dims, int k, size_t* bytes);

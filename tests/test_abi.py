@@ -143,5 +143,9 @@ def test_unknown_flags_rejected(H):
     n = ctypes.c_size_t(0)
     d = H.dims_for(1, 32, 8, 128, 128, 1024, "bf16", flags=H.HATA_FLAG_EARLY_PREFETCH)
     assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 0
-    d.flags = 6
-    assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 1
+    for known in (H.HATA_FLAG_TEST_EXPIRE_WAIT, H.HATA_FLAG_ALL_SM_SCAN, 7):
+        d.flags = known
+        assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 0
+    for unknown in (8, 1 | 16, 1 << 30):
+        d.flags = unknown
+        assert H.lib.hata_workspace_size(ctypes.byref(d), 512, ctypes.byref(n)) == 1

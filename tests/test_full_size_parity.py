@@ -53,11 +53,12 @@ def test_decode_step_full_size(H, name):
     assert H.hata_read_device_status(got["ws"]) == 0
 
 
-def test_decode_step_full_size_early_prefetch(H):
-    """The headline shape with the early-prefetch launch flag (codes streamed before
-    the preceding kernel finishes) gives the same results."""
+@pytest.mark.parametrize("flags", [1, 4, 5])
+def test_decode_step_full_size_other_launch_forms(H, flags):
+    """The headline shape with early prefetch (codes streamed before the preceding
+    kernel finishes), in the all-SM form, and both: the same results."""
     wl, inp, codes0 = _inputs("llama8b_128k")
-    got = run_step(H, wl, inp, codes0, flags=H.HATA_FLAG_EARLY_PREFETCH)
+    got = run_step(H, wl, inp, codes0, flags=flags)
     check_step(wl, inp, codes0, got)
     assert H.hata_read_device_status(got["ws"]) == 0
 

@@ -306,22 +306,27 @@ STEP_CASES = {
 }
 
 
+FORMS = {"auto": 0, "all_sm": 4}  # the planner's choice, and the all-SM form forced (HATA_FLAG_ALL_SM_SCAN)
+
+
+@pytest.mark.parametrize("form", list(FORMS))
 @pytest.mark.parametrize("name", list(STEP_CASES))
-def test_decode_step(H, name):
+def test_decode_step(H, name, form):
     wl = STEP_CASES[name]
     inp = make_inputs(wl, seed=7)
     codes0, _ = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"])
-    got = run_step(H, wl, inp, codes0)
+    got = run_step(H, wl, inp, codes0, flags=FORMS[form])
     check_step(wl, inp, codes0, got)
     assert H.hata_read_device_status(got["ws"]) == 0
 
 
-def test_decode_step_equals_granular_chain(H):
-    """The fused call and the chain of granular calls agree bit for bit in codes and indices."""
+@pytest.mark.parametrize("form", list(FORMS))
+def test_decode_step_equals_granular_chain(H, form):
+    """Both fused forms and the chain of granular calls agree bit for bit in codes and indices."""
     wl = STEP_CASES["ragged_b3"]
     inp = make_inputs(wl, seed=9)
     codes0, _ = oracle.encode_cache(inp["K"], inp["W_H"], inp["seq_lens"])
-    fused = run_step(H, wl, inp, codes0)
+    fused = run_step(H, wl, inp, codes0, flags=FORMS[form])
     d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype)
     ws = new_workspace(d, wl.k)
     q, K, V = (dev_float(inp[n], wl.dtype) for n in ("q", "K", "V"))
@@ -402,17 +407,21 @@ def test_decode_step_flags_length_beyond_cache(H):
     assert H.hata_read_device_status(got["ws"]) == H.HATA_ERR_INVALID_ARG
 
 
-def test_kernel_count_reports_fused_and_chain(H):
-    # scan kernel + tail kernel, or the chain of six granular launches (G = 3)
-    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 2
+def test_kernel_count_reports_the_form(H):
+    # the cluster form (one launch), the all-SM form (encode, scan and tail kernels),
+    # and the chain of six granular launches (G = 3)
+    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 1
+    assert H.hata_decode_step_kernel_count(H.dims_for(16, 32, 8, 128, 128, 65536, "bf16"), 1024) == 3
+    assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16", 4), 512) == 3
     assert H.hata_decode_step_kernel_count(H.dims_for(1, 6, 2, 128, 128, 3000, "bf16"), 100) == 6
 
 
 def _custom_step(H, wl, seed, codes0):
     inp = make_inputs(wl, seed=seed, plant=False)
-    got = run_step(H, wl, inp, codes0)
-    check_step(wl, inp, codes0, got)
-    assert H.hata_read_device_status(got["ws"]) == 0
+    for flags in FORMS.values():
+        got = run_step(H, wl, inp, codes0, flags=flags)
+        check_step(wl, inp, codes0, got)
+        assert H.hata_read_device_status(got["ws"]) == 0
 
 
 def test_decode_step_heavy_ties(H):
