@@ -353,6 +353,44 @@ def run_reference(args, wl):
 # GPU arm
 # ----------------------------------------------------------------------------
 
+def run_e2e(H, dims, k, steps, layers, stages, in_host, out_host, ws, stream):
+    """The end-to-end loop of hash_aware_top_b200/libhata_e2e.so; returns (device ms, host wall ms).
+
+    in_host: pinned [B*Hq + 2*B*Hkv][d] (q, the new K rows, the new V rows); stages: one
+    device buffer of that shape per layer; out_host: pinned [B][Hq][d], written by the step."""
+    import ctypes
+
+    lib = ctypes.CDLL(os.path.join(os.path.dirname(H.LIB_PATH), "libhata_e2e.so"))
+    P = ctypes.c_void_p
+    R = len(layers)
+
+    def arr(ts):
+        return (P * R)(*[P(t.data_ptr()) for t in ts])
+
+    dms, hms = ctypes.c_float(0), ctypes.c_float(0)
+    fn = lib.hata_e2e_run
+    fn.restype = ctypes.c_int
+    rc = fn(ctypes.byref(dims), int(k), int(steps), R, P(in_host.data_ptr()), P(out_host.data_ptr()), arr(stages),
+            arr([lay["K"] for lay in layers]), arr([lay["V"] for lay in layers]), arr([lay["W"] for lay in layers]),
+            arr([lay["codes"] for lay in layers]), arr([lay["lens"] for lay in layers]), P(ws.data_ptr()),
+            ctypes.c_size_t(ws.numel()), P(stream.cuda_stream), ctypes.byref(dms), ctypes.byref(hms))
+    if rc != 0:
+        raise RuntimeError(f"end-to-end loop failed: status {rc}")
+    return dms.value, hms.value
+
+
+def e2e_inputs(wl, layer, seq_lens):
+    """Pinned host inputs of one end-to-end step -- the layer's queries and the new token's
+    K and V rows (those already at slot L_b - 1, so the step's result is unchanged) -- and a
+    pinned output buffer."""
+    import torch
+
+    rows = lambda C: torch.stack([C[b, :, int(seq_lens[b]) - 1] for b in range(wl.batch)])  # noqa: E731
+    flat = torch.cat([layer["q"].reshape(-1, wl.head_dim), rows(layer["K"]).reshape(-1, wl.head_dim),
+                      rows(layer["V"]).reshape(-1, wl.head_dim)])
+    return flat.cpu().pin_memory(), torch.empty_like(layer["out"], device="cpu").pin_memory()
+
+
 def graph_upload(g, stream):
     """Upload an instantiated graph to the device before it is timed, so that the first
     timed replay does not pay for it (driver call cuGraphUpload on the graph's exec handle)."""
@@ -499,39 +537,20 @@ def run_gpu(args, wl):
         raise RuntimeError(f"device status {status}: {H.hata_status_string(status)}")
     ms_per_step = ms / args.steps
     value = job_throughput(world, args.steps, ms / 1e3)
-    # end to end through the public call: pinned host inputs in, output read back, every step
-    e2e_steps = min(args.steps, 300)
-    L0 = layers[0]
-    q_host = L0["q"].cpu().pin_memory()
-    kv_host = torch.stack([torch.stack([L0["K"][b, :, int(inp["seq_lens"][b]) - 1] for b in range(wl.batch)]),
-                           torch.stack([L0["V"][b, :, int(inp["seq_lens"][b]) - 1] for b in range(wl.batch)])]
-                          ).cpu().pin_memory()
-    out_host = torch.empty_like(L0["out"], device="cpu").pin_memory()
-    h2d = q_host.numel() * q_host.element_size() + kv_host.numel() * kv_host.element_size()
+    # end to end through the public C ABI (a native loop, hash_aware_top_b200/e2e): every step
+    # copies its inputs (q and the new token's K and V rows) from pinned host memory in one
+    # copy, appends the rows to the caches (hata_append_kv), runs hata_decode_step with the
+    # output in pinned host memory, and waits for it
+    e2e_steps = min(args.steps, 2000)
+    in_host, out_host = e2e_inputs(wl, layers[0], inp["seq_lens"])
+    stages = [torch.empty_like(in_host, device=dev) for _ in layers]
+    h2d = in_host.numel() * in_host.element_size()
     d2h = out_host.numel() * out_host.element_size()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    kv_stage = torch.empty(kv_host.shape, dtype=kv_host.dtype, device=dev)
-    # timed on the device: events on the stream around the loop; every step waits for its
-    # result on the host, so the host side of each step lies inside the interval
-    e_e2e0, e_e2e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e_e2e0.record(stream)
-        for i in range(e2e_steps):
-            L = layers[i % R]
-            L["q"].copy_(q_host, non_blocking=True)
-            kv_stage.copy_(kv_host, non_blocking=True)
-            for b in range(wl.batch):
-                pos = int(inp["seq_lens"][b]) - 1
-                L["K"][b, :, pos].copy_(kv_stage[0, b])
-                L["V"][b, :, pos].copy_(kv_stage[1, b])
-            step(i)
-            out_host.copy_(L["out"], non_blocking=True)
-            stream.synchronize()
-        e_e2e1.record(stream)
-        e_e2e1.synchronize()
-    e2e_s = max_over_ranks(e_e2e0.elapsed_time(e_e2e1) / 1e3, dist, dev)
+    e2e_dev_ms, e2e_host_ms = run_e2e(H, dims, wl.k, e2e_steps, layers, stages, in_host, out_host, ws, stream)
+    e2e_s = max_over_ranks(e2e_dev_ms / 1e3, dist, dev)
     e2e_value = job_throughput(world, e2e_steps, e2e_s)
 
     # the dense flash-decode baseline on the same layer buffers (the comparison the pages report)
@@ -682,7 +701,10 @@ def run_gpu(args, wl):
             "algorithmic_bytes_per_step": step_bytes,
         },
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "host_wall_ms": e2e_host_ms,
+                "loop": "native loop over the C ABI, every step: one H2D of q and the new K/V rows, "
+                        "hata_append_kv, hata_decode_step writing its output into mapped pinned host memory "
+                        "(the D2H bytes), stream synchronize"},
         "gpu_launches": args.steps * H.hata_decode_step_kernel_count(dims, wl.k),
         "workloads": workloads,
         "dense_baseline": dense,

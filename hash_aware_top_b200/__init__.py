@@ -26,6 +26,7 @@ __all__ = [
     "dims_for",
     "hata_workspace_size",
     "hata_workspace_init",
+    "hata_append_kv",
     "hata_encode_append",
     "hata_hamming_scores",
     "hata_topk",
@@ -56,6 +57,7 @@ HATA_FLAG_ALL_SM_SCAN = 4  # the all-SM form of the decode step for any shape it
 EXPORTED_SYMBOLS = (
     "hata_workspace_size",
     "hata_workspace_init",
+    "hata_append_kv",
     "hata_encode_append",
     "hata_hamming_scores",
     "hata_topk",
@@ -99,6 +101,11 @@ class Dims(ctypes.Structure):
     def words(self) -> int:
         return self.hash_bits // 32
 
+    def code_shape(self, *lead) -> tuple:
+        """Shape of a code tensor with leading dims `lead`: packed 32-bit words [..., r/32] (int32 or
+        uint32), or for r = 16 one 16-bit code per token [...] (int16 or uint16)."""
+        return tuple(lead) if self.hash_bits == 16 else tuple(lead) + (self.words,)
+
     @property
     def torch_dtype(self):
         return torch.float32 if self.dtype == HATA_F32 else torch.bfloat16
@@ -113,6 +120,7 @@ def _load():
     sig = {
         "hata_workspace_size": (I, [DP, I, ctypes.POINTER(S)]),
         "hata_workspace_init": (I, [P, S, P]),
+        "hata_append_kv": (I, [DP, P, P, P, P, P, P]),
         "hata_encode_append": (I, [DP, P, I, I, I, P, P, P, I, P, S, P]),
         "hata_hamming_scores": (I, [DP, P, P, P, P, P]),
         "hata_topk": (I, [DP, P, P, I, P, P, P, S, P]),
@@ -188,9 +196,12 @@ def _ptr(t, name, shape=None, dtype=None, optional=False, numel=None):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def _codes_dtype(t):
-    if t is not None and t.dtype not in (torch.int32, torch.uint32):
-        raise TypeError("codes must be int32 or uint32 tensors holding the packed words")
+def _codes_dtype(t, dims=None):
+    wide = dims is None or dims.hash_bits != 16
+    ok = (torch.int32, torch.uint32) if wide else (torch.int16, torch.uint16)
+    if t is not None and t.dtype not in ok:
+        raise TypeError("codes must be int32 or uint32 tensors holding the packed words"
+                        if wide else "16-bit codes must be int16 or uint16 tensors, one code per token")
     return t.dtype if t is not None else None
 
 
@@ -203,6 +214,20 @@ def hata_workspace_size(dims: Dims, k: int) -> int:
 def hata_workspace_init(ws: torch.Tensor, stream=None):
     _check(lib.hata_workspace_init(_ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
            "hata_workspace_init")
+
+
+def hata_append_kv(dims: Dims, new_k, new_v, K, V, seq_lens, stream=None):
+    """Write the new token's rows new_k/new_v ([B][Hkv][d]) to slot seq_lens[b] - 1 of K/V."""
+    d = dims
+    row = (d.batch, d.n_kv_heads, d.head_dim)
+    cache = (d.batch, d.n_kv_heads, d.max_seq, d.head_dim)
+    _check(
+        lib.hata_append_kv(
+            ctypes.byref(d),
+            _ptr(new_k, "new_k", row, d.torch_dtype), _ptr(new_v, "new_v", row, d.torch_dtype),
+            _ptr(K, "K", cache, d.torch_dtype), _ptr(V, "V", cache, d.torch_dtype),
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), _stream(stream)),
+        "hata_append_kv")
 
 
 def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len, ws, stream=None):
@@ -218,7 +243,8 @@ def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes
             int(x_heads), int(x_len), int(n_tok),
             _ptr(seq_end, "seq_end", (d.batch,), torch.int32, optional=True),
             _ptr(W_H, "W_H", (d.n_kv_heads, d.head_dim, d.hash_bits), torch.float32),
-            _ptr(codes, "codes", dtype=_codes_dtype(codes), numel=d.batch * x_heads * codes_len * d.words),
+            _ptr(codes, "codes", dtype=_codes_dtype(codes, d),
+                 numel=d.batch * x_heads * codes_len * max(d.words, 1)),
             int(codes_len), _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_encode_append")
 
@@ -228,8 +254,8 @@ def hata_hamming_scores(dims: Dims, qcode, codes, seq_lens, scores, stream=None)
     _check(
         lib.hata_hamming_scores(
             ctypes.byref(d),
-            _ptr(qcode, "qcode", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode)),
-            _ptr(codes, "codes", (d.batch, d.n_kv_heads, d.max_seq, d.words), _codes_dtype(codes)),
+            _ptr(qcode, "qcode", d.code_shape(d.batch, d.n_q_heads), _codes_dtype(qcode, d)),
+            _ptr(codes, "codes", d.code_shape(d.batch, d.n_kv_heads, d.max_seq), _codes_dtype(codes, d)),
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32),
             _ptr(scores, "scores", (d.batch, d.n_kv_heads, d.max_seq), torch.int32),
             _stream(stream)),
@@ -310,10 +336,11 @@ def hata_decode_step(dims: Dims, q, K, V, W_H, codes, seq_lens, k, scale, out, q
             _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
             _ptr(K, "K", kv, d.torch_dtype), _ptr(V, "V", kv, d.torch_dtype),
             _ptr(W_H, "W_H", (d.n_kv_heads, d.head_dim, d.hash_bits), torch.float32),
-            _ptr(codes, "codes", (d.batch, d.n_kv_heads, d.max_seq, d.words), _codes_dtype(codes)),
+            _ptr(codes, "codes", d.code_shape(d.batch, d.n_kv_heads, d.max_seq), _codes_dtype(codes, d)),
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k), float(scale),
             _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
-            _ptr(qcode_out, "qcode_out", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode_out), optional=True),
+            _ptr(qcode_out, "qcode_out", d.code_shape(d.batch, d.n_q_heads), _codes_dtype(qcode_out, d),
+                 optional=True),
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step")
@@ -331,10 +358,11 @@ def hata_decode_step_qk(dims: Dims, q, K, V, W_q, W_k, codes, seq_lens, k, scale
             _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
             _ptr(K, "K", kv, d.torch_dtype), _ptr(V, "V", kv, d.torch_dtype),
             _ptr(W_q, "W_q", wshape, torch.float32), _ptr(W_k, "W_k", wshape, torch.float32),
-            _ptr(codes, "codes", (d.batch, d.n_kv_heads, d.max_seq, d.words), _codes_dtype(codes)),
+            _ptr(codes, "codes", d.code_shape(d.batch, d.n_kv_heads, d.max_seq), _codes_dtype(codes, d)),
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k), float(scale),
             _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
-            _ptr(qcode_out, "qcode_out", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode_out), optional=True),
+            _ptr(qcode_out, "qcode_out", d.code_shape(d.batch, d.n_q_heads), _codes_dtype(qcode_out, d),
+                 optional=True),
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step_qk")
@@ -355,11 +383,12 @@ def hata_decode_step_paged(dims: Dims, q, K_pool, V_pool, W_q, W_k, codes_pool, 
             _ptr(q, "q", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
             _ptr(K_pool, "K_pool", pool, d.torch_dtype), _ptr(V_pool, "V_pool", pool, d.torch_dtype),
             _ptr(W_q, "W_q", wshape, torch.float32), _ptr(W_k, "W_k", wshape, torch.float32),
-            _ptr(codes_pool, "codes_pool", (n_blocks, d.n_kv_heads, bs, d.words), _codes_dtype(codes_pool)),
+            _ptr(codes_pool, "codes_pool", d.code_shape(n_blocks, d.n_kv_heads, bs), _codes_dtype(codes_pool, d)),
             _ptr(block_table, "block_table", (d.batch, max_blocks), torch.int32), bs, n_blocks,
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), int(k), float(scale),
             _ptr(out, "out", (d.batch, d.n_q_heads, d.head_dim), d.torch_dtype),
-            _ptr(qcode_out, "qcode_out", (d.batch, d.n_q_heads, d.words), _codes_dtype(qcode_out), optional=True),
+            _ptr(qcode_out, "qcode_out", d.code_shape(d.batch, d.n_q_heads), _codes_dtype(qcode_out, d),
+                 optional=True),
             _ptr(idx_out, "idx_out", (d.batch, d.n_kv_heads, k), torch.int32, optional=True),
             _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
         "hata_decode_step_paged")

@@ -55,7 +55,7 @@ def _stale(target, deps) -> bool:
 def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     srcs = _sources()
     hdrs = _headers()
-    if not force and not _stale(LIB, srcs + hdrs):
+    if not force and not _stale(LIB, srcs + hdrs) and not _stale(E2E_LIB, [E2E_SRC, LIB]):
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
@@ -84,7 +84,26 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    build_e2e(cc, flags, verbose)
     return LIB
+
+
+E2E_SRC = os.path.join(PKG, "e2e", "hata_e2e.cu")
+E2E_LIB = os.path.join(PKG, "libhata_e2e.so")
+
+
+def build_e2e(cc, flags, verbose=False):
+    """The benchmark's end-to-end loop (native, calling libhata.so's C ABI)."""
+    obj = os.path.join(BUILD, "hata_e2e.o")
+    cmds = [[cc, *ARCH, *flags, "-c", E2E_SRC, "-o", obj],
+            [cc, *ARCH, "-shared", "-o", E2E_LIB + ".tmp", obj, "-L" + PKG, "-lhata", "-Xlinker", "-rpath=$ORIGIN"]]
+    for cmd in cmds:
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"e2e driver build failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(E2E_LIB + ".tmp", E2E_LIB)
 
 
 def main(argv=None):

@@ -85,6 +85,15 @@ hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_h
                                    static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream)));
 }
 
+hata_status_t hata_append_kv(const hata_dims_t* dims, const void* new_k, const void* new_v, void* K, void* V,
+                             const int32_t* seq_lens, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!new_k || !new_v || !K || !V || !seq_lens) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(new_k) || !aligned16(new_v) || !aligned16(K) || !aligned16(V)) return HATA_ERR_INVALID_ARG;
+  return cuda_status(launch_append_kv(*dims, new_k, new_v, K, V, seq_lens, static_cast<cudaStream_t>(stream)));
+}
+
 hata_status_t hata_hamming_scores(const hata_dims_t* dims, const uint32_t* qcode, const uint32_t* codes,
                                   const int32_t* seq_lens, int32_t* scores, void* stream) {
   hata_status_t s = check_dims(dims);

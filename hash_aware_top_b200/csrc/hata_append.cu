@@ -1,0 +1,48 @@
+// KV cache update of a decode step ("HATA" paper notes, Decode 阶段算法: the new
+// token's key and value join the cache before the step scores it): the new rows
+// K_new[b][g][:] and V_new[b][g][:] are written to slot L_b - 1 of their slabs.
+// A plain row copy, one 16-byte vector per thread: both rows of a (b, g) pair are
+// d * sizeof(T) bytes (256 or 512), so every vector is aligned when the bases are.
+#include "hata_kernels.cuh"
+
+namespace hata {
+
+namespace {
+
+constexpr int kAppThreads = 256;
+
+__global__ void __launch_bounds__(kAppThreads)
+    append_kv_kernel(const uint4* __restrict__ new_k, const uint4* __restrict__ new_v, uint4* __restrict__ K,
+                     uint4* __restrict__ V, const int32_t* __restrict__ seq_lens, int hkv, int max_seq,
+                     int vec_per_row, long long n_vec) {
+  const long long e = (long long)blockIdx.x * kAppThreads + threadIdx.x;
+  if (e >= n_vec) return;
+  const long long half = n_vec / 2;  // vectors of all K rows, then of all V rows
+  const bool is_v = e >= half;
+  const long long ev = is_v ? e - half : e;
+  const long long row = ev / vec_per_row;  // (b, g) pair
+  const int c = (int)(ev % vec_per_row);
+  const int b = (int)(row / hkv);
+  const int L = seq_lens[b];
+  if (L < 1 || L > max_seq) return;  // no slot to write
+  const size_t dst = ((size_t)row * max_seq + (L - 1)) * vec_per_row + c;
+  if (is_v) V[dst] = new_v[ev];
+  else K[dst] = new_k[ev];
+}
+
+}  // namespace
+
+cudaError_t launch_append_kv(const hata_dims_t& d, const void* new_k, const void* new_v, void* K, void* V,
+                             const int32_t* seq_lens, cudaStream_t st) {
+  const int esize = d.dtype == HATA_BF16 ? 2 : 4;
+  const int vec_per_row = d.head_dim * esize / 16;
+  const long long n_vec = 2LL * d.batch * d.n_kv_heads * vec_per_row;
+  const long long blocks = (n_vec + kAppThreads - 1) / kAppThreads;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  append_kv_kernel<<<(unsigned)blocks, kAppThreads, 0, st>>>(
+      static_cast<const uint4*>(new_k), static_cast<const uint4*>(new_v), static_cast<uint4*>(K),
+      static_cast<uint4*>(V), seq_lens, d.n_kv_heads, d.max_seq, vec_per_row, n_vec);
+  return cudaGetLastError();
+}
+
+}  // namespace hata

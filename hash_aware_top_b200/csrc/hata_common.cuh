@@ -29,8 +29,9 @@ inline hata_status_t check_dims(const hata_dims_t* d) {
   if (d->flags & ~(HATA_FLAG_EARLY_PREFETCH | HATA_FLAG_TEST_EXPIRE_WAIT | HATA_FLAG_ALL_SM_SCAN))
     return HATA_ERR_INVALID_ARG;
   if (d->head_dim != kHeadDim) return HATA_ERR_UNSUPPORTED;
-  if (d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
+  if (d->hash_bits != 16 && d->hash_bits != 32 && d->hash_bits != 64 && d->hash_bits != 128 && d->hash_bits != 256)
     return HATA_ERR_UNSUPPORTED;
+  if (d->hash_bits == 16 && (d->max_seq & 1)) return HATA_ERR_INVALID_ARG;  // 16-bit codes: whole 32-bit pairs
   const long long G = d->n_q_heads / d->n_kv_heads;
   if (G > 16 || G * d->hash_bits + 1 > kMaxBins) return HATA_ERR_UNSUPPORTED;
   return HATA_OK;
@@ -59,7 +60,7 @@ struct FusedPlan;  // defined in hata_step.cu
 inline WsLayout make_layout(const hata_dims_t& d, int k, size_t fused_bytes) {
   WsLayout L{};
   const size_t B = d.batch, Hq = d.n_q_heads, Hkv = d.n_kv_heads, Lm = d.max_seq;
-  const size_t W = d.hash_bits / 32, G = Hq / Hkv;
+  const size_t CB = (size_t)d.hash_bits / 8, G = Hq / Hkv;  // bytes per code
   L.nchunk = (int)((Lm + kTopkChunk - 1) / kTopkChunk);
   L.nbins = (int)(G * d.hash_bits + 1);
   L.nsplit = (k + kSparseRows - 1) / kSparseRows;
@@ -70,7 +71,7 @@ inline WsLayout make_layout(const hata_dims_t& d, int k, size_t fused_bytes) {
     return o;
   };
   L.status = take(kAlign);
-  L.qcode = take(B * Hq * W * 4);
+  L.qcode = take(B * Hq * CB);
   L.scores = take(B * Hkv * Lm * 4);
   L.idx = take(B * Hkv * (size_t)k * 4);
   L.topk_hist = take(B * Hkv * (size_t)L.nchunk * L.nbins * 4);

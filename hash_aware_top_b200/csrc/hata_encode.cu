@@ -56,16 +56,17 @@ __global__ void __launch_bounds__(kEncThreads)
     }
     xs[rr][i] = v;
   }
+  const int CW = R < 32 ? R : 32;  // columns of this code word (16 for 16-bit codes)
   const float* Wg = W + (size_t)g * D * R + 32 * w;
   for (int e = tid; e < 32 * D; e += kEncThreads) {
     const int i = e / 32, c = e % 32;
-    ws[c][i] = __ldg(Wg + (size_t)i * R + c);
+    ws[c][i] = c < CW ? __ldg(Wg + (size_t)i * R + c) : 0.f;
   }
   if (tid < kDecRows) words[tid] = 0u;
   __syncthreads();
   const int nrows = min(kDecRows, rows_total - row0);
-  for (int pr = warp; pr < nrows * 32; pr += kEncThreads / 32) {
-    const int rr = pr / 32, c = pr % 32;
+  for (int pr = warp; pr < nrows * CW; pr += kEncThreads / 32) {
+    const int rr = pr / CW, c = pr % CW;
     const float y = warp_dot128(xs[rr], ws[c], lane);
     if (lane == 0 && y > 0.f) atomicOr(&words[rr], 1u << c);
   }
@@ -73,7 +74,11 @@ __global__ void __launch_bounds__(kEncThreads)
   if (tid < nrows) {
     const int rho = row0 + tid;
     const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
-    if (t >= 0 && t < lim) codes[(((size_t)bb * x_heads + h) * codes_len + t) * (R / 32) + w] = words[tid];
+    const size_t slot = ((size_t)bb * x_heads + h) * codes_len + t;
+    if (t >= 0 && t < lim) {
+      if (R == 16) reinterpret_cast<uint16_t*>(codes)[slot] = (uint16_t)words[tid];
+      else codes[slot * (R / 32) + w] = words[tid];
+    }
   }
 }
 
@@ -122,9 +127,14 @@ __global__ void __launch_bounds__(kEncThreads)
   for (int q = 0; q < RPT; ++q) {
     const unsigned word = __ballot_sync(0xffffffffu, acc[q] > 0.f);
     const int rho = row0 + s + q * NS;
-    if (lane == 0 && rho < rows_total) {
+    // 16-bit codes: a warp holds two rows' codes, lanes 0 and 16 each write one half
+    if ((R == 16 ? (lane & 15) : lane) == 0 && rho < rows_total) {
       const int h = g * hpg + rho / n_tok, t = t_lo + rho % n_tok;
-      if (t >= 0 && t < lim) codes[(((size_t)b * x_heads + h) * codes_len + t) * NW + j / 32] = word;
+      const size_t slot = ((size_t)b * x_heads + h) * codes_len + t;
+      if (t >= 0 && t < lim) {
+        if constexpr (R == 16) reinterpret_cast<uint16_t*>(codes)[slot] = (uint16_t)(word >> (lane & 16));
+        else codes[slot * NW + j / 32] = word;
+      }
     }
   }
 }
@@ -135,7 +145,7 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
   const int hpg = x_heads / d.n_kv_heads;
   if (n_tok <= kDecodeTok) {
     const int nbz = (hpg * n_tok + kDecRows - 1) / kDecRows;
-    dim3 grid(d.hash_bits / 32, d.n_kv_heads, d.batch * nbz);
+    dim3 grid((d.hash_bits + 31) / 32, d.n_kv_heads, d.batch * nbz);
     encode_decode_kernel<T><<<grid, kEncThreads, 0, st>>>(static_cast<const T*>(x), x_heads, x_len, n_tok, seq_end,
                                                           W, codes, codes_len, hpg, d.hash_bits);
     return cudaGetLastError();
@@ -149,6 +159,7 @@ cudaError_t launch_t(const hata_dims_t& d, const void* x, int x_heads, int x_len
   dim3 grid((unsigned)((rows + kEncRows - 1) / kEncRows), d.n_kv_heads, d.batch);
   const T* xp = static_cast<const T*>(x);
   switch (d.hash_bits) {
+    case 16: encode_kernel<T, 16><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
     case 32: encode_kernel<T, 32><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
     case 64: encode_kernel<T, 64><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;
     case 128: encode_kernel<T, 128><<<grid, kEncThreads, 0, st>>>(xp, x_heads, x_len, n_tok, seq_end, W, codes, codes_len, hpg); break;

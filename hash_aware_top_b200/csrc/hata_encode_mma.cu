@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kEmThreads, 2)
 cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
                               const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
                               cudaStream_t st) {
-  if (d.dtype != HATA_BF16 || d.hash_bits > 128) return cudaErrorNotSupported;
+  if (d.dtype != HATA_BF16 || d.hash_bits > 128 || d.hash_bits < 32) return cudaErrorNotSupported;
   static int sms = 0;
   if (!sms) {
     int dev = 0;

@@ -382,7 +382,7 @@ cudaError_t tc_device_setup(int* sms_out) {
 cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, int x_len, int n_tok,
                              const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
                              uint32_t* status, cudaStream_t st) {
-  if (d.dtype != HATA_BF16 || d.hash_bits > 128) return cudaErrorNotSupported;
+  if (d.dtype != HATA_BF16 || d.hash_bits > 128 || d.hash_bits < 32) return cudaErrorNotSupported;
   int sms = 0;
   if (tc_device_setup(&sms) != cudaSuccess) return cudaErrorNotSupported;
   const int hpg = x_heads / d.n_kv_heads;

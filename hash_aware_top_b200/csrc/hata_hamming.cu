@@ -16,7 +16,8 @@ namespace {
 constexpr int kHamThreads = 256;
 constexpr int kHamTPT = 8;  // tokens per thread
 
-template <int NW, int G>
+// H16: 16-bit codes, one uint16 per token (the word holds it zero-extended, NW = 1)
+template <int NW, int G, bool H16>
 __global__ void __launch_bounds__(kHamThreads)
     hamming_kernel(const uint32_t* __restrict__ qcode, const uint32_t* __restrict__ codes,
                    const int32_t* __restrict__ seq_lens, int32_t* __restrict__ scores, int max_seq, int hkv,
@@ -27,20 +28,25 @@ __global__ void __launch_bounds__(kHamThreads)
   const int t0 = blockIdx.x * kHamThreads * kHamTPT;
   if (t0 >= L) return;
   const int Gn = G ? G : g_rt;
-  const uint32_t* qg = qcode + ((size_t)b * hkv * Gn + (size_t)g * Gn) * NW;
-  for (int e = threadIdx.x; e < Gn * NW; e += kHamThreads) qs[e] = qg[e];
+  const size_t q0 = ((size_t)b * hkv * Gn + (size_t)g * Gn) * NW;
+  for (int e = threadIdx.x; e < Gn * NW; e += kHamThreads)
+    qs[e] = H16 ? (uint32_t)reinterpret_cast<const uint16_t*>(qcode)[q0 + e] : qcode[q0 + e];
   __syncthreads();
   GroupQuery<NW, G> gq;
   gq.init(qs);
 
   const size_t slab = (size_t)b * hkv + g;
   const uint32_t* cb = codes + slab * max_seq * NW;
+  const uint16_t* cb16 = reinterpret_cast<const uint16_t*>(codes) + slab * max_seq;
   int32_t* out = scores + slab * max_seq;
   uint32_t kw[kHamTPT][NW];
 #pragma unroll
   for (int u = 0; u < kHamTPT; ++u) {
     const int t = t0 + u * kHamThreads + threadIdx.x;
-    if (t < L) load_code<NW>(cb + (size_t)t * NW, kw[u]);
+    if (t < L) {
+      if constexpr (H16) kw[u][0] = (uint32_t)__ldg(cb16 + t);
+      else load_code<NW>(cb + (size_t)t * NW, kw[u]);
+    }
   }
 #pragma unroll
   for (int u = 0; u < kHamTPT; ++u) {
@@ -49,18 +55,18 @@ __global__ void __launch_bounds__(kHamThreads)
   }
 }
 
-template <int NW>
+template <int NW, bool H16 = false>
 cudaError_t launch_nw(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes, const int32_t* seq_lens,
                       int32_t* scores, cudaStream_t st) {
   const int G = d.n_q_heads / d.n_kv_heads;
   dim3 grid((d.max_seq + kHamThreads * kHamTPT - 1) / (kHamThreads * kHamTPT), d.n_kv_heads, d.batch);
   const size_t smem = (size_t)G * NW * 4;
   switch (G) {
-    case 1: hamming_kernel<NW, 1><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
-    case 2: hamming_kernel<NW, 2><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
-    case 4: hamming_kernel<NW, 4><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
-    case 8: hamming_kernel<NW, 8><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
-    default: hamming_kernel<NW, 0><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
+    case 1: hamming_kernel<NW, 1, H16><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
+    case 2: hamming_kernel<NW, 2, H16><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
+    case 4: hamming_kernel<NW, 4, H16><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
+    case 8: hamming_kernel<NW, 8, H16><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
+    default: hamming_kernel<NW, 0, H16><<<grid, kHamThreads, smem, st>>>(qcode, codes, seq_lens, scores, d.max_seq, d.n_kv_heads, G); break;
   }
   return cudaGetLastError();
 }
@@ -70,6 +76,7 @@ cudaError_t launch_nw(const hata_dims_t& d, const uint32_t* qcode, const uint32_
 cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,
                            const int32_t* seq_lens, int32_t* scores, cudaStream_t stream) {
   switch (d.hash_bits) {
+    case 16: return launch_nw<1, true>(d, qcode, codes, seq_lens, scores, stream);
     case 32: return launch_nw<1>(d, qcode, codes, seq_lens, scores, stream);
     case 64: return launch_nw<2>(d, qcode, codes, seq_lens, scores, stream);
     case 128: return launch_nw<4>(d, qcode, codes, seq_lens, scores, stream);

@@ -11,6 +11,8 @@ cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int 
                           const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len, uint32_t* status,
                           cudaStream_t stream);
 
+cudaError_t launch_append_kv(const hata_dims_t& d, const void* new_k, const void* new_v, void* K, void* V,
+                             const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,
                            const int32_t* seq_lens, int32_t* scores, cudaStream_t stream);
 

@@ -72,7 +72,8 @@ class Workload:
 
     @property
     def words(self) -> int:
-        return self.hash_bits // 32
+        """32-bit words per code in the oracle's packing (a 16-bit code fills the low half of one)."""
+        return (self.hash_bits + 31) // 32
 
     @property
     def elem_bytes(self) -> int:
@@ -171,9 +172,11 @@ def make_inputs(wl: Workload, seed: int = 0, plant: bool = True) -> dict:
 
 
 def random_codes(shape, hash_bits: int, seed: int = 0) -> np.ndarray:
-    """Uniformly random packed codes: uint32 array of shape (*shape, hash_bits // 32)."""
+    """Uniformly random packed codes: uint32 array of shape (*shape, ceil(hash_bits / 32)); a 16-bit code
+    occupies the low half of its one word."""
     rng = _streams(seed)[S_CODES]
-    return rng.integers(0, 2**32, size=tuple(shape) + (hash_bits // 32,), dtype=np.uint64).astype(np.uint32)
+    top = 2 ** min(hash_bits, 32)
+    return rng.integers(0, top, size=tuple(shape) + ((hash_bits + 31) // 32,), dtype=np.uint64).astype(np.uint32)
 
 
 def random_scores(shape, max_value: int, seed: int = 0, n_distinct: Optional[int] = None) -> np.ndarray:

@@ -46,8 +46,9 @@
  *       q, out      [B][Hq][d]            (dtype)
  *       K, V        [B][Hkv][max_seq][d]  (dtype), one contiguous row per token
  *       W_H         [Hkv][d][r]           fp32, used as x . W_H
- *       codes       [B][Hkv][max_seq][r/32] uint32 (the hash-code cache)
- *       qcode       [B][Hq][r/32]         uint32
+ *       codes       [B][Hkv][max_seq][r/32] uint32 (the hash-code cache);
+ *                   for r = 16, [B][Hkv][max_seq] uint16, one code per token
+ *       qcode       [B][Hq][r/32]         uint32 ([B][Hq] uint16 for r = 16)
  *       seq_lens    [B]                   int32, cached length incl. the new token
  *       scores      [B][Hkv][max_seq]     int32
  *       idx         [B][Hkv][k]           int32, ascending, -1 padded
@@ -87,7 +88,7 @@ typedef struct {
   int n_q_heads;  /* Hq >= 1, a multiple of n_kv_heads */
   int n_kv_heads; /* Hkv >= 1 */
   int head_dim;   /* d; this version supports 128 */
-  int hash_bits;  /* r in {32, 64, 128, 256} */
+  int hash_bits;  /* r in {16, 32, 64, 128, 256}; 16 needs an even max_seq */
   int max_seq;    /* token capacity of each (b, kv head) cache slab, >= 1 */
   int dtype;      /* hata_dtype_t of q, K, V and out */
   int flags;      /* HATA_FLAG_* bits, 0 for none */
@@ -130,6 +131,21 @@ HATA_API hata_status_t hata_workspace_size(const hata_dims_t* dims, int k, size_
  * the workspace's counters back at zero, so this is needed once, and again
  * only after a call reported HATA_ERR_TIMEOUT. */
 HATA_API hata_status_t hata_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * KV cache update of a decode step (Decode 阶段算法: the new token's key and
+ * value enter the cache before it is scored): for every batch b with
+ * 1 <= L_b = seq_lens[b] <= max_seq and every KV head g,
+ *     K[b][g][L_b - 1][:] = new_k[b][g][:]     V[b][g][L_b - 1][:] = new_v[b][g][:]
+ * Batches with L_b outside [1, max_seq] are left unchanged.  hata_decode_step
+ * then encodes K[b][g][L_b - 1] and appends its code.
+ *   new_k, new_v  device [B][Hkv][d], dims->dtype, 16-byte aligned
+ *   K, V          device [B][Hkv][max_seq][d], dims->dtype, 16-byte aligned
+ *   seq_lens      device [B] int32
+ * No workspace.  Enqueued on `stream`; the caller owns every buffer.
+ */
+HATA_API hata_status_t hata_append_kv(const hata_dims_t* dims, const void* new_k, const void* new_v, void* K, void* V,
+                             const int32_t* seq_lens, void* stream);
 
 /*
  * HashEncode + cache update (Decode 阶段算法, first two steps; 硬件高效优化,

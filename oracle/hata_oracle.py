@@ -54,6 +54,7 @@ __all__ = [
     "sparse_attention",
     "decode_step",
     "encode_cache",
+    "append_kv",
 ]
 
 
@@ -117,6 +118,23 @@ def encode_cache(K: np.ndarray, W_H: np.ndarray, seq_lens: np.ndarray, upto_last
             codes[b, g, :n] = c
             ys[(b, g)] = y
     return codes, ys
+
+
+def append_kv(K: np.ndarray, V: np.ndarray, new_k: np.ndarray, new_v: np.ndarray, seq_lens: np.ndarray):
+    """KV cache update of a decode step (§Decode 阶段算法: the new token's key and value join the cache).
+
+    K, V: [B][Hkv][Lmax][d]; new_k, new_v: [B][Hkv][d].  Returns copies of K and V
+    with slot L_b - 1 of every slab of batch b replaced by the new rows, for
+    1 <= L_b <= Lmax; other batches are returned unchanged (no slot to write).
+    """
+    K2, V2 = K.copy(), V.copy()
+    Lmax = K.shape[2]
+    for b in range(K.shape[0]):
+        L = int(seq_lens[b])
+        if 1 <= L <= Lmax:
+            K2[b, :, L - 1] = new_k[b]
+            V2[b, :, L - 1] = new_v[b]
+    return K2, V2
 
 
 # ----------------------------------------------------------------------------

@@ -25,12 +25,21 @@ def dev_float(a: np.ndarray, dtype: str) -> torch.Tensor:
     return t.to(torch.bfloat16) if dtype == "bf16" else t
 
 
-def dev_codes(a: np.ndarray) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint32).view(np.int32)).cuda()
+def dev_codes(a: np.ndarray, r: int = 32) -> torch.Tensor:
+    """Oracle-packed codes (uint32 words, [..., r/32]) as the library's code tensor: int32 words, or for
+    r = 16 one int16 code per token (the word dimension dropped)."""
+    a = np.ascontiguousarray(a, dtype=np.uint32)
+    if r == 16:
+        return torch.from_numpy(np.ascontiguousarray(a[..., 0].astype(np.uint16).view(np.int16))).cuda()
+    return torch.from_numpy(a.view(np.int32)).cuda()
 
 
 def host_codes(t: torch.Tensor) -> np.ndarray:
-    return t.cpu().numpy().view(np.uint32)
+    """The library's code tensor in the oracle's packing (uint32 words; a 16-bit code in the low half)."""
+    a = t.cpu().numpy()
+    if a.dtype == np.int16:
+        return a.view(np.uint16).astype(np.uint32)[..., None]
+    return a.view(np.uint32)
 
 
 def new_workspace(dims, k) -> torch.Tensor:
@@ -67,9 +76,10 @@ def run_step(H, wl, inp, codes0, ws=None, with_debug=True, flags=0):
     """One hata_decode_step through the C ABI on the workload's inputs, with the cache holding codes0."""
     d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype, flags)
     ws = ws if ws is not None else new_workspace(d, wl.k)
-    codes = dev_codes(codes0)
+    codes = dev_codes(codes0, wl.hash_bits)
     out = torch.full((wl.batch, wl.n_q_heads, 128), float("nan"), dtype=d.torch_dtype, device="cuda")
-    qcode = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda") if with_debug else None
+    cdt = torch.int16 if wl.hash_bits == 16 else torch.int32
+    qcode = torch.zeros(d.code_shape(wl.batch, wl.n_q_heads), dtype=cdt, device="cuda") if with_debug else None
     idx = torch.full((wl.batch, wl.n_kv_heads, wl.k), -99, dtype=torch.int32, device="cuda") if with_debug else None
     H.hata_decode_step(d, dev_float(inp["q"], wl.dtype), dev_float(inp["K"], wl.dtype), dev_float(inp["V"], wl.dtype),
                        torch.from_numpy(inp["W_H"]).cuda(), codes, torch.from_numpy(inp["seq_lens"]).cuda(), wl.k,

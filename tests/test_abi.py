@@ -83,6 +83,10 @@ def test_calls_reject_bad_arguments_before_launch(H):
     assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, P(0x1008), 16, null) == 5
     assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, fake, 8, null) == 5
     assert lib.hata_hamming_scores(ctypes.byref(d), fake, fake, null, fake, null) == 1
+    # the cache update: every pointer required, all 16-byte aligned
+    assert lib.hata_append_kv(ctypes.byref(d), fake, fake, fake, fake, null, null) == 1
+    assert lib.hata_append_kv(ctypes.byref(d), null, fake, fake, fake, fake, null) == 1
+    assert lib.hata_append_kv(ctypes.byref(d), fake, fake, P(0x1008), fake, fake, null) == 1
     # k < 1
     assert lib.hata_topk(ctypes.byref(d), fake, fake, 0, fake, null, fake, 1 << 20, null) == 1
     # workspace too small / missing

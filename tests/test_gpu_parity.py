@@ -135,6 +135,28 @@ def test_encode_append_single_slot(H):
             assert np.array_equal(got[b, g][mask], codes0[b, g][mask])
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_append_kv(H, dtype):
+    """The cache update writes the new rows at slot L_b - 1, bit for bit, and nothing else;
+    lengths 0 and max_seq + 1 write nothing, lengths 1 and max_seq write the first and last slots."""
+    B, Hkv, Lmax = 6, 3, 257
+    rng = np.random.default_rng(17)
+    K0 = rng.standard_normal((B, Hkv, Lmax, 128)).astype(np.float32)
+    V0 = rng.standard_normal((B, Hkv, Lmax, 128)).astype(np.float32)
+    nk = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    nv = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    lens = np.array([1, Lmax, 0, Lmax + 1, 100, 2], dtype=np.int32)
+    d = _dims(H, B, 2 * Hkv, Hkv, 128, Lmax, dtype)
+    K, V = dev_float(K0, dtype), dev_float(V0, dtype)
+    nkd, nvd = dev_float(nk, dtype), dev_float(nv, dtype)
+    H.hata_append_kv(d, nkd, nvd, K, V, torch.from_numpy(lens).cuda())
+    # the expected caches, built by the oracle from the same (device-rounded) values
+    K2, V2 = oracle.append_kv(dev_float(K0, dtype).float().cpu().numpy(), dev_float(V0, dtype).float().cpu().numpy(),
+                              nkd.float().cpu().numpy(), nvd.float().cpu().numpy(), lens)
+    assert np.array_equal(K.float().cpu().numpy(), K2)
+    assert np.array_equal(V.float().cpu().numpy(), V2)
+
+
 # ----------------------------------------------------------------------------
 # Hamming + GQA sum
 # ----------------------------------------------------------------------------
@@ -361,9 +383,10 @@ def test_decode_step_without_debug_outputs_and_repeat(H):
 def run_step_qk(H, wl, inp, W_k, codes0, ws=None):
     d = H.dims_for(wl.batch, wl.n_q_heads, wl.n_kv_heads, 128, wl.hash_bits, wl.max_seq, wl.dtype)
     ws = ws if ws is not None else new_workspace(d, wl.k)
-    codes = dev_codes(codes0)
+    codes = dev_codes(codes0, wl.hash_bits)
     out = torch.full((wl.batch, wl.n_q_heads, 128), float("nan"), dtype=d.torch_dtype, device="cuda")
-    qcode = torch.zeros((wl.batch, wl.n_q_heads, wl.words), dtype=torch.int32, device="cuda")
+    qcode = torch.zeros(d.code_shape(wl.batch, wl.n_q_heads), dtype=torch.int16 if wl.hash_bits == 16 else torch.int32,
+                        device="cuda")
     idx = torch.full((wl.batch, wl.n_kv_heads, wl.k), -99, dtype=torch.int32, device="cuda")
     H.hata_decode_step_qk(d, dev_float(inp["q"], wl.dtype), dev_float(inp["K"], wl.dtype),
                           dev_float(inp["V"], wl.dtype), torch.from_numpy(inp["W_H"]).cuda(),

@@ -175,7 +175,7 @@ def test_simhash_expected_distance(theta):
 # Hamming and the GQA sum
 # ----------------------------------------------------------------------------
 
-@pytest.mark.parametrize("r", [32, 64, 128, 256])
+@pytest.mark.parametrize("r", [16, 32, 64, 128, 256])
 def test_hamming_against_integer_popcount(r):
     a = random_codes((300,), r, seed=1)
     b = random_codes((300,), r, seed=2)
@@ -184,7 +184,7 @@ def test_hamming_against_integer_popcount(r):
     assert got.tolist() == want
 
 
-@pytest.mark.parametrize("r", [32, 128])
+@pytest.mark.parametrize("r", [16, 32, 128])
 def test_hamming_metric_properties(r):
     a = random_codes((64,), r, seed=3)
     b = random_codes((64,), r, seed=4)
@@ -193,6 +193,16 @@ def test_hamming_metric_properties(r):
     assert np.all(oracle.hamming(a, ~a, r) == r)
     assert np.array_equal(oracle.hamming(a, b, r), oracle.hamming(b, a, r))
     assert np.all(oracle.hamming(a, c, r) <= oracle.hamming(a, b, r) + oracle.hamming(b, c, r))
+
+
+def test_sixteen_bit_code_packing():
+    """A 16-bit code is bits 0..15 of one word, bit j at position j (hand-worked): the sign
+    pattern + - + + - - - + (then all -) packs to 0b10001101 = 141; all positive gives 0xFFFF."""
+    y = -np.ones(16)
+    y[[0, 2, 3, 7]] = 1.0
+    assert oracle.pack_bits(oracle.sign_bits(y)).tolist() == [141]
+    assert oracle.pack_bits(oracle.sign_bits(np.ones(16))).tolist() == [0xFFFF]
+    assert oracle.unpack_bits(np.array([141], dtype=np.uint32), 16).nonzero()[0].tolist() == [0, 2, 3, 7]
 
 
 def test_hamming_bit_by_bit_brute_force_tiny():
@@ -205,7 +215,7 @@ def test_hamming_bit_by_bit_brute_force_tiny():
         assert got[i] == want
 
 
-@pytest.mark.parametrize("G,r", [(1, 32), (4, 128), (8, 64), (3, 256)])
+@pytest.mark.parametrize("G,r", [(1, 32), (4, 128), (8, 64), (3, 256), (4, 16)])
 def test_gqa_sum_is_sum_of_heads(G, r):
     q = random_codes((G,), r, seed=8)
     k = random_codes((200,), r, seed=9)
@@ -374,3 +384,23 @@ def test_bf16_rounding_of_inputs():
     x = np.random.default_rng(0).standard_normal(10000).astype(np.float32) * 100
     want = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
     assert np.array_equal(round_to_bf16(x), want)
+
+
+def test_append_kv_writes_only_the_new_slot():
+    """The cache update puts the new rows at slot L_b - 1 (the position of the new
+    token in a cache of L_b tokens) and nowhere else; L_b outside [1, Lmax] writes nothing."""
+    rng = np.random.default_rng(5)
+    B, Hkv, Lmax, d = 4, 2, 6, 3
+    K = rng.standard_normal((B, Hkv, Lmax, d))
+    V = rng.standard_normal((B, Hkv, Lmax, d))
+    nk = rng.standard_normal((B, Hkv, d))
+    nv = rng.standard_normal((B, Hkv, d))
+    lens = np.array([1, 6, 0, 7])
+    K2, V2 = oracle.append_kv(K, V, nk, nv, lens)
+    for b in range(B):
+        for g in range(Hkv):
+            for t in range(Lmax):
+                hit = 1 <= lens[b] <= Lmax and t == lens[b] - 1
+                assert np.array_equal(K2[b, g, t], nk[b, g] if hit else K[b, g, t])
+                assert np.array_equal(V2[b, g, t], nv[b, g] if hit else V[b, g, t])
+    assert np.array_equal(K2[0, :, 0], nk[0]) and np.array_equal(V2[1, :, 5], nv[1])
