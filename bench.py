@@ -391,6 +391,82 @@ def e2e_inputs(wl, layer, seq_lens):
     return flat.cpu().pin_memory(), torch.empty_like(layer["out"], device="cpu").pin_memory()
 
 
+PREFILL_WORKLOAD = "narrow32_b4_64k"
+
+
+def tensor_peak_bf16_sustained():
+    """Measured dense bf16 tensor throughput held for seconds under the power cap (TFLOP/s), or None."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+def bench_prefill_attention(H, dev, local, seed, stream, reps=3):
+    """Causal prefill attention over the narrow-code workload's prompts (4 x 65,536 tokens,
+    32 query / 8 KV heads, r = 32): attention alone, attention with the key encode fused
+    (hata_prefill_attention with codes), and the standalone prefill encode of the same keys
+    (hata_encode_append), timed interleaved with CUDA events on the launching stream.  The
+    attention launches last about 0.3 s, so they run at the clocks the power cap allows; the
+    roofline is the sustained measured bf16 peak."""
+    import torch
+
+    wl = WORKLOADS[PREFILL_WORKLOAD]
+    B, Hq, Hkv, L, r = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.max_seq, wl.hash_bits
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 17)
+    Q = torch.randn((B, Hq, L, wl.head_dim), device=dev, generator=g).to(torch.bfloat16)
+    K = torch.randn((B, Hkv, L, wl.head_dim), device=dev, generator=g).to(torch.bfloat16)
+    V = torch.randn((B, Hkv, L, wl.head_dim), device=dev, generator=g).to(torch.bfloat16)
+    W = (torch.randn((Hkv, wl.head_dim, r), device=dev, generator=g) / (wl.head_dim ** 0.5)).float()
+    lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+    out = torch.empty_like(Q)
+    codes = torch.zeros((B, Hkv, L, wl.words), dtype=torch.int32, device=dev)
+    d = H.dims_for(B, Hq, Hkv, wl.head_dim, r, L, "bf16")
+    ws = torch.zeros(H.hata_prefill_workspace_size(d), dtype=torch.uint8, device=dev)
+    ews = torch.zeros(H.hata_workspace_size(d, wl.k), dtype=torch.uint8, device=dev)
+    calls = {
+        "attention": lambda: H.hata_prefill_attention(d, Q, K, V, None, None, lens, 0.0, out, ws, stream),
+        "fused": lambda: H.hata_prefill_attention(d, Q, K, V, W, codes, lens, 0.0, out, ws, stream),
+        "encode": lambda: H.hata_encode_append(d, K, Hkv, L, L, lens, W, codes, L, ews, stream),
+    }
+    times = {n: [] for n in calls}
+    with torch.cuda.stream(stream):
+        for fn in calls.values():
+            fn()
+        torch.cuda.synchronize()
+        with ClockSampler(local) as clk:
+            for _ in range(reps):
+                for name, fn in calls.items():
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    e1.synchronize()
+                    times[name].append(e0.elapsed_time(e1))
+    for w_ in (ws, ews):
+        if H.hata_read_device_status(w_) != 0:
+            raise RuntimeError("device status set by the prefill attention or encode")
+    ms = {n: statistics.median(v) for n, v in times.items()}
+    flops = 4.0 * wl.head_dim * Hq * B * L * (L + 1) / 2  # q.K and P.V over the causal triangle
+    tflops = flops / (ms["attention"] * 1e-3) / 1e12
+    res = {"workload": f"{PREFILL_WORKLOAD}: {B} x {L}-token prompts, {Hq}/{Hkv} heads, d {wl.head_dim}, r {r}, bf16",
+           "kernel": "hata_prefill_attention (tcgen05 causal attention; key encode fused on the diagonal tile)",
+           "reps": reps, "attention_ms": ms["attention"], "fused_ms": ms["fused"],
+           "fused_encode_overhead_ms": ms["fused"] - ms["attention"],
+           "standalone_encode_ms": ms["encode"], "flops": flops, "tflops": tflops,
+           "clocks": clk.summary()}
+    tpeak = tensor_peak_bf16_sustained()
+    if tpeak:
+        res["peak_tflops"] = tpeak
+        res["peak_kind"] = "measured sustained"
+        res["frac_of_tensor_peak"] = tflops / tpeak
+    del Q, K, V, out, codes
+    torch.cuda.empty_cache()
+    return res
+
+
 def graph_upload(g, stream):
     """Upload an instantiated graph to the device before it is timed, so that the first
     timed replay does not pay for it (driver call cuGraphUpload on the graph's exec handle)."""
@@ -674,6 +750,10 @@ def run_gpu(args, wl):
         del ls2
         torch.cuda.empty_cache()
 
+    prefill_attn = None
+    if not args.no_prefill_attention:
+        prefill_attn = bench_prefill_attention(H, dev, local, args.seed, stream)
+
     line = {
         "metric": METRIC,
         "value": value,
@@ -710,6 +790,7 @@ def run_gpu(args, wl):
         "dense_baseline": dense,
         "paged_step": paged,
         "prefill_encode": prefill,
+        "prefill_attention": prefill_attn,
         "clocks": sampler.summary(),
     }
     if cpu is not None:
@@ -732,6 +813,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=None, help="layer buffers to rotate over (default: > 4x L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill-attention", action="store_true",
+                    help="skip the prefill attention timing (about 3 s of GPU time)")
     ap.add_argument("--also", nargs="*", default=None,
                     help="other workloads timed in the same run (default: llama8b_32k beside the 128K headline)")
     args = ap.parse_args(argv)

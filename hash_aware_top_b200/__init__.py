@@ -27,6 +27,8 @@ __all__ = [
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_append_kv",
+    "hata_prefill_workspace_size",
+    "hata_prefill_attention",
     "hata_encode_append",
     "hata_hamming_scores",
     "hata_topk",
@@ -58,6 +60,8 @@ EXPORTED_SYMBOLS = (
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_append_kv",
+    "hata_prefill_workspace_size",
+    "hata_prefill_attention",
     "hata_encode_append",
     "hata_hamming_scores",
     "hata_topk",
@@ -121,6 +125,8 @@ def _load():
         "hata_workspace_size": (I, [DP, I, ctypes.POINTER(S)]),
         "hata_workspace_init": (I, [P, S, P]),
         "hata_append_kv": (I, [DP, P, P, P, P, P, P]),
+        "hata_prefill_workspace_size": (I, [DP, ctypes.POINTER(S)]),
+        "hata_prefill_attention": (I, [DP, P, P, P, P, P, P, F, P, P, S, P]),
         "hata_encode_append": (I, [DP, P, I, I, I, P, P, P, I, P, S, P]),
         "hata_hamming_scores": (I, [DP, P, P, P, P, P]),
         "hata_topk": (I, [DP, P, P, I, P, P, P, S, P]),
@@ -228,6 +234,30 @@ def hata_append_kv(dims: Dims, new_k, new_v, K, V, seq_lens, stream=None):
             _ptr(K, "K", cache, d.torch_dtype), _ptr(V, "V", cache, d.torch_dtype),
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), _stream(stream)),
         "hata_append_kv")
+
+
+def hata_prefill_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib.hata_prefill_workspace_size(ctypes.byref(dims), ctypes.byref(n)), "hata_prefill_workspace_size")
+    return n.value
+
+
+def hata_prefill_attention(dims: Dims, q, K, V, W_H, codes, seq_lens, scale, out, ws, stream=None):
+    """Causal prefill attention (q/out [B][Hq][max_seq][d], K/V [B][Hkv][max_seq][d], bf16); when codes is
+    given (W_H [Hkv][d][r]), every key's code is written as by hata_encode_append."""
+    d = dims
+    qs = (d.batch, d.n_q_heads, d.max_seq, d.head_dim)
+    ks = (d.batch, d.n_kv_heads, d.max_seq, d.head_dim)
+    _check(
+        lib.hata_prefill_attention(
+            ctypes.byref(d), _ptr(q, "q", qs, d.torch_dtype), _ptr(K, "K", ks, d.torch_dtype),
+            _ptr(V, "V", ks, d.torch_dtype),
+            _ptr(W_H, "W_H", (d.n_kv_heads, d.head_dim, d.hash_bits), torch.float32, optional=codes is None),
+            _ptr(codes, "codes", d.code_shape(d.batch, d.n_kv_heads, d.max_seq), _codes_dtype(codes, d),
+                 optional=True),
+            _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), float(scale), _ptr(out, "out", qs, d.torch_dtype),
+            _ptr(ws, "workspace", dtype=torch.uint8), ws.numel(), _stream(stream)),
+        "hata_prefill_attention")
 
 
 def hata_encode_append(dims: Dims, x, x_heads, x_len, n_tok, seq_end, W_H, codes, codes_len, ws, stream=None):

@@ -85,6 +85,34 @@ hata_status_t hata_encode_append(const hata_dims_t* dims, const void* x, int x_h
                                    static_cast<uint32_t*>(workspace), static_cast<cudaStream_t>(stream)));
 }
 
+hata_status_t hata_prefill_workspace_size(const hata_dims_t* dims, size_t* bytes) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!bytes) return HATA_ERR_INVALID_ARG;
+  *bytes = prefill_ws_bytes(*dims);
+  return HATA_OK;
+}
+
+hata_status_t hata_prefill_attention(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                     const float* W_H, void* codes, const int32_t* seq_lens, float scale, void* out,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  const hata_dims_t& d = *dims;
+  if (d.dtype != HATA_BF16) return HATA_ERR_UNSUPPORTED;
+  if (codes && d.hash_bits > 128) return HATA_ERR_UNSUPPORTED;
+  if (!q || !K || !V || !seq_lens || !out || (codes && !W_H)) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (codes && !aligned16(codes)))
+    return HATA_ERR_INVALID_ARG;
+  if (!(scale >= 0.f) || scale == INFINITY) return HATA_ERR_INVALID_ARG;
+  if ((long long)d.batch * d.n_q_heads * d.max_seq + 128 > 0x7fffffffLL) return HATA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < prefill_ws_bytes(d)) return HATA_ERR_WORKSPACE;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf((float)d.head_dim);
+  cudaError_t e = launch_prefill(d, q, K, V, W_H, codes, seq_lens, sc, out, static_cast<char*>(workspace),
+                                 static_cast<cudaStream_t>(stream));
+  return e == cudaErrorNotSupported ? HATA_ERR_UNSUPPORTED : cuda_status(e);
+}
+
 hata_status_t hata_append_kv(const hata_dims_t* dims, const void* new_k, const void* new_v, void* K, void* V,
                              const int32_t* seq_lens, void* stream) {
   hata_status_t s = check_dims(dims);

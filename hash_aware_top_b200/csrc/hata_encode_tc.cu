@@ -36,14 +36,12 @@
 // caller's status word (the workspace passed to hata_encode_append), stops
 // issuing work, waits (bounded) for the MMAs it issued, frees its TMEM and
 // returns.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 #include <map>
 #include <mutex>
 
 #include "hata_kernels.cuh"
+#include "hata_tc.cuh"
 
 namespace hata {
 
@@ -68,32 +66,6 @@ __device__ __forceinline__ uint32_t cm_off(int row, int k) {
   return (uint32_t)((((row >> 3) * (kHeadDim / 8) + (k >> 3)) << 7) + ((row & 7) << 4));
 }
 
-// shared-memory matrix descriptor: K-major, no swizzle, leading byte offset 128
-// (next core matrix along K), stride byte offset 2048 (next 8-row group),
-// descriptor version 1 (bits 46-47), base offset 0
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
-  const uint32_t lo = ((saddr >> 4) & 0x3fffu) | ((128u >> 4) << 16);
-  const uint32_t hi = ((2048u >> 4) & 0x3fffu) | (1u << 14);
-  return (uint64_t)lo | ((uint64_t)hi << 32);
-}
-
-// descriptor of a K-major tile written by TMA with the 128-byte swizzle: 8-row
-// groups 1024 bytes apart (stride byte offset), leading byte offset unused (1),
-// layout type 2 (bits 61-63); a K step of 16 elements inside the 128-byte swizzle
-// span advances the start address by 32 bytes
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
-  const uint32_t lo = ((saddr >> 4) & 0x3fffu) | (1u << 16);
-  const uint32_t hi = ((1024u >> 4) & 0x3fffu) | (1u << 14) | (2u << 29);
-  return (uint64_t)lo | ((uint64_t)hi << 32);
-}
-
-// instruction descriptor: fp32 accumulator (bits 4-5), bf16 A (7-9) and B (10-12),
-// both K-major, N / 8 (bits 17-22), M / 16 (bits 24-28)
-template <int N>
-__device__ __forceinline__ uint32_t instr_desc() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kTcTile >> 4) << 24);
-}
-
 // r <= 64: the three W_H^T parts, stacked, are one B operand of N = 3r (each key
 // slice is read from shared memory once per K step); the epilogue adds the three
 // column groups.  r = 128: three accumulating MMAs of N = r per K step.
@@ -103,70 +75,8 @@ __host__ __device__ constexpr int tc_tmem_cols(int R) {  // two accumulators, ro
   return 2 * tc_acc_cols(R) <= 64 ? 64 : 2 * tc_acc_cols(R) <= 128 ? 128 : 2 * tc_acc_cols(R) <= 256 ? 256 : 512;
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-
-// 32 consecutive fp32 columns of this thread's TMEM lane
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]),
-        "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
-
-// 2-D TMA tile load (no multicast) completing on an mbarrier of this CTA
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"((uint32_t)__cvta_generic_to_shared(bar))
-      : "memory");
-}
-__device__ __forceinline__ void mbar_expect(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(
-                   (uint32_t)__cvta_generic_to_shared(bar)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"((uint32_t)__cvta_generic_to_shared(bar))
-               : "memory");
-}
-
 // bounded wait for the phase of the given parity (false: not complete after the limit)
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = (uint32_t)__cvta_generic_to_shared(bar);
-  for (uint32_t i = 0; i < kTcWaitTries; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
-}
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity) { return tc::mbar_wait(bar, parity, kTcWaitTries); }
 
 template <int R>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -214,9 +124,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto issue_load = [&](int i) {
     const int tile = (int)blockIdx.x + i * (int)gridDim.x;
     const uint32_t dst = xbase + (uint32_t)(i % S) * kTcTileBytes;
-    mbar_expect(&full[i % S], (uint32_t)kTcTileBytes);
-    tma_load_2d(dst, &xmap, 0, row_base + tile * kTcTile, &full[i % S]);
-    tma_load_2d(dst + kTcTileBytes / 2, &xmap, 64, row_base + tile * kTcTile, &full[i % S]);
+    tc::mbar_expect(&full[i % S], (uint32_t)kTcTileBytes);
+    tc::tma_load_2d(dst, &xmap, 0, row_base + tile * kTcTile, &full[i % S]);
+    tc::tma_load_2d(dst + kTcTileBytes / 2, &xmap, 64, row_base + tile * kTcTile, &full[i % S]);
     loaded_s = i + 1;
   };
   if (tid == 0) {
@@ -254,12 +164,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       *reinterpret_cast<uint4*>(sm + 2 * WPART + off) = *reinterpret_cast<const uint4*>(p3);
     }
   }
-  fence_async_smem();  // the W_H parts (generic stores) before the tensor core reads them
+  tc::fence_async_smem();  // the W_H parts (generic stores) before the tensor core reads them
   __syncthreads();
-  tc_fence_after();
+  tc::fence_after();
   const uint32_t tmem = tmem_base_s;
-  const uint32_t idesc = instr_desc<CAT ? 3 * R : R>();
-  const uint64_t bd0 = smem_desc(sbase);  // W_H^T part 0, first K step
+  const uint32_t idesc = tc::idesc_bf16(kTcTile, CAT ? 3 * R : R, false);
+  const uint64_t bd0 = tc::desc_kmajor_cm(sbase);  // W_H^T part 0, first K step
 
   // bounded wait; on expiry record the timeout once and stop issuing work
   auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
@@ -277,11 +187,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int c = 0; c < NWd; ++c) {
       const uint32_t ta = tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)((i & 1) * AC + 32 * c);
       uint32_t v[32];
-      tc_ld32(ta, v);
+      tc::ld32(ta, v);
       if constexpr (CAT) {  // y = (x.w1 + x.w2) + x.w3
         uint32_t v2[32], v3[32];
-        tc_ld32(ta + R, v2);
-        tc_ld32(ta + 2 * R, v3);
+        tc::ld32(ta + R, v2);
+        tc::ld32(ta + 2 * R, v3);
 #pragma unroll
         for (int j = 0; j < 32; ++j)
           v[j] = __float_as_uint((__uint_as_float(v[j]) + __uint_as_float(v2[j])) + __uint_as_float(v3[j]));
@@ -309,18 +219,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool ok = wait_or_abort(&full[i % S], (uint32_t)((i / S) & 1));
         if (ok && i >= 2) ok = wait_or_abort(&acc_free[i & 1], (uint32_t)(((i - 2) >> 1) & 1));
         if (!ok) break;
-        tc_fence_after();
+        tc::fence_after();
         // descriptors advance by adding (byte offset >> 4) to the start-address field
         // (every address stays below 256 KB, so the field never carries)
-        const uint64_t ad0 = smem_desc_sw128(xbase + (uint32_t)(i % S) * kTcTileBytes);
+        const uint64_t ad0 = tc::desc_kmajor_sw128(xbase + (uint32_t)(i % S) * kTcTileBytes);
         const uint32_t d = tmem + (uint32_t)((i & 1) * AC);
 #pragma unroll
         for (int p = 0; p < (CAT ? 1 : 3); ++p)
 #pragma unroll
           for (int ks = 0; ks < D / 16; ++ks)
-            tc_mma(d, ad0 + (uint64_t)(((ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32) >> 4),
+            tc::mma(d, ad0 + (uint64_t)(((ks >> 2) * (kTcTileBytes / 2) + (ks & 3) * 32) >> 4),
                    bd0 + (uint64_t)((p * WPART + ks * 256) >> 4), idesc, (p | ks) ? 1u : 0u);
-        tc_commit(&mma_done[i & 1]);
+        tc::commit(&mma_done[i & 1]);
         issued_s = i + 1;
         if (i >= 1 && i - 1 + S < nmine) {  // tile i - 1's MMAs done: its stage takes tile i - 1 + S
           if (!wait_or_abort(&mma_done[(i - 1) & 1], (uint32_t)(((i - 1) >> 1) & 1))) break;
@@ -331,10 +241,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {  // epilogue warps: tile j's codes once its MMAs are done, then free its accumulator
     for (int j = 0; j < nmine; ++j) {
       const bool ok = wait_or_abort(&mma_done[j & 1], (uint32_t)((j >> 1) & 1));
-      tc_fence_after();
+      tc::fence_after();
       if (ok) epilogue(j);
-      tc_fence_before();
-      mbar_arrive(&acc_free[j & 1]);
+      tc::fence_before();
+      tc::mbar_arrive(&acc_free[j & 1]);
       if (!ok) break;
     }
   }
@@ -345,7 +255,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (issued_s > 0) tc_wait(&mma_done[(issued_s - 1) & 1], (uint32_t)(((issued_s - 1) >> 1) & 1));
     }
     __syncwarp();
-    tc_fence_after();
+    tc::fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(TCOLS) : "memory");
   }
 }
@@ -392,26 +302,7 @@ cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, i
   if (rows + kTcTile >= 0x7fffffffLL) return cudaErrorNotSupported;
   // x as a 2-D tensor [rows][128] bf16; boxes of 128 rows x 64 elements, 128-byte swizzle
   CUtensorMap xmap;
-  const cuuint64_t gdim[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  const cuuint64_t gstride[1] = {(cuuint64_t)kHeadDim * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)kTcTile};
-  const cuuint32_t estride[2] = {1, 1};
-  // the driver's tensor-map encoder, looked up once through the runtime (no link-time driver dependency)
-  static const PFN_cuTensorMapEncodeTiled encode_tiled = []() -> PFN_cuTensorMapEncodeTiled {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess) {
-      (void)cudaGetLastError();
-      return nullptr;
-    }
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
-  }();
-  if (!encode_tiled) return cudaErrorNotSupported;
-  if (encode_tiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorNotSupported;
+  if (!make_bf16_rows_map(&xmap, x, rows, kTcTile)) return cudaErrorNotSupported;
   // one wave: one CTA per SM, split evenly over the (batch, head) pairs
   const unsigned per_head = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms / heads));
   dim3 grid(per_head, (unsigned)heads);

@@ -11,6 +11,10 @@ cudaError_t launch_encode(const hata_dims_t& d, const void* x, int x_heads, int 
                           const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len, uint32_t* status,
                           cudaStream_t stream);
 
+size_t prefill_ws_bytes(const hata_dims_t& d);
+cudaError_t launch_prefill(const hata_dims_t& d, const void* q, const void* K, const void* V, const float* W,
+                           void* codes, const int32_t* seq_lens, float scale, void* out, char* ws,
+                           cudaStream_t stream);
 cudaError_t launch_append_kv(const hata_dims_t& d, const void* new_k, const void* new_v, void* K, void* V,
                              const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,

@@ -24,6 +24,9 @@ Recipe (all draws from numpy PCG64 streams spawned from SeedSequence(seed)):
     0.8 * qbar_g + 0.6 * N(0, 1) and rounded, where qbar_g is the fp32 mean of
     the G query heads of KV group g.  n_p = 40 for the tiny workload, otherwise
     floor(0.01 * L_b).
+  * prefill prompts: queries at every position, [Lmax][d] per (batch, query head)
+    ~ N(0, 1) (optionally scaled, for sharper softmax), each slab from its own
+    stream so that sampled rows can be redrawn without the rest.
 """
 from __future__ import annotations
 
@@ -42,10 +45,12 @@ __all__ = [
     "random_codes",
     "random_scores",
     "random_indices",
+    "prompt_queries",
 ]
 
 N_STREAMS = 8
 S_Q, S_K, S_V, S_W, S_LENS, S_PLANT_POS, S_PLANT_NOISE, S_CODES = range(N_STREAMS)
+PROMPT_TAG = 0x5071  # spawn key of the prompt queries' streams
 
 
 @dataclass(frozen=True)
@@ -169,6 +174,15 @@ def make_inputs(wl: Workload, seed: int = 0, plant: bool = True) -> dict:
             )
             planted.append(pos)
     return {"q": q, "K": K, "V": V, "W_H": W, "seq_lens": seq_lens, "planted": planted}
+
+
+def prompt_queries(wl: Workload, seed: int, b: int, h: int, q_scale: float = 1.0) -> np.ndarray:
+    """The prefill prompt's queries of batch b, query head h: [Lmax][d] ~ N(0, q_scale^2),
+    rounded to the workload dtype.  Each (b, h) slab has its own stream (SeedSequence
+    of (seed, PROMPT_TAG, b, h)), so a slab can be drawn again without the rest."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, PROMPT_TAG, b, h]))
+    x = rng.standard_normal((wl.max_seq, wl.head_dim), dtype=np.float32)
+    return _round(x * np.float32(q_scale), wl.dtype)
 
 
 def random_codes(shape, hash_bits: int, seed: int = 0) -> np.ndarray:

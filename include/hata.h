@@ -286,6 +286,34 @@ HATA_API hata_status_t hata_dense_decode(const hata_dims_t* dims, const void* q,
                                          size_t workspace_bytes, void* stream);
 
 /*
+ * Causal prefill attention with the key HashEncode fused in (整体框架, prefill
+ * phase: the prompt runs full attention while every key is hashed and its code
+ * cached for decode; 实验: the encode costs under 1%).  For every batch b, query
+ * head h (KV group g = h / G) and position t < L_b = seq_lens[b]:
+ *     out[b][h][t][:] = sum_{s <= t} softmax_s(scale * q[b][h][t] . K[b][g][s]) V[b][g][s][:]
+ * and, when codes is not NULL, for every s < L_b:
+ *     codes[b][g][s] = pack(K[b][g][s][:] . W_H[g] > 0)      (as hata_encode_append)
+ *   q, out      device [B][Hq][max_seq][d] bf16; rows t >= L_b of out are not written
+ *   K, V        device [B][Hkv][max_seq][d] bf16
+ *   W_H         device [Hkv][d][r] fp32 (ignored when codes is NULL)
+ *   codes       device [B][Hkv][max_seq][r/32] uint32 ([..][max_seq] uint16 for
+ *               r = 16), or NULL for plain prefill attention; r <= 128
+ *   scale       softmax scale, > 0; 0 selects 1/sqrt(d)
+ * bf16 only (HATA_ERR_UNSUPPORTED otherwise).  Logits and P.V run on tcgen05
+ * tensor-core tiles (bf16 in, fp32 accumulate, probabilities rounded to bf16),
+ * so outputs agree with exact attention within the bf16 tolerance; code bits
+ * can differ from the exact sign only where |x . W_H| is within fp32 rounding
+ * of zero.  The workspace (hata_prefill_workspace_size bytes, 16-byte aligned)
+ * holds the status word and W_H split into bf16 parts; no initialisation is
+ * needed.  L_b > max_seq is clamped and flagged in the status word; a bounded
+ * wait that runs out records HATA_ERR_TIMEOUT there (hata_read_device_status).
+ */
+HATA_API hata_status_t hata_prefill_workspace_size(const hata_dims_t* dims, size_t* bytes);
+HATA_API hata_status_t hata_prefill_attention(const hata_dims_t* dims, const void* q, const void* K, const void* V,
+                                     const float* W_H, void* codes, const int32_t* seq_lens, float scale, void* out,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * hata_topk without a workspace, for callers that cannot allocate device memory
  * (no counterpart on the pages: it only changes where scratch lives).  Same
  * inputs, outputs and results as hata_topk.  Its scratch is one 8 MiB array of

@@ -55,6 +55,7 @@ __all__ = [
     "decode_step",
     "encode_cache",
     "append_kv",
+    "prefill_attention_row",
 ]
 
 
@@ -190,6 +191,25 @@ def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, S: np.ndarray,
         p = np.exp(s - m)
         out[h] = (p @ Vs) / np.sum(p)
     return out
+
+
+# ----------------------------------------------------------------------------
+# Prefill attention  (§整体框架 prefill phase: full attention over the prompt,
+# during which every key is encoded and its code cached)
+# ----------------------------------------------------------------------------
+
+def prefill_attention_row(q_t: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, scale: float) -> np.ndarray:
+    """Causal attention output of prompt position t for one query head, in float64:
+    o = sum_{s <= t} softmax_s(scale * q_t . K_s) V_s, with K/V the head's KV group
+    ([L][d], L > t).  Written out directly from the definition; the prefill of a
+    whole prompt is this row for every position t < L_b and every query head h
+    (KV group h // G)."""
+    q64 = np.asarray(q_t, dtype=np.float64)
+    Ks = np.asarray(K[: t + 1], dtype=np.float64)
+    Vs = np.asarray(V[: t + 1], dtype=np.float64)
+    logits = scale * (Ks @ q64)
+    w = np.exp(logits - np.max(logits))
+    return (w / np.sum(w)) @ Vs
 
 
 # ----------------------------------------------------------------------------

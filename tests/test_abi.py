@@ -83,6 +83,19 @@ def test_calls_reject_bad_arguments_before_launch(H):
     assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, P(0x1008), 16, null) == 5
     assert lib.hata_encode_append(ctypes.byref(d), fake, 1, 64, 1, null, fake, fake, 64, fake, 8, null) == 5
     assert lib.hata_hamming_scores(ctypes.byref(d), fake, fake, null, fake, null) == 1
+    # prefill attention: bf16 only, pointers required, scale >= 0, workspace large enough
+    F0 = ctypes.c_float(0.0)
+    pf = lambda dd, q, codes, W, scale, ws, wsb: lib.hata_prefill_attention(  # noqa: E731
+        ctypes.byref(dd), q, fake, fake, W, codes, fake, scale, fake, ws, wsb, null)
+    db = H.dims_for(1, 4, 1, 128, 32, 64, "bf16")
+    assert pf(H.dims_for(1, 4, 1, 128, 32, 64, "f32"), fake, fake, fake, F0, fake, 1 << 30) == 2
+    assert pf(db, null, fake, fake, F0, fake, 1 << 30) == 1
+    assert pf(db, fake, fake, null, F0, fake, 1 << 30) == 1  # codes without W_H
+    assert pf(db, fake, fake, fake, ctypes.c_float(-1.0), fake, 1 << 30) == 1
+    assert pf(db, fake, fake, fake, F0, fake, 16) == 5
+    assert pf(db, fake, fake, fake, F0, null, 1 << 30) == 5
+    n = ctypes.c_size_t(0)
+    assert lib.hata_prefill_workspace_size(ctypes.byref(db), ctypes.byref(n)) == 0 and n.value >= 16 + 3 * 32 * 256
     # the cache update: every pointer required, all 16-byte aligned
     assert lib.hata_append_kv(ctypes.byref(d), fake, fake, fake, fake, null, null) == 1
     assert lib.hata_append_kv(ctypes.byref(d), null, fake, fake, fake, fake, null) == 1

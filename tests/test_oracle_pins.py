@@ -404,3 +404,39 @@ def test_append_kv_writes_only_the_new_slot():
                 assert np.array_equal(K2[b, g, t], nk[b, g] if hit else K[b, g, t])
                 assert np.array_equal(V2[b, g, t], nv[b, g] if hit else V[b, g, t])
     assert np.array_equal(K2[0, :, 0], nk[0]) and np.array_equal(V2[1, :, 5], nv[1])
+
+
+def test_prefill_row_closed_forms():
+    """Causal prefill attention: position 0 sees only itself (output = V_0 exactly);
+    identical keys give the plain mean of the visible values; two positions give
+    the two-term softmax written by hand."""
+    rng = np.random.default_rng(9)
+    d, L = 4, 6
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal(d)
+    assert np.array_equal(oracle.prefill_attention_row(q, K, V, 0, 0.5), V[0])
+    Keq = np.tile(K[:1], (L, 1))
+    assert np.allclose(oracle.prefill_attention_row(q, Keq, V, 4, 0.5), V[:5].mean(axis=0), atol=1e-15)
+    s0, s1 = 0.5 * q @ K[0], 0.5 * q @ K[1]
+    want = (math.exp(s0) * V[0] + math.exp(s1) * V[1]) / (math.exp(s0) + math.exp(s1))
+    assert np.allclose(oracle.prefill_attention_row(q, K, V, 1, 0.5), want, atol=1e-14)
+    # later positions never influence earlier rows
+    K2, V2 = K.copy(), V.copy()
+    K2[3:] += 100.0
+    V2[3:] -= 7.0
+    assert np.array_equal(oracle.prefill_attention_row(q, K2, V2, 2, 0.5), oracle.prefill_attention_row(q, K, V, 2, 0.5))
+
+
+def test_prefill_row_is_sparse_attention_over_the_prefix():
+    """Row t of the causal prefill equals attention over the selected set {0..t}
+    (the decode step's attention with every earlier token selected)."""
+    rng = np.random.default_rng(10)
+    d, L = 8, 40
+    K = rng.standard_normal((L, d))
+    V = rng.standard_normal((L, d))
+    q = rng.standard_normal(d)
+    for t in (0, 7, 39):
+        got = oracle.prefill_attention_row(q, K, V, t, 0.3)
+        want = oracle.sparse_attention(q[None, :], K, V, np.arange(t + 1), 0.3)[0]
+        assert np.allclose(got, want, atol=1e-12)
