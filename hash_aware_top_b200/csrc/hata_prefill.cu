@@ -18,7 +18,7 @@
 //   * warps 0-3 own one query row per thread (TMEM lane = row): a first pass over
 //     S_j finds the row maximum, a second writes p = 2^(s * scale * log2 e - m)
 //     as bf16 straight into the K-major swizzled layout the tensor core reads for
-//     P_j, and sums the rounded p.  The running maximum m used for O moves only
+//     P_j, and sums p.  The running maximum m used for O moves only
 //     when a row's maximum exceeds it by more than 2^8; then O's row is rescaled
 //     in TMEM (before PV_j is issued).  The diagonal tile masks keys after the row.
 // On the diagonal tile the key tile K_i is already in shared memory: the CTA of
@@ -107,6 +107,52 @@ __global__ void __launch_bounds__(256) split_w_kernel(const float* __restrict__ 
     *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(p1);
     *reinterpret_cast<uint4*>(dst + WPART + off) = *reinterpret_cast<const uint4*>(p2);
     *reinterpret_cast<uint4*>(dst + 2 * WPART + off) = *reinterpret_cast<const uint4*>(p3);
+  }
+}
+
+// scores of keys after row m (column col0 + e > m) set to -inf: the causal mask of the diagonal tile
+__device__ __forceinline__ void mask_after_row(uint32_t (&va)[32], uint32_t (&vb)[32], int col0, int m) {
+  const uint32_t ninf = 0xff800000u;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    va[e] = col0 + e <= m ? va[e] : ninf;
+    vb[e] = col0 + 32 + e <= m ? vb[e] : ninf;
+  }
+}
+
+__device__ __forceinline__ float tree_max64(uint32_t (&va)[32], const uint32_t (&vb)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) va[e] = __float_as_uint(fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int e = 0; e < w; ++e) va[e] = __float_as_uint(fmaxf(__uint_as_float(va[e]), __uint_as_float(va[e + w])));
+  return __uint_as_float(va[0]);
+}
+
+// sum of 64 values by a tree of additions (consumes va)
+__device__ __forceinline__ float tree_sum64(uint32_t (&va)[32], const uint32_t (&vb)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) va[e] = __float_as_uint(__uint_as_float(va[e]) + __uint_as_float(vb[e]));
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+    for (int e = 0; e < w; ++e) va[e] = __float_as_uint(__uint_as_float(va[e]) + __uint_as_float(va[e + w]));
+  return __uint_as_float(va[0]);
+}
+
+// 32 probabilities of row m as bf16 into the P tile's 128-byte row (16-byte chunks
+// q0 .. q0 + 3 of the row, placed by the 128-byte swizzle: chunk ^ (m & 7))
+__device__ __forceinline__ void store_p_chunk(unsigned char* row, int q0, int m, const uint32_t (&v)[32]) {
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 2 * e]), __uint_as_float(v[8 * qq + 2 * e + 1]));
+      w4[e] = *reinterpret_cast<const uint32_t*>(&pb);
+    }
+    *reinterpret_cast<uint4*>(row + (((q0 + qq) ^ (m & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
 }
 
@@ -307,17 +353,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::fence_after();
       const uint32_t sa = lane_base + (uint32_t)((j & 1) * kPfTile);
       const bool diag = j == i;
-      // pass 1: the row maximum over the visible keys (scale > 0, so of the raw scores)
+      // pass 1: the row maximum over the visible keys (scale > 0, so of the raw scores); two
+      // 32-column loads at a time, a tree of maxima (short dependency chains), the diagonal
+      // tile's keys after the row set to -inf first
       float mx = -INFINITY;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tc::ld32(sa + 32 * cc, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float s = __uint_as_float(v[e]);
-          mx = (!diag || 32 * cc + e <= m) ? fmaxf(mx, s) : mx;
-        }
+#pragma unroll 1
+      for (int cc = 0; cc < 4; cc += 2) {
+        uint32_t va[32], vb[32];
+        tc::ld32_nowait(sa + 32 * cc, va);
+        tc::ld32_nowait(sa + 32 * cc + 32, vb);
+        tc::ld_wait();
+        if (diag) mask_after_row(va, vb, 32 * cc, m);
+        mx = fmaxf(mx, tree_max64(va, vb));
       }
       const float m_tile = mx * c;
       // the previous PV is done: P may be overwritten and O is stable
@@ -330,7 +377,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       } else if (__any_sync(0xffffffffu, m_tile > m_used + kRescaleSlack)) {
         const float m_new = fmaxf(m_used, m_tile);
         const float alpha = ex2(m_used - m_new);
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
           tc::ld32(lane_base + kColO + 32 * cc, o);
@@ -342,29 +389,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2: p = 2^(s c - m_used) as bf16 into P (K-major, 128-byte swizzle), row sum of the rounded p
+      // pass 2: p = 2^(s c - m_used) (0 for masked keys) as bf16 into P (K-major, 128-byte
+      // swizzle), and the row sum of p
       unsigned char* prow = pf_smem + (base - tc::smem_u32(pf_smem)) + kPfP + (m >> 3) * 1024 + (m & 7) * 128;
       float sum = 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; cc += 2) {
+        uint32_t va[32], vb[32];
+        tc::ld32_nowait(sa + 32 * cc, va);
+        tc::ld32_nowait(sa + 32 * cc + 32, vb);
+        tc::ld_wait();
+        if (diag) mask_after_row(va, vb, 32 * cc, m);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t v[32];
-        tc::ld32(sa + 32 * cc, v);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const bool vis0 = !diag || 32 * cc + e <= m, vis1 = !diag || 32 * cc + e + 1 <= m;
-          const float p0 = vis0 ? ex2(fmaf(__uint_as_float(v[e]), c, -m_used)) : 0.f;
-          const float p1 = vis1 ? ex2(fmaf(__uint_as_float(v[e + 1]), c, -m_used)) : 0.f;
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          sum += __low2float(pb) + __high2float(pb);
-          pk[e >> 1] = *reinterpret_cast<const uint32_t*>(&pb);
+        for (int e = 0; e < 32; ++e) {
+          va[e] = __float_as_uint(ex2(fmaf(__uint_as_float(va[e]), c, -m_used)));
+          vb[e] = __float_as_uint(ex2(fmaf(__uint_as_float(vb[e]), c, -m_used)));
         }
-        unsigned char* half = prow + (cc >> 1) * (kPfTileBytes / 2);
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int ch = ((cc & 1) * 4 + qq) ^ (m & 7);
-          *reinterpret_cast<uint4*>(half + ch * 16) = make_uint4(pk[4 * qq], pk[4 * qq + 1], pk[4 * qq + 2], pk[4 * qq + 3]);
-        }
+        store_p_chunk(prow + (cc >> 1) * (kPfTileBytes / 2), 0, m, va);
+        store_p_chunk(prow + (cc >> 1) * (kPfTileBytes / 2), 4, m, vb);
+        sum += tree_sum64(va, vb);
       }
       l += sum;
       // the last tile of the sequence: value rows at or beyond L_b (never visible, possibly not finite)
