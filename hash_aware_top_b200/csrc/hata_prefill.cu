@@ -10,20 +10,22 @@
 //
 // One CTA of five warps per (query tile of 128 positions, query head, batch),
 // heaviest tiles launched first.  For key tiles j = 0 .. i (i = the query tile):
-//   * warp 4 (one lane) streams Q once and K / V tiles (TMA, 128-byte swizzle; a
-//     3-deep K ring and a 2-deep V ring), issues S_j = Q K_j^T (M = N = 128,
-//     K = 16 per MMA) into one of two TMEM score buffers, and, once P_j is in
-//     shared memory, O += P_j V_j into the TMEM output accumulator (V read as an
-//     MN-major operand, so it needs no transpose);
+//   * warp 4 (one lane) streams Q once and K / V tiles (TMA, 128-byte swizzle; 3-deep
+//     K and V rings), issues S_j = Q K_j^T (M = N = 128, K = 16 per MMA) into one of
+//     three TMEM score buffers, and, once P_j is written, O += P_j V_j into the TMEM
+//     output accumulator, with P_j read from TMEM and V as an MN-major operand (no
+//     transpose);
 //   * warps 0-3 own one query row per thread (TMEM lane = row): a first pass over
-//     S_j finds the row maximum, a second writes p = 2^(s * scale * log2 e - m)
-//     as bf16 straight into the K-major swizzled layout the tensor core reads for
-//     P_j, and sums p.  The running maximum m used for O moves only
-//     when a row's maximum exceeds it by more than 2^8; then O's row is rescaled
-//     in TMEM (before PV_j is issued).  The diagonal tile masks keys after the row.
+//     S_j finds the row maximum, a second computes p = 2^(s * scale * log2 e - m),
+//     stores it as bf16 pairs over the first 64 columns of S_j's buffer (the A
+//     operand of PV_j) and sums p.  A buffer is reused three tiles later, after
+//     PV_j has read it, so the softmax of tile j never waits for PV_{j-1}.  The
+//     running maximum m used for O moves only when a row's maximum exceeds it by
+//     more than 2^8; then O's row is rescaled in TMEM once PV_{j-1} has landed
+//     (PV_j is issued after).  The diagonal tile masks keys after the row.
 // On the diagonal tile the key tile K_i is already in shared memory: the CTA of
 // the group's first query head copies W_H^T (three bf16 parts, split once per
-// call into the workspace) into the freed V / P buffers and runs Y = K_i W_H as
+// call into the workspace) into the freed V ring and runs Y = K_i W_H as
 // three accumulating MMAs of N = r into TMEM; the softmax warps turn Y into code
 // words after writing the output.  Only the summation order differs from an
 // fp32 dot product, so a code bit can differ from the exact sign only where |y|
@@ -43,23 +45,26 @@ namespace hata {
 
 namespace {
 
-constexpr int kPfThreads = 160;  // warps 0-3: softmax / epilogue, warp 4: TMA + MMA issue
+constexpr int kPfThreads = 320;  // warps 0-7: two softmax / epilogue warpgroups, 8: MMA issue, 9: TMA
+constexpr int kPfSoftmax = 256;
+constexpr int kPfMmaWarp = 8, kPfTmaWarp = 9;
 constexpr int kPfTile = 128;
 constexpr int kPfTileBytes = kPfTile * kHeadDim * 2;  // 32 KB of bf16
-constexpr int kPfKStages = 3, kPfVStages = 2;
+constexpr int kPfKStages = 3, kPfVStages = 3;
+constexpr int kPfSBufs = 3;  // TMEM score buffers; P_j overwrites the first 64 columns of S_j
 constexpr uint32_t kPfQ = 0;
 constexpr uint32_t kPfK = kPfQ + kPfTileBytes;
 constexpr uint32_t kPfV = kPfK + kPfKStages * kPfTileBytes;
-constexpr uint32_t kPfP = kPfV + kPfVStages * kPfTileBytes;
-constexpr uint32_t kPfW = kPfV;  // W_H^T parts on the diagonal: the V ring and P, 96 KB contiguous
-constexpr int kPfSmem = (int)(kPfP + kPfTileBytes) + 1024;  // + alignment to 1024 bytes
-constexpr uint32_t kPfTmemCols = 512;  // S0 [0,128) S1 [128,256) O [256,384) Y [384,512)
-constexpr uint32_t kColO = 256, kColY = 384;
+constexpr uint32_t kPfEnd = kPfV + kPfVStages * kPfTileBytes;
+constexpr uint32_t kPfW = kPfV;  // W_H^T parts on the diagonal: the V ring, 96 KB
+constexpr int kPfSmem = (int)kPfEnd + 1024;  // + alignment to 1024 bytes
+constexpr uint32_t kPfTmemCols = 512;  // S0 [0,128) S1 [128,256) S2 [256,384) O [384,512); Y in S0
+constexpr uint32_t kColO = 384, kColY = 0;
 constexpr uint32_t kPfWaitTries = 1u << 22;
 constexpr uint32_t kPfTestWaitTries = 1u << 10;
 constexpr float kRescaleSlack = 8.f;  // log2 units: p <= 2^8 between rescales
 
-static_assert(kPfW + 3 * 128 * kHeadDim * 2 <= kPfP + kPfTileBytes, "W_H^T parts fit the V ring and P");
+static_assert(kPfW + 3 * 128 * kHeadDim * 2 <= kPfEnd, "W_H^T parts fit the V ring");
 
 struct PfParams {
   int B, Hq, Hkv, G, max_seq, n_qt;
@@ -141,19 +146,9 @@ __device__ __forceinline__ float tree_sum64(uint32_t (&va)[32], const uint32_t (
   return __uint_as_float(va[0]);
 }
 
-// 32 probabilities of row m as bf16 into the P tile's 128-byte row (16-byte chunks
-// q0 .. q0 + 3 of the row, placed by the 128-byte swizzle: chunk ^ (m & 7))
-__device__ __forceinline__ void store_p_chunk(unsigned char* row, int q0, int m, const uint32_t (&v)[32]) {
-#pragma unroll
-  for (int qq = 0; qq < 4; ++qq) {
-    uint32_t w4[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(v[8 * qq + 2 * e]), __uint_as_float(v[8 * qq + 2 * e + 1]));
-      w4[e] = *reinterpret_cast<const uint32_t*>(&pb);
-    }
-    *reinterpret_cast<uint4*>(row + (((q0 + qq) ^ (m & 7)) * 16)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-  }
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo, uint32_t hi) {
+  const __nv_bfloat162 pb = __floats2bfloat162_rn(__uint_as_float(lo), __uint_as_float(hi));
+  return *reinterpret_cast<const uint32_t*>(&pb);
 }
 
 template <int R>  // R = 0: attention only
@@ -162,10 +157,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                    const __grid_constant__ CUtensorMap vmap, const PfParams p) {
   extern __shared__ __align__(1024) unsigned char pf_smem[];
   __shared__ __align__(8) uint64_t q_full, k_full[kPfKStages], k_free[kPfKStages], v_full[kPfVStages],
-      v_free[kPfVStages], s_full[2], p_full, pv_done, w_full, y_done, drain, never;
+      v_free[kPfVStages], s_full[kPfSBufs], s_free[kPfSBufs], p_full, pv_done, w_full, y_done, drain, never;
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
   __shared__ int k_issued_s, v_issued_s, w_issued_s;
+  __shared__ float l_part[2][kPfTile];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbh = p.B * p.Hq;
@@ -184,7 +180,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int kv_row = (b * p.Hkv + g) * p.max_seq;
 
   if (warp == 0) tc::tmem_alloc(&tmem_s, kPfTmemCols);
-  if (tid == 128) {
+  if (tid == kPfSoftmax) {
     tc::mbar_init(&q_full, 1);
     for (int s = 0; s < kPfKStages; ++s) {
       tc::mbar_init(&k_full[s], 1);
@@ -194,9 +190,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::mbar_init(&v_full[s], 1);
       tc::mbar_init(&v_free[s], 1);
     }
-    tc::mbar_init(&s_full[0], 1);
-    tc::mbar_init(&s_full[1], 1);
-    tc::mbar_init(&p_full, 128);
+    for (int s = 0; s < kPfSBufs; ++s) {
+      tc::mbar_init(&s_full[s], 1);
+      tc::mbar_init(&s_free[s], 1);
+    }
+    tc::mbar_init(&p_full, kPfSoftmax);
     tc::mbar_init(&pv_done, 1);
     tc::mbar_init(&w_full, 1);
     tc::mbar_init(&y_done, 1);
@@ -224,9 +222,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     return false;
   };
 
-  if (warp == 4) {
+  if (warp == kPfTmaWarp) {
     if (lane == 0) {
-      // ---------------- producer: TMA loads and MMA issue ----------------
+      // ---------------- loader: Q once, then K_t / V_t into 3-deep rings ----------------
       auto load_k = [&](int t) {
         const uint32_t dst = base + kPfK + (uint32_t)(t % kPfKStages) * kPfTileBytes;
         tc::mbar_expect(&k_full[t % kPfKStages], (uint32_t)kPfTileBytes);
@@ -244,8 +242,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::mbar_expect(&q_full, (uint32_t)kPfTileBytes);
       tc::tma_load_2d(base + kPfQ, &qmap, 0, q_row, &q_full);
       tc::tma_load_2d(base + kPfQ + kPfTileBytes / 2, &qmap, 64, q_row, &q_full);
-      for (int t = 0; t < min(kPfKStages, n); ++t) load_k(t);
-      for (int t = 0; t < min(kPfVStages, n); ++t) load_v(t);
+      // K_t once S_{t-3} is done with its stage, V_t once PV_{t-3} is
+      for (int t = 0; t < n; ++t) {
+        if (t >= kPfKStages && !wait_ok(&k_free[t % kPfKStages], (uint32_t)(((t - kPfKStages) / kPfKStages) & 1)))
+          break;
+        load_k(t);
+        if (t >= kPfVStages && !wait_ok(&v_free[t % kPfVStages], (uint32_t)(((t - kPfVStages) / kPfVStages) & 1)))
+          break;
+        load_v(t);
+      }
+      // drain: every copy still in flight lands before the CTA leaves
+      const int kl = k_issued_s, vl = v_issued_s;
+      for (int t = max(0, kl - kPfKStages); t < kl; ++t)
+        tc::mbar_wait(&k_full[t % kPfKStages], (uint32_t)((t / kPfKStages) & 1), kPfWaitTries);
+      for (int t = max(0, vl - kPfVStages); t < vl; ++t)
+        tc::mbar_wait(&v_full[t % kPfVStages], (uint32_t)((t / kPfVStages) & 1), kPfWaitTries);
+      tc::mbar_wait(&q_full, 0, kPfWaitTries);
+    }
+  } else if (warp == kPfMmaWarp) {
+    if (lane == 0) {
+      // ---------------- MMA issue: S_j, then PV_{j-1} ----------------
       bool ok = true;
       if (p.test_expire && !tc::mbar_wait(&never, 0, kPfTestWaitTries)) {  // test hook: this wait runs out
         set_status(p.status, HATA_ERR_TIMEOUT);
@@ -255,44 +271,40 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       ok = ok && wait_ok(&q_full, 0);
       constexpr uint32_t idS = tc::idesc_bf16(kPfTile, kPfTile, false);
       constexpr uint32_t idPV = tc::idesc_bf16(kPfTile, kHeadDim, true);
-      auto issue_pv = [&](int t) {  // O (+)= P_t V_t
+      auto issue_pv = [&](int t) {  // O (+)= P_t V_t, P_t read from TMEM (8 columns per 16 keys)
         tc::fence_after();
         const uint32_t vb = base + kPfV + (uint32_t)(t % kPfVStages) * kPfTileBytes;
+        const uint32_t pa = tmem + (uint32_t)((t % kPfSBufs) * kPfTile);
 #pragma unroll
-        for (int ks = 0; ks < kPfTile / 16; ++ks)
-          tc::mma(tmem + kColO,
-                  tc::desc_kmajor_sw128(base + kPfP + (uint32_t)((ks >> 2) * (kPfTileBytes / 2) + (ks & 3) * 32)),
-                  tc::desc_mnmajor_sw128(vb + (uint32_t)ks * 2048u, (uint32_t)(kPfTileBytes / 2)), idPV,
-                  (t > 0 || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < kPfTile / 16; ++ks)  // keys 64 w .. 64 w + 63 of P at columns 64 w ..
+          tc::mma_ts(tmem + kColO, pa + (uint32_t)((ks >> 2) * 64 + (ks & 3) * 8),
+                     tc::desc_mnmajor_sw128(vb + (uint32_t)ks * 2048u, (uint32_t)(kPfTileBytes / 2)), idPV,
+                     (t > 0 || ks > 0) ? 1u : 0u);
         tc::commit(&pv_done);
         tc::commit(&v_free[t % kPfVStages]);
+        tc::commit(&s_free[t % kPfSBufs]);
       };
       for (int j = 0; ok && j < n; ++j) {
         if (!(ok = wait_ok(&k_full[j % kPfKStages], (uint32_t)((j / kPfKStages) & 1)))) break;
+        // score buffer j % 3 is free once PV_{j-3} (which read P_{j-3} from it) is done
+        if (j >= kPfSBufs &&
+            !(ok = wait_ok(&s_free[j % kPfSBufs], (uint32_t)(((j - kPfSBufs) / kPfSBufs) & 1))))
+          break;
         tc::fence_after();
-        // S_j = Q K_j^T into score buffer j & 1 (free: P_{j-2} was waited for before PV_{j-2})
+        // S_j = Q K_j^T
         const uint32_t kb = base + kPfK + (uint32_t)(j % kPfKStages) * kPfTileBytes;
 #pragma unroll
         for (int ks = 0; ks < kHeadDim / 16; ++ks) {
           const uint32_t off = (uint32_t)((ks >> 2) * (kPfTileBytes / 2) + (ks & 3) * 32);
-          tc::mma(tmem + (uint32_t)((j & 1) * kPfTile), tc::desc_kmajor_sw128(base + kPfQ + off),
+          tc::mma(tmem + (uint32_t)((j % kPfSBufs) * kPfTile), tc::desc_kmajor_sw128(base + kPfQ + off),
                   tc::desc_kmajor_sw128(kb + off), idS, ks > 0 ? 1u : 0u);
         }
-        tc::commit(&s_full[j & 1]);
+        tc::commit(&s_full[j % kPfSBufs]);
         tc::commit(&k_free[j % kPfKStages]);
         if (j >= 1) {
           if (!(ok = wait_ok(&p_full, (uint32_t)((j - 1) & 1)))) break;
           if (!(ok = wait_ok(&v_full[(j - 1) % kPfVStages], (uint32_t)(((j - 1) / kPfVStages) & 1)))) break;
           issue_pv(j - 1);
-          // refills: K_{j+2} into K_{j-1}'s stage once S_{j-1} is done, V_{j+1} into V_{j-1}'s once PV_{j-1} is
-          if (j + 2 < n) {
-            if (!(ok = wait_ok(&k_free[(j - 1) % kPfKStages], (uint32_t)(((j - 1) / kPfKStages) & 1)))) break;
-            load_k(j + 2);
-          }
-          if (j + 1 < n) {
-            if (!(ok = wait_ok(&v_free[(j - 1) % kPfVStages], (uint32_t)(((j - 1) / kPfVStages) & 1)))) break;
-            load_v(j + 1);
-          }
         }
       }
       if (ok) ok = wait_ok(&p_full, (uint32_t)((n - 1) & 1));
@@ -300,7 +312,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (ok) issue_pv(n - 1);
       if constexpr (R > 0) {
         if (ok && enc) {
-          // Y = K_i W_H: the W_H^T parts into the V ring and P once the last PV has read them
+          // Y = K_i W_H: the W_H^T parts into the V ring once the last PV has read it
           ok = wait_ok(&pv_done, (uint32_t)((n - 1) & 1));
           if (ok) {
             constexpr uint32_t wbytes = 3u * R * kHeadDim * 2u;
@@ -325,21 +337,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
-      // drain: every MMA issued above, and every copy still in flight, completes before the CTA leaves
+      // drain: every MMA issued above completes before the CTA leaves
       tc::commit(&drain);
       tc::mbar_wait(&drain, 0, kPfWaitTries);
-      const int kl = k_issued_s, vl = v_issued_s;
-      for (int t = max(0, kl - kPfKStages); t < kl; ++t)
-        tc::mbar_wait(&k_full[t % kPfKStages], (uint32_t)((t / kPfKStages) & 1), kPfWaitTries);
-      for (int t = max(0, vl - kPfVStages); t < vl; ++t)
-        tc::mbar_wait(&v_full[t % kPfVStages], (uint32_t)((t / kPfVStages) & 1), kPfWaitTries);
-      tc::mbar_wait(&q_full, 0, kPfWaitTries);
       if (w_issued_s) tc::mbar_wait(&w_full, 0, kPfWaitTries);
     }
   } else {
-    // ---------------- softmax warps: query row m = tid ----------------
-    const int m = tid;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
+    // ---------------- softmax warpgroups: query row m = tid % 128 ----------------
+    // Both warpgroups find the full row maximum (identical arithmetic, so identical m);
+    // warpgroup w then owns keys 64 w .. 64 w + 63 of each tile (exponentials, P, its
+    // part of the row sum) and columns 64 w .. 64 w + 63 of O (rescale, output).
+    const int wg = warp >> 2;
+    const int m = tid & 127;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const float c = p.scale_log2;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -349,9 +359,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     for (int j = 0; j < n; ++j) {
-      if (!(ok = wait_warp(&s_full[j & 1], (uint32_t)((j >> 1) & 1)))) break;
+      if (!(ok = wait_warp(&s_full[j % kPfSBufs], (uint32_t)((j / kPfSBufs) & 1)))) break;
       tc::fence_after();
-      const uint32_t sa = lane_base + (uint32_t)((j & 1) * kPfTile);
+      const uint32_t sa = lane_base + (uint32_t)((j % kPfSBufs) * kPfTile);
       const bool diag = j == i;
       // pass 1: the row maximum over the visible keys (scale > 0, so of the raw scores); two
       // 32-column loads at a time, a tree of maxima (short dependency chains), the diagonal
@@ -367,18 +377,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mx = fmaxf(mx, tree_max64(va, vb));
       }
       const float m_tile = mx * c;
-      // the previous PV is done: P may be overwritten and O is stable
-      if (j >= 1) {
-        if (!(ok = wait_warp(&pv_done, (uint32_t)((j - 1) & 1)))) break;
-        tc::fence_after();
-      }
       if (j == 0) {
         m_used = m_tile;
       } else if (__any_sync(0xffffffffu, m_tile > m_used + kRescaleSlack)) {
+        // O is rescaled once the previous PV has landed (PV_j is issued only after this tile's P)
+        if (!(ok = wait_warp(&pv_done, (uint32_t)((j - 1) & 1)))) break;
+        tc::fence_after();
         const float m_new = fmaxf(m_used, m_tile);
         const float alpha = ex2(m_used - m_new);
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 2 * wg; cc < 2 * wg + 2; ++cc) {
           uint32_t o[32];
           tc::ld32(lane_base + kColO + 32 * cc, o);
 #pragma unroll
@@ -389,12 +397,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2: p = 2^(s c - m_used) (0 for masked keys) as bf16 into P (K-major, 128-byte
-      // swizzle), and the row sum of p
-      unsigned char* prow = pf_smem + (base - tc::smem_u32(pf_smem)) + kPfP + (m >> 3) * 1024 + (m & 7) * 128;
+      // pass 2 (this warpgroup's 64 keys): p = 2^(s c - m_used) (0 for masked keys), packed as
+      // bf16 pairs over the first half of the scores it just read (columns 64 w .. 64 w + 31
+      // of this buffer), and its part of the row sum
       float sum = 0.f;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; cc += 2) {
+      {
+        const int cc = 2 * wg;
         uint32_t va[32], vb[32];
         tc::ld32_nowait(sa + 32 * cc, va);
         tc::ld32_nowait(sa + 32 * cc + 32, vb);
@@ -405,30 +413,37 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           va[e] = __float_as_uint(ex2(fmaf(__uint_as_float(va[e]), c, -m_used)));
           vb[e] = __float_as_uint(ex2(fmaf(__uint_as_float(vb[e]), c, -m_used)));
         }
-        store_p_chunk(prow + (cc >> 1) * (kPfTileBytes / 2), 0, m, va);
-        store_p_chunk(prow + (cc >> 1) * (kPfTileBytes / 2), 4, m, vb);
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          pk[e] = pack_bf16x2(va[2 * e], va[2 * e + 1]);
+          pk[16 + e] = pack_bf16x2(vb[2 * e], vb[2 * e + 1]);
+        }
+        tc::st32(sa + 32 * cc, pk);
         sum += tree_sum64(va, vb);
       }
       l += sum;
+      tc::st_wait();
       // the last tile of the sequence: value rows at or beyond L_b (never visible, possibly not finite)
       // are zeroed so that 0 * V stays 0 in PV
       if (j == n - 1 && kPfTile * n > L) {
         if (!(ok = wait_warp(&v_full[j % kPfVStages], (uint32_t)((j / kPfVStages) & 1)))) break;
-        if (kPfTile * j + m >= L) {
+        if (kPfTile * j + m >= L) {  // warpgroup w: the row's half in box w (elements 64 w ..)
           unsigned char* vrow = pf_smem + (base - tc::smem_u32(pf_smem)) + kPfV + (j % kPfVStages) * kPfTileBytes +
-                                (m >> 3) * 1024 + (m & 7) * 128;
+                                wg * (kPfTileBytes / 2) + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
-          for (int qq = 0; qq < 8; ++qq) {
-            *reinterpret_cast<uint4*>(vrow + qq * 16) = make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(vrow + kPfTileBytes / 2 + qq * 16) = make_uint4(0u, 0u, 0u, 0u);
-          }
+          for (int qq = 0; qq < 8; ++qq) *reinterpret_cast<uint4*>(vrow + qq * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       tc::fence_async_smem();
       tc::fence_before();
       tc::mbar_arrive(&p_full);
     }
-    // output rows: O / l once the last PV is done
+    // the row sum of both halves (every softmax thread reaches this barrier, also after an abort)
+    l_part[wg][m] = l;
+    asm volatile("bar.sync 1, %0;\n" ::"n"(kPfSoftmax) : "memory");
+    l = l_part[0][m] + l_part[1][m];
+    // output rows: O / l once the last PV is done (warpgroup w: columns 64 w .. 64 w + 63)
     if (ok) ok = wait_warp(&pv_done, (uint32_t)((n - 1) & 1));
     if (ok) {
       tc::fence_after();
@@ -436,7 +451,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.out + ((size_t)(b * p.Hq + h) * p.max_seq + t) * kHeadDim;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 2 * wg; cc < 2 * wg + 2; ++cc) {
         uint32_t o[32];
         tc::ld32(lane_base + kColO + 32 * cc, o);
         if (t < L) {
@@ -455,7 +470,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
     if constexpr (R > 0) {
-      if (ok && enc) {
+      if (ok && enc && wg == 0) {
         ok = wait_warp(&y_done, 0);
         if (ok) {
           tc::fence_after();
