@@ -572,6 +572,47 @@ class LayerSet:
                 "l2_mb": round(self.l2 / 1e6)}
 
 
+def time_prefill_encode(H, ls, stream):
+    """hata_encode_append over every cached key of the layer buffers (prefill form), timed with CUDA
+    events on the launching stream; the keys/s, bytes and tensor-core figures of one call."""
+    import torch
+
+    wl, layers, R, inp = ls.wl, ls.layers, ls.R, ls.inp
+    reps = max(2, min(R, 8))
+    with torch.cuda.stream(stream):
+        L0 = layers[0]
+        H.hata_encode_append(ls.dims, L0["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L0["lens"], L0["W"],
+                             L0["codes"], wl.max_seq, ls.ws, stream)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(reps):
+            L = layers[i % R]
+            H.hata_encode_append(ls.dims, L["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L["lens"], L["W"],
+                                 L["codes"], wl.max_seq, ls.ws, stream)
+        e1.record(stream)
+        e1.synchronize()
+    pre_ms = e0.elapsed_time(e1) / reps
+    n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
+    pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + max(wl.hash_bits // 8, 2))
+    res = {"kernel": "hata_encode_append (prefill form; bf16 keys: tcgen05 tensor cores)",
+           "us_per_call": pre_ms * 1e3, "keys": n_keys,
+           "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
+           "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
+           "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
+    if wl.dtype == "bf16" and 32 <= wl.hash_bits <= 128:
+        # the tensor cores run W_H as three bf16 parts: 3x the algorithmic flops
+        res["mma_tflops"] = 3.0 * res["tflops"]
+        tpeak = tensor_peak_bf16()
+        if tpeak:
+            res["frac_of_tensor_peak"] = res["mma_tflops"] / tpeak
+    if H.hata_read_device_status(ls.ws) != 0:
+        raise RuntimeError("device status set by the prefill encode")
+    peak, _ = peak_hbm()
+    res["frac_of_peak"] = res["achieved_gbs"] / peak
+    return res
+
+
 def run_gpu(args, wl):
     world, rank, local = dist_env()
     inp = make_inputs(wl, seed=args.seed)
@@ -648,35 +689,7 @@ def run_gpu(args, wl):
                  "hata_speedup": d_ms / ms_per_step}
 
     # prefill encode (hata_encode_append over every cached key of every layer buffer)
-    pre_reps = max(2, min(R, 8))
-    with torch.cuda.stream(stream):
-        H.hata_encode_append(dims, layers[0]["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, layers[0]["lens"],
-                             layers[0]["W"], layers[0]["codes"], wl.max_seq, ws, stream)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(pre_reps):
-            L = layers[i % R]
-            H.hata_encode_append(dims, L["K"], wl.n_kv_heads, wl.max_seq, wl.max_seq, L["lens"], L["W"], L["codes"],
-                                 wl.max_seq, ws, stream)
-        e1.record(stream)
-        e1.synchronize()
-    pre_ms = e0.elapsed_time(e1) / pre_reps
-    n_keys = int(sum(int(Lb) for Lb in inp["seq_lens"])) * wl.n_kv_heads
-    pre_bytes = n_keys * (wl.head_dim * (2 if wl.dtype == "bf16" else 4) + wl.hash_bits // 8)
-    prefill = {"kernel": "hata_encode_append (prefill form; bf16 keys: tcgen05 tensor cores)",
-               "us_per_call": pre_ms * 1e3, "keys": n_keys,
-               "keys_per_s": n_keys / (pre_ms * 1e-3), "bytes_per_call": pre_bytes,
-               "achieved_gbs": pre_bytes / (pre_ms * 1e-3) / 1e9,
-               "tflops": 2.0 * n_keys * wl.head_dim * wl.hash_bits / (pre_ms * 1e-3) / 1e12}
-    if wl.dtype == "bf16" and wl.hash_bits <= 128:
-        # the tensor cores run W_H as three bf16 parts: 3x the algorithmic flops
-        prefill["mma_tflops"] = 3.0 * prefill["tflops"]
-        tpeak = tensor_peak_bf16()
-        if tpeak:
-            prefill["frac_of_tensor_peak"] = prefill["mma_tflops"] / tpeak
-    if H.hata_read_device_status(ws) != 0:
-        raise RuntimeError("device status set by the prefill encode")
+    prefill = time_prefill_encode(H, ls, stream)
 
     # the same step over a paged cache: every layer's K, V and codes are rearranged in
     # place into pools of 256-token blocks placed by a random (non-contiguous) block
@@ -722,7 +735,6 @@ def run_gpu(args, wl):
 
     peak, peak_kind = peak_hbm()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
-    prefill["frac_of_peak"] = prefill["achieved_gbs"] / peak
     if dense is not None:
         dense["frac_of_peak"] = dense["achieved_gbs"] / peak
 
@@ -746,7 +758,8 @@ def run_gpu(args, wl):
         gbs2 = ls2.step_bytes / (ms2 * 1e-3) / 1e9
         workloads[name] = {"steps": n2, "us_per_step": ms2 * 1e3, "steps_per_s": 1e3 / ms2,
                            "algorithmic_bytes_per_step": ls2.step_bytes, "achieved_gbs": gbs2,
-                           "frac": gbs2 / peak, **ls2.timing_note()}
+                           "frac": gbs2 / peak, **ls2.timing_note(),
+                           "prefill_encode": time_prefill_encode(H, ls2, stream)}
         del ls2
         torch.cuda.empty_cache()
 

@@ -303,8 +303,13 @@ cudaError_t launch_encode_tc(const hata_dims_t& d, const void* x, int x_heads, i
   // x as a 2-D tensor [rows][128] bf16; boxes of 128 rows x 64 elements, 128-byte swizzle
   CUtensorMap xmap;
   if (!make_bf16_rows_map(&xmap, x, rows, kTcTile)) return cudaErrorNotSupported;
-  // one wave: one CTA per SM, split evenly over the (batch, head) pairs
-  const unsigned per_head = (unsigned)std::max<long long>(1, std::min<long long>(tiles, sms / heads));
+  // Few (batch, head) pairs: one wave, one CTA per SM split evenly over the pairs.  Many
+  // pairs (per-sequence lengths are only known on the device, and may differ widely): about
+  // four waves of CTAs, several per pair striding over its tiles, so that the block
+  // scheduler evens out long and short sequences.
+  long long per = sms / heads;
+  if (per < 4) per = (4LL * sms + heads - 1) / heads;
+  const unsigned per_head = (unsigned)std::max<long long>(1, std::min<long long>(tiles, per));
   dim3 grid(per_head, (unsigned)heads);
   switch (d.hash_bits) {
     case 32:
