@@ -403,7 +403,7 @@ def tensor_peak_bf16_sustained():
         return None
 
 
-def bench_prefill_attention(H, dev, local, seed, stream, reps=3):
+def bench_prefill_attention(H, dev, local, seed, stream, reps=3, shape=None):
     """Causal prefill attention over the narrow-code workload's prompts (4 x 65,536 tokens,
     32 query / 8 KV heads, r = 32): attention alone, attention with the key encode fused
     (hata_prefill_attention with codes), and the standalone prefill encode of the same keys
@@ -414,6 +414,8 @@ def bench_prefill_attention(H, dev, local, seed, stream, reps=3):
 
     wl = WORKLOADS[PREFILL_WORKLOAD]
     B, Hq, Hkv, L, r = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.max_seq, wl.hash_bits
+    if shape is not None:  # a smaller prompt of the same heads (e.g. for a profiler capture)
+        B, L = shape
     g = torch.Generator(device=dev)
     g.manual_seed(seed + 17)
     Q = torch.randn((B, Hq, L, wl.head_dim), device=dev, generator=g).to(torch.bfloat16)
@@ -451,7 +453,8 @@ def bench_prefill_attention(H, dev, local, seed, stream, reps=3):
     ms = {n: statistics.median(v) for n, v in times.items()}
     flops = 4.0 * wl.head_dim * Hq * B * L * (L + 1) / 2  # q.K and P.V over the causal triangle
     tflops = flops / (ms["attention"] * 1e-3) / 1e12
-    res = {"workload": f"{PREFILL_WORKLOAD}: {B} x {L}-token prompts, {Hq}/{Hkv} heads, d {wl.head_dim}, r {r}, bf16",
+    name = PREFILL_WORKLOAD if shape is None else f"{PREFILL_WORKLOAD} heads"
+    res = {"workload": f"{name}: {B} x {L}-token prompts, {Hq}/{Hkv} heads, d {wl.head_dim}, r {r}, bf16",
            "kernel": "hata_prefill_attention (tcgen05 causal attention; key encode fused on the diagonal tile)",
            "reps": reps, "attention_ms": ms["attention"], "fused_ms": ms["fused"],
            "fused_encode_overhead_ms": ms["fused"] - ms["attention"],
@@ -765,7 +768,7 @@ def run_gpu(args, wl):
 
     prefill_attn = None
     if not args.no_prefill_attention:
-        prefill_attn = bench_prefill_attention(H, dev, local, args.seed, stream)
+        prefill_attn = bench_prefill_attention(H, dev, local, args.seed, stream, shape=args.prefill_shape)
 
     line = {
         "metric": METRIC,
@@ -828,6 +831,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill-attention", action="store_true",
                     help="skip the prefill attention timing (about 3 s of GPU time)")
+    ap.add_argument("--prefill-shape", type=int, nargs=2, metavar=("B", "L"), default=None,
+                    help="prompts of the prefill attention leg (default: the narrow-code workload's 4 x 65536)")
     ap.add_argument("--also", nargs="*", default=None,
                     help="other workloads timed in the same run (default: llama8b_32k beside the 128K headline)")
     args = ap.parse_args(argv)

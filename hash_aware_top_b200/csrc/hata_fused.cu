@@ -1,4 +1,4 @@
-// The HATA decode step as two kernels chained by programmatic dependent launch
+// The HATA decode step as three kernels chained by programmatic dependent launch
 // ("HATA" paper notes, Decode 阶段算法 end to end, with the fusions of 硬件高效优化:
 // projection + sign + bitpack + cache update in one kernel, XOR + popc Hamming
 // scan with coalesced access, gather fused into the attention).
@@ -6,12 +6,17 @@
 // Every (batch, KV head) unit's L cached tokens are cut into chunks of C tokens,
 // and the chunks of all units are spread over all SMs.
 //
-// scan kernel (one CTA per SM, persistent over chunks).  Per chunk:
+// encode kernel (one small CTA per (unit, 32-column code word)):
+//   0. the G query codes and the new key's code (written to cache slot L - 1),
+//      fp32 FMAs in the order of warp_dot128, so the codes equal
+//      hata_encode_append's decode form; the query codes go to the workspace.
+// scan kernel (one CTA per SM, persistent over chunks; it starts once the encode
+// kernel has passed its own wait on the preceding kernel).  Per chunk:
 //   1. bulk-copy (TMA engine, no tensor map) the chunk's codes into shared
-//      memory, all of it in flight at once, one mbarrier per 16 KB piece;
-//   2. encode the G queries of the unit (and the new key, if the chunk holds
-//      slot L - 1: its code is written to the cache) with fp32 FMAs in the order
-//      of warp_dot128, so the codes equal hata_encode_append's decode form;
+//      memory, all of it in flight at once, one mbarrier per 16 KB piece (slots
+//      [0, L - 1) are final before the encode kernel ends, so this overlaps it);
+//   2. wait for the encode kernel, then read the query codes (and patch slot L - 1
+//      of a chunk that holds it with the new key's code);
 //   3. score every token (xor + popc, the GQA sum folded into per-word
 //      constants), keeping u16 scores and their histogram in shared memory;
 //   4. write the chunk record: the cumulative histogram (u16 per score), and, in
