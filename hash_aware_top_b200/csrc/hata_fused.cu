@@ -141,8 +141,8 @@ __host__ __device__ inline TailSmem tail_smem(int G, int NW, int esize, const St
     return r;
   };
   s.rec = take((int)geo.unit_bytes);
-  // the K rows' buffer also holds the warps' attention partials [warps][G][d + 2] fp32
-  s.Kr = take(std::max(GB * kHeadDim * esize, (kTThreads / 32) * G * (kHeadDim + 2) * 4));
+  // the K rows' buffer also holds the P.V partial sums [row groups][G][d] fp32
+  s.Kr = take(std::max(GB * kHeadDim * esize, (kTThreads / (kHeadDim / 2)) * G * kHeadDim * 4));
   s.Vr = take(GB * kHeadDim * esize);
   s.lg = take(G * GB * 4);
   s.rowtok = take(GB * 4);
@@ -733,8 +733,9 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   constexpr int BPT = (NBP + kTThreads - 1) / kTThreads;
   constexpr int EPV = 16 / ESZ;
   constexpr int RPR = D * ESZ / 16;          // 16-byte pieces per K or V row
-  constexpr int CPL = D / 32;                // columns of a row per lane in the attention
-  constexpr int RPW = G <= 2 ? 4 : (G == 4 ? 2 : 1);  // rows a warp takes at once (register budget)
+  constexpr int LT = 16;                     // lanes per row in the logits
+  constexpr int LE = D / LT;                 // elements per lane in the logits (8)
+  constexpr int PVG = kTThreads / (D / 2);   // row groups in P.V: thread = (column pair, row group)
   constexpr int OPT = (G * D + kTThreads - 1) / kTThreads;
   static_assert((2 * RPR) % 32 == 0, "a row's K and V pieces fill whole warps");
 
@@ -882,17 +883,17 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   float oacc[OPT];
 #pragma unroll
   for (int q = 0; q < OPT; ++q) oacc[q] = 0.f;
-  // Flash decode per warp: warp w takes rows w, w + 16, ... of every batch (RPW at a
-  // time), keeping per head a running maximum and sum (warp-uniform) and the weighted
-  // sum of V for the lane's columns CPL lane .. CPL lane + CPL - 1.  Exp2 domain: the
-  // logits are scaled by scale * log2(e).
-  float wm[G], wsum[G], wo[G][CPL], xq[G][CPL];
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    wm[h] = -INFINITY;
-    wsum[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < CPL; ++e) wo[h][e] = 0.f;
+  // Attention per gather batch, in the exp2 domain (logits scaled by scale * log2 e):
+  // logits by LT lanes per row into lg, the batch's per-head maximum, p = 2^(logit - m)
+  // in place, then P.V by (column pair, row group) threads whose partial sums meet in
+  // shared memory and fold into oacc against the running per-head (maximum, sum).
+  __shared__ int s_bmax[G];         // the batch's maximum logit per head (order-preserving int)
+  __shared__ float s_m[G], s_l[G];  // running maximum and sum per head
+  __shared__ float s_redl[PVG * G];
+  if (tid < G) {
+    s_bmax[tid] = ord_of(-INFINITY);
+    s_m[tid] = -INFINITY;
+    s_l[tid] = 0.f;
   }
   uint32_t gphase = 0;
   const T* Kg = static_cast<const T*>(p.K);
@@ -967,111 +968,154 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
     __syncthreads();
     if (s_abort) break;  // block-uniform (read after the barrier)
 
-    if (cur == r0) {  // the lane's slice of the queries (xp is ready long before)
+    // logits: LT lanes per row, LE consecutive elements each (xp is ready long before)
+    {
+      const int sgi = lane % LT;
+      float xq[G][LE];
 #pragma unroll
       for (int h = 0; h < G; ++h)
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) xq[h][e] = xp[h * D + CPL * lane + e];
-    }
-    for (int rb = warp; rb < nr; rb += RPW * kNWarp) {  // warp-uniform
-      float lgt[RPW][G];
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const int r = min(rb + i * kNWarp, nr - 1);
-        float kv[CPL];
-        if constexpr (ESZ == 2) {
-          const uint2 w2 = *reinterpret_cast<const uint2*>(Kr + (size_t)r * D + CPL * lane);
-          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.x));
-          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.y));
-          kv[0] = f0.x; kv[1] = f0.y; kv[2] = f1.x; kv[3] = f1.y;
-        } else {
-          const float4 f = *reinterpret_cast<const float4*>(Kr + (size_t)r * D + CPL * lane);
-          kv[0] = f.x; kv[1] = f.y; kv[2] = f.z; kv[3] = f.w;
+        for (int e = 0; e < LE; e += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(xp + h * D + sgi * LE + e);
+          xq[h][e] = a.x;
+          xq[h][e + 1] = a.y;
+          xq[h][e + 2] = a.z;
+          xq[h][e + 3] = a.w;
         }
+      float mx[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
+      for (int rb = warp * (32 / LT); rb < nr; rb += kNWarp * (32 / LT)) {  // warp-uniform trip count
+        const int r = rb + lane / LT;
+        const bool valid = r < nr;
+        const T* kr = Kr + (size_t)(valid ? r : 0) * D + sgi * LE;
+        float kv[LE];
+        if constexpr (ESZ == 2) {
+          const uint4 w4 = *reinterpret_cast<const uint4*>(kr);
+          const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+            kv[2 * e] = f.x;
+            kv[2 * e + 1] = f.y;
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < LE; e += 4) {
+            const float4 f = *reinterpret_cast<const float4*>(kr + e);
+            kv[e] = f.x;
+            kv[e + 1] = f.y;
+            kv[e + 2] = f.z;
+            kv[e + 3] = f.w;
+          }
+        }
+        float acc[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float a = xq[h][0] * kv[0];
 #pragma unroll
-          for (int e = 1; e < CPL; ++e) a = fmaf(xq[h][e], kv[e], a);
-          lgt[i][h] = a;
+          for (int e = 1; e < LE; ++e) a = fmaf(xq[h][e], kv[e], a);
+          acc[h] = a;
         }
-      }
 #pragma unroll
-      for (int o = 16; o; o >>= 1)
+        for (int o = 1; o < LT; o <<= 1)
 #pragma unroll
-        for (int i = 0; i < RPW; ++i)
-#pragma unroll
-          for (int h = 0; h < G; ++h) lgt[i][h] += __shfl_xor_sync(0xffffffffu, lgt[i][h], o);
-#pragma unroll
-      for (int i = 0; i < RPW; ++i) {
-        const int r = rb + i * kNWarp;
-        if (r < nr) {  // warp-uniform
-          float vv[CPL];
-          if constexpr (ESZ == 2) {
-            const uint2 w2 = *reinterpret_cast<const uint2*>(Vr + (size_t)r * D + CPL * lane);
-            const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.x));
-            const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w2.y));
-            vv[0] = f0.x; vv[1] = f0.y; vv[2] = f1.x; vv[3] = f1.y;
-          } else {
-            const float4 f = *reinterpret_cast<const float4*>(Vr + (size_t)r * D + CPL * lane);
-            vv[0] = f.x; vv[1] = f.y; vv[2] = f.z; vv[3] = f.w;
-          }
+          for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+        if (valid && sgi == 0) {
 #pragma unroll
           for (int h = 0; h < G; ++h) {
-            const float l = lgt[i][h] * p.scale_log2;
-            const float mn = fmaxf(wm[h], l);
-            const float alpha = exp2f(wm[h] - mn);  // 0 while the maximum is -inf
-            const float pr = exp2f(l - mn);
-            wsum[h] = fmaf(wsum[h], alpha, pr);
-#pragma unroll
-            for (int e = 0; e < CPL; ++e) wo[h][e] = fmaf(wo[h][e], alpha, pr * vv[e]);
-            wm[h] = mn;
+            const float lv = acc[h] * p.scale_log2;
+            lg[h * GB + r] = lv;
+            mx[h] = fmaxf(mx[h], lv);
           }
         }
       }
-    }
-    __syncthreads();  // every warp is done with the K and V rows of this batch
-  }
-  // combine the warps' partials through shared memory (the K rows' buffer, free now)
-  {
-    constexpr int WS = D + 2;  // per warp and head: the D columns, then the maximum and sum
-    float* wbuf = reinterpret_cast<float*>(Kr);  // [kNWarp][G][WS]
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < G; ++h) {
+        float m = mx[h];
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) wbuf[(warp * G + h) * WS + CPL * lane + e] = wo[h][e];
-      if (lane == 0) {
-        wbuf[(warp * G + h) * WS + D] = wm[h];
-        wbuf[(warp * G + h) * WS + D + 1] = wsum[h];
+        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0 && m != -INFINITY) atomicMax(&s_bmax[h], ord_of(m));
       }
     }
     __syncthreads();
-#pragma unroll
-    for (int q = 0; q < OPT; ++q) {
-      const int e = tid + q * kTThreads;
-      if (e < G * D) {
-        const int h = e / D, col = e % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNWarp; ++w) M = fmaxf(M, wbuf[(w * G + h) * WS + D]);
-        float l = 0.f, o = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < kNWarp; ++w) {
-            const float sc = exp2f(wbuf[(w * G + h) * WS + D] - M);
-            l = fmaf(wbuf[(w * G + h) * WS + D + 1], sc, l);
-            o = fmaf(wbuf[(w * G + h) * WS + col], sc, o);
-          }
-        }
-        oacc[q] = o;
-        if (col == 0) {
-          part[2 * h] = M;
-          part[2 * h + 1] = l;
-        }
-      }
+    // probabilities against the new running maximum of each head
+    for (int e = tid; e < G * nr; e += kTThreads) {
+      const int h = e / nr, i = e - h * nr;
+      const float mn = fmaxf(s_m[h], float_of_ord(s_bmax[h]));
+      lg[h * GB + i] = exp2f(lg[h * GB + i] - mn);
     }
     __syncthreads();
+    // P.V: thread (column pair cp, row group rg) over rows rg, rg + PVG, ...; the PVG partial
+    // sums of each output meet in the K rows' buffer (free once the logits are done)
+    {
+      const int cp = tid % (D / 2), rg = tid / (D / 2);
+      float pacc[G][2], lsum[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
+#pragma unroll 4
+      for (int r = rg; r < nr; r += PVG) {
+        float v0, v1;
+        if constexpr (ESZ == 2) {
+          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * D)[cp]);
+          v0 = f.x;
+          v1 = f.y;
+        } else {
+          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * D)[cp];
+          v0 = f.x;
+          v1 = f.y;
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pr = lg[h * GB + r];
+          pacc[h][0] = fmaf(pr, v0, pacc[h][0]);
+          pacc[h][1] = fmaf(pr, v1, pacc[h][1]);
+          lsum[h] += pr;
+        }
+      }
+      float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+        reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
+      if (cp == 0)
+#pragma unroll
+        for (int h = 0; h < G; ++h) s_redl[rg * G + h] = lsum[h];
+      __syncthreads();
+#pragma unroll
+      for (int q = 0; q < OPT; ++q) {
+        const int e = tid + q * kTThreads;
+        if (e < G * D) {
+          const int h = e / D, i = e % D;
+          const float m_old = s_m[h];
+          const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
+          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
+          oacc[q] = fmaf(oacc[q], alpha, sum);
+        }
+      }
+      __syncthreads();  // every thread has read the running maxima and the partial sums
+      if (tid < G) {
+        const int h = tid;
+        const float m_old = s_m[h];
+        const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
+        const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+        float ls = 0.f;
+#pragma unroll
+        for (int j = 0; j < PVG; ++j) ls += s_redl[j * G + h];
+        s_l[h] = s_l[h] * alpha + ls;
+        s_m[h] = mn;
+        s_bmax[h] = ord_of(-INFINITY);
+      }
+    }
   }
+  __syncthreads();
+  if (tid < G) {  // this CTA's partial: running maximum and sum per head (oacc holds the weighted V sums)
+    part[2 * tid] = s_m[tid];
+    part[2 * tid + 1] = s_l[tid];
+  }
+  __syncthreads();
   if (ix && rank == 0) {
     for (int jx = n + tid; jx < p.k; jx += kTThreads) ix[jx] = -1;
     if (!active)

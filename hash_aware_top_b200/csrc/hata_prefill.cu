@@ -8,26 +8,29 @@
 //   codes[b][g][s] = pack(K[b][g][s] . W_H[g] > 0)        (when codes != NULL)
 // for t, s < L_b, with g = h / G.
 //
-// One CTA of five warps per (query tile of 128 positions, query head, batch),
+// One CTA of ten warps per (query tile of 128 positions, query head, batch),
 // heaviest tiles launched first.  For key tiles j = 0 .. i (i = the query tile):
-//   * warp 4 (one lane) streams Q once and K / V tiles (TMA, 128-byte swizzle; 3-deep
-//     K and V rings), issues S_j = Q K_j^T (M = N = 128, K = 16 per MMA) into one of
-//     three TMEM score buffers, and, once P_j is written, O += P_j V_j into the TMEM
-//     output accumulator, with P_j read from TMEM and V as an MN-major operand (no
-//     transpose);
-//   * warps 0-3 own one query row per thread (TMEM lane = row): a first pass over
-//     S_j finds the row maximum, a second computes p = 2^(s * scale * log2 e - m),
-//     stores it as bf16 pairs over the first 64 columns of S_j's buffer (the A
-//     operand of PV_j) and sums p.  A buffer is reused three tiles later, after
-//     PV_j has read it, so the softmax of tile j never waits for PV_{j-1}.  The
-//     running maximum m used for O moves only when a row's maximum exceeds it by
-//     more than 2^8; then O's row is rescaled in TMEM once PV_{j-1} has landed
-//     (PV_j is issued after).  The diagonal tile masks keys after the row.
+//   * warp 9 (one lane) streams Q once and K / V tiles through 3-deep rings (TMA,
+//     128-byte swizzle), refilling a stage once the MMAs reading it are done;
+//   * warp 8 (one lane) issues S_j = Q K_j^T (M = N = 128, K = 16 per MMA) into one
+//     of three TMEM score buffers and, once P_j is written, O += P_j V_j into the
+//     TMEM output accumulator, with P_j read from TMEM and V as an MN-major operand
+//     (no transpose);
+//   * warps 0-7 are two softmax warpgroups over the same 128 query rows (TMEM lane =
+//     row).  Both find the row maximum over all 128 scores of S_j (identical
+//     arithmetic, so the same m); warpgroup w then computes p = 2^(s * scale * log2 e
+//     - m) for keys 64 w .. 64 w + 63, stores it as bf16 pairs over the first half of
+//     the scores it just read (the A operand of PV_j), and sums it.  A buffer is
+//     reused three tiles later, after PV_j has read it, so the softmax of tile j
+//     never waits for PV_{j-1}.  The running maximum m used for O moves only when a
+//     row's maximum exceeds it by more than 2^8; then each warpgroup rescales its half
+//     of O's row in TMEM once PV_{j-1} has landed (PV_j is issued after).  The
+//     diagonal tile masks keys after the row.
 // On the diagonal tile the key tile K_i is already in shared memory: the CTA of
 // the group's first query head copies W_H^T (three bf16 parts, split once per
 // call into the workspace) into the freed V ring and runs Y = K_i W_H as
-// three accumulating MMAs of N = r into TMEM; the softmax warps turn Y into code
-// words after writing the output.  Only the summation order differs from an
+// three accumulating MMAs of N = r into TMEM; warpgroup 0 turns Y into code words
+// after writing its output columns.  Only the summation order differs from an
 // fp32 dot product, so a code bit can differ from the exact sign only where |y|
 // is within fp32 rounding of zero.
 //
