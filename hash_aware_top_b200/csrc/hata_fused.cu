@@ -130,8 +130,13 @@ __host__ __device__ inline ScanSmem scan_smem(int G, int NW) {
 
 // Dynamic shared memory of the tail kernel.
 struct TailSmem {
-  int rec, Kr, Vr, lg, rowtok, rowslot, xp, mslot, sst, qcs, mbar, total;
+  int rec, Kr, Vr, lg, pb, rowtok, rowslot, xp, mslot, sst, qcs, mbar, total;
 };
+// Row stride (elements) of the gathered K and V rows: bf16 rows are padded by 16 bytes so
+// that the tensor-core fragment loads of eight consecutive rows hit distinct banks.
+__host__ __device__ constexpr int tail_row_stride(int esize) { return esize == 2 ? kHeadDim + 8 : kHeadDim; }
+// Row stride (elements) of the bf16 probability tile [8 heads][GB + 8].
+__host__ __device__ constexpr int tail_p_stride(int GB) { return GB + 8; }
 __host__ __device__ inline TailSmem tail_smem(int G, int NW, int esize, const StepGeom& geo, int GB, int CS) {
   TailSmem s{};
   int o = 0;
@@ -142,9 +147,10 @@ __host__ __device__ inline TailSmem tail_smem(int G, int NW, int esize, const St
   };
   s.rec = take((int)geo.unit_bytes);
   // the K rows' buffer also holds the P.V partial sums [row groups][G][d] fp32
-  s.Kr = take(std::max(GB * kHeadDim * esize, (kTThreads / (kHeadDim / 2)) * G * kHeadDim * 4));
-  s.Vr = take(GB * kHeadDim * esize);
+  s.Kr = take(std::max(GB * tail_row_stride(esize) * esize, (kTThreads / (kHeadDim / 2)) * G * kHeadDim * 4));
+  s.Vr = take(GB * tail_row_stride(esize) * esize);
   s.lg = take(G * GB * 4);
+  s.pb = take(esize == 2 ? 8 * tail_p_stride(GB) * 2 : 0);
   s.rowtok = take(GB * 4);
   s.rowslot = take(GB * 8);
   s.xp = take(G * kHeadDim * 4);
@@ -154,6 +160,25 @@ __host__ __device__ inline TailSmem tail_smem(int G, int NW, int esize, const St
   s.mbar = take(2 * 8);
   s.total = o;
   return s;
+}
+
+// D += A * B for a 16x16 bf16 A (row), a 16x8 bf16 B (col) and fp32 D, in the fragment
+// layout of mma.m16n8k16 (g = lane / 4, c = lane % 4): a0 = A[g][2c..2c+1], a2 = A[g][2c+8..];
+// rows 8-15 of A are zero (a1 = a3 = 0); b0 = B[2c..2c+1][g], b1 = B[2c+8..2c+9][g];
+// d0 = D[g][2c], d1 = D[g][2c+1] (d2, d3: rows g + 8).
+__device__ __forceinline__ void mma_16816_top(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// Two transposed 8x8 b16 tiles; lanes 0-7 address tile 0's rows, lanes 8-15 tile 1's.
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t& r0, uint32_t& r1, const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];\n"
+               : "=r"(r0), "=r"(r1)
+               : "r"((unsigned)__cvta_generic_to_shared(row))
+               : "memory");
 }
 
 // Order-preserving map of a float (not NaN) to an int, for integer atomicMax.
@@ -733,6 +758,7 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   constexpr int BPT = (NBP + kTThreads - 1) / kTThreads;
   constexpr int EPV = 16 / ESZ;
   constexpr int RPR = D * ESZ / 16;          // 16-byte pieces per K or V row
+  constexpr int RS = tail_row_stride(ESZ);  // row stride of the gathered rows (elements)
   constexpr int LT = 16;                     // lanes per row in the logits
   constexpr int LE = D / LT;                 // elements per lane in the logits (8)
   constexpr int PVG = kTThreads / (D / 2);   // row groups in P.V: thread = (column pair, row group)
@@ -749,6 +775,7 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   T* Kr = reinterpret_cast<T*>(smem + S.Kr);
   T* Vr = reinterpret_cast<T*>(smem + S.Vr);
   float* lg = reinterpret_cast<float*>(smem + S.lg);
+  __nv_bfloat16* pbt = reinterpret_cast<__nv_bfloat16*>(smem + S.pb);  // (bf16) probabilities [8][GB + 8]
   int* rowtok = reinterpret_cast<int*>(smem + S.rowtok);
   long long* rowslot = reinterpret_cast<long long*>(smem + S.rowslot);  // (paged) cache slot of each row
   float* xp = reinterpret_cast<float*>(smem + S.xp);
@@ -888,6 +915,27 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
   // in place, then P.V by (column pair, row group) threads whose partial sums meet in
   // shared memory and fold into oacc against the running per-head (maximum, sum).
   __shared__ int s_bmax[G];         // the batch's maximum logit per head (order-preserving int)
+  __shared__ float s_wsum[kNWarp];  // (bf16) each warp's sum of its head's probabilities
+  const int PS = tail_p_stride(GB);
+  // (bf16) lane (gq, cq): Q fragments of head gq (zero beyond G) for the logits' A operand, and
+  // the running weighted V sums of head gq, columns 8 w + 2 cq, 8 w + 2 cq + 1 (rows gq + 8 unused)
+  const int gq = lane >> 2, cq = lane & 3;
+  uint32_t qa0[ESZ == 2 ? D / 16 : 1], qa2[ESZ == 2 ? D / 16 : 1];
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if constexpr (ESZ == 2) {
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qa0[ks] = 0u;
+      qa2[ks] = 0u;
+      if (gq < G) {
+        const float* xq_ = xp + gq * D + 16 * ks + 2 * cq;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(xq_[0], xq_[1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(xq_[8], xq_[9]);
+        qa0[ks] = *reinterpret_cast<const uint32_t*>(&lo);
+        qa2[ks] = *reinterpret_cast<const uint32_t*>(&hi);
+      }
+    }
+  }
   __shared__ float s_m[G], s_l[G];  // running maximum and sum per head
   __shared__ float s_redl[PVG * G];
   if (tid < G) {
@@ -956,8 +1004,8 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
       if constexpr (PAGED) slot = (size_t)rowslot[r];
       else slot = token_slot<false>(p, b, g, checked(rowtok[r]));
       const size_t row = slot * D;
-      if (w < RPR) ptx::cp_async16(Kr + (size_t)r * D + w * EPV, Kg + row + w * EPV);
-      else ptx::cp_async16(Vr + (size_t)r * D + (w - RPR) * EPV, Vg + row + (w - RPR) * EPV);
+      if (w < RPR) ptx::cp_async16(Kr + (size_t)r * RS + w * EPV, Kg + row + w * EPV);
+      else ptx::cp_async16(Vr + (size_t)r * RS + (w - RPR) * EPV, Vg + row + (w - RPR) * EPV);
     }
     ptx::cp_async_mbar_arrive_noinc(&mb[1]);
     if (!ptx::mbar_wait_spin(&mb[1], gphase & 1u, kWaitTries)) {
@@ -968,149 +1016,244 @@ __global__ void __launch_bounds__(kTThreads, 1) step_tail_kernel(const StepParam
     __syncthreads();
     if (s_abort) break;  // block-uniform (read after the barrier)
 
-    // logits: LT lanes per row, LE consecutive elements each (xp is ready long before)
-    {
-      const int sgi = lane % LT;
-      float xq[G][LE];
+    if constexpr (ESZ == 2) {
+      // ---- tensor cores (bf16): S = Q K^T and O += P V as mma.m16n8k16, heads as the rows ----
+      const int nr16 = (nr + 15) & ~15;
+      // logits: warp w takes the 8-token groups w, w + 16, ...; lane (gq, cq) gets head gq's
+      // logits of tokens 2 cq and 2 cq + 1 of the group
+      float mxl = -INFINITY;
+      for (int t0 = warp * 8; t0 < nr; t0 += kNWarp * 8) {  // warp-uniform
+        const __nv_bfloat16* krow =
+            reinterpret_cast<const __nv_bfloat16*>(Kr) + (size_t)min(t0 + gq, nr - 1) * RS + 2 * cq;
+        float c4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int e = 0; e < LE; e += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(xp + h * D + sgi * LE + e);
-          xq[h][e] = a.x;
-          xq[h][e + 1] = a.y;
-          xq[h][e + 2] = a.z;
-          xq[h][e + 3] = a.w;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(krow + 16 * ks);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(krow + 16 * ks + 8);
+          mma_16816_top(c4, qa0[ks], qa2[ks], b0, b1);
         }
-      float mx[G];
+        if (gq < G)
 #pragma unroll
-      for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
-      for (int rb = warp * (32 / LT); rb < nr; rb += kNWarp * (32 / LT)) {  // warp-uniform trip count
-        const int r = rb + lane / LT;
-        const bool valid = r < nr;
-        const T* kr = Kr + (size_t)(valid ? r : 0) * D + sgi * LE;
-        float kv[LE];
-        if constexpr (ESZ == 2) {
-          const uint4 w4 = *reinterpret_cast<const uint4*>(kr);
-          const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
-            kv[2 * e] = f.x;
-            kv[2 * e + 1] = f.y;
+          for (int tt = 0; tt < 2; ++tt) {
+            const int t = t0 + 2 * cq + tt;
+            if (t < nr) {
+              const float lv = c4[tt] * p.scale_log2;
+              lg[gq * GB + t] = lv;
+              mxl = fmaxf(mxl, lv);
+            }
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < LE; e += 4) {
-            const float4 f = *reinterpret_cast<const float4*>(kr + e);
-            kv[e] = f.x;
-            kv[e + 1] = f.y;
-            kv[e + 2] = f.z;
-            kv[e + 3] = f.w;
-          }
-        }
-        float acc[G];
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float a = xq[h][0] * kv[0];
-#pragma unroll
-          for (int e = 1; e < LE; ++e) a = fmaf(xq[h][e], kv[e], a);
-          acc[h] = a;
-        }
-#pragma unroll
-        for (int o = 1; o < LT; o <<= 1)
-#pragma unroll
-          for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-        if (valid && sgi == 0) {
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float lv = acc[h] * p.scale_log2;
-            lg[h * GB + r] = lv;
-            mx[h] = fmaxf(mx[h], lv);
-          }
-        }
       }
-#pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float m = mx[h];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0 && m != -INFINITY) atomicMax(&s_bmax[h], ord_of(m));
-      }
-    }
-    __syncthreads();
-    // probabilities against the new running maximum of each head
-    for (int e = tid; e < G * nr; e += kTThreads) {
-      const int h = e / nr, i = e - h * nr;
-      const float mn = fmaxf(s_m[h], float_of_ord(s_bmax[h]));
-      lg[h * GB + i] = exp2f(lg[h * GB + i] - mn);
-    }
-    __syncthreads();
-    // P.V: thread (column pair cp, row group rg) over rows rg, rg + PVG, ...; the PVG partial
-    // sums of each output meet in the K rows' buffer (free once the logits are done)
-    {
-      const int cp = tid % (D / 2), rg = tid / (D / 2);
-      float pacc[G][2], lsum[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
-#pragma unroll 4
-      for (int r = rg; r < nr; r += PVG) {
-        float v0, v1;
-        if constexpr (ESZ == 2) {
-          const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * D)[cp]);
-          v0 = f.x;
-          v1 = f.y;
-        } else {
-          const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * D)[cp];
-          v0 = f.x;
-          v1 = f.y;
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const float pr = lg[h * GB + r];
-          pacc[h][0] = fmaf(pr, v0, pacc[h][0]);
-          pacc[h][1] = fmaf(pr, v1, pacc[h][1]);
-          lsum[h] += pr;
-        }
-      }
-      float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
-#pragma unroll
-      for (int h = 0; h < G; ++h)
-        reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
-      if (cp == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) s_redl[rg * G + h] = lsum[h];
+      mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, 1));
+      mxl = fmaxf(mxl, __shfl_xor_sync(0xffffffffu, mxl, 2));
+      if (cq == 0 && gq < G && mxl != -INFINITY) atomicMax(&s_bmax[gq], ord_of(mxl));
+      // V rows [nr, nr16) enter the last k-step with p = 0: make them finite (zero)
+      for (int e = tid; e < (nr16 - nr) * (D / 8); e += kTThreads)
+        *reinterpret_cast<uint4*>(Vr + (size_t)(nr + e / (D / 8)) * RS + (e % (D / 8)) * 8) = make_uint4(0u, 0u, 0u, 0u);
       __syncthreads();
+      // probabilities: warp w takes head w % G, rows (w / G) * 32 + lane, ...; bf16 into the P
+      // tile (zero for rows [nr, nr16)), and the head's sum of the rounded values
+      {
+        const int h = warp % G, wph = kNWarp / G;
+        const float mn = fmaxf(s_m[h], float_of_ord(s_bmax[h]));
+        float sm = 0.f;
+        for (int t = (warp / G) * 32 + lane; t < nr16; t += 32 * wph) {
+          const __nv_bfloat16 pv = __float2bfloat16_rn(t < nr ? exp2f(lg[h * GB + t] - mn) : 0.f);
+          pbt[h * PS + t] = pv;
+          sm += __bfloat162float(pv);
+        }
 #pragma unroll
-      for (int q = 0; q < OPT; ++q) {
-        const int e = tid + q * kTThreads;
-        if (e < G * D) {
-          const int h = e / D, i = e % D;
-          const float m_old = s_m[h];
-          const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
-          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
-          float sum = 0.f;
-#pragma unroll
-          for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
-          oacc[q] = fmaf(oacc[q], alpha, sum);
+        for (int o = 16; o; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
+        if (lane == 0) s_wsum[warp] = sm;
+      }
+      __syncthreads();
+      // P.V into output columns 8 w .. 8 w + 7: the running output is rescaled first
+      {
+        const float m_old = gq < G ? s_m[gq] : 0.f;
+        const float mn = gq < G ? fmaxf(m_old, float_of_ord(s_bmax[gq])) : 0.f;
+        const float al = gq < G && m_old != -INFINITY ? exp2f(m_old - mn) : 0.f;
+        acc[0] *= al;
+        acc[1] *= al;
+        const __nv_bfloat16* ph = pbt + min(gq, G - 1) * PS + 2 * cq;
+        const __nv_bfloat16* vcol = reinterpret_cast<const __nv_bfloat16*>(Vr) + (size_t)(lane & 15) * RS + 8 * warp;
+        for (int ks = 0; ks < nr16 / 16; ++ks) {
+          const uint32_t a0 = gq < G ? *reinterpret_cast<const uint32_t*>(ph + 16 * ks) : 0u;
+          const uint32_t a2 = gq < G ? *reinterpret_cast<const uint32_t*>(ph + 16 * ks + 8) : 0u;
+          uint32_t b0, b1;
+          ldsm_x2_trans(b0, b1, vcol + (size_t)16 * ks * RS);
+          mma_16816_top(acc, a0, a2, b0, b1);
         }
       }
-      __syncthreads();  // every thread has read the running maxima and the partial sums
+      __syncthreads();  // every thread has read the running maxima, the P tile and the V rows
       if (tid < G) {
         const int h = tid;
         const float m_old = s_m[h];
         const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
         const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
         float ls = 0.f;
-#pragma unroll
-        for (int j = 0; j < PVG; ++j) ls += s_redl[j * G + h];
+        for (int w = h; w < kNWarp; w += G) ls += s_wsum[w];
         s_l[h] = s_l[h] * alpha + ls;
         s_m[h] = mn;
         s_bmax[h] = ord_of(-INFINITY);
       }
+    } else {
+      // logits: LT lanes per row, LE consecutive elements each (xp is ready long before)
+      {
+        const int sgi = lane % LT;
+        float xq[G][LE];
+  #pragma unroll
+        for (int h = 0; h < G; ++h)
+  #pragma unroll
+          for (int e = 0; e < LE; e += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(xp + h * D + sgi * LE + e);
+            xq[h][e] = a.x;
+            xq[h][e + 1] = a.y;
+            xq[h][e + 2] = a.z;
+            xq[h][e + 3] = a.w;
+          }
+        float mx[G];
+  #pragma unroll
+        for (int h = 0; h < G; ++h) mx[h] = -INFINITY;
+        for (int rb = warp * (32 / LT); rb < nr; rb += kNWarp * (32 / LT)) {  // warp-uniform trip count
+          const int r = rb + lane / LT;
+          const bool valid = r < nr;
+          const T* kr = Kr + (size_t)(valid ? r : 0) * RS + sgi * LE;
+          float kv[LE];
+          if constexpr (ESZ == 2) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(kr);
+            const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[e]));
+              kv[2 * e] = f.x;
+              kv[2 * e + 1] = f.y;
+            }
+          } else {
+  #pragma unroll
+            for (int e = 0; e < LE; e += 4) {
+              const float4 f = *reinterpret_cast<const float4*>(kr + e);
+              kv[e] = f.x;
+              kv[e + 1] = f.y;
+              kv[e + 2] = f.z;
+              kv[e + 3] = f.w;
+            }
+          }
+          float acc[G];
+  #pragma unroll
+          for (int h = 0; h < G; ++h) {
+            float a = xq[h][0] * kv[0];
+  #pragma unroll
+            for (int e = 1; e < LE; ++e) a = fmaf(xq[h][e], kv[e], a);
+            acc[h] = a;
+          }
+  #pragma unroll
+          for (int o = 1; o < LT; o <<= 1)
+  #pragma unroll
+            for (int h = 0; h < G; ++h) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+          if (valid && sgi == 0) {
+  #pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float lv = acc[h] * p.scale_log2;
+              lg[h * GB + r] = lv;
+              mx[h] = fmaxf(mx[h], lv);
+            }
+          }
+        }
+  #pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float m = mx[h];
+  #pragma unroll
+          for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0 && m != -INFINITY) atomicMax(&s_bmax[h], ord_of(m));
+        }
+      }
+      __syncthreads();
+      // probabilities against the new running maximum of each head
+      for (int e = tid; e < G * nr; e += kTThreads) {
+        const int h = e / nr, i = e - h * nr;
+        const float mn = fmaxf(s_m[h], float_of_ord(s_bmax[h]));
+        lg[h * GB + i] = exp2f(lg[h * GB + i] - mn);
+      }
+      __syncthreads();
+      // P.V: thread (column pair cp, row group rg) over rows rg, rg + PVG, ...; the PVG partial
+      // sums of each output meet in the K rows' buffer (free once the logits are done)
+      {
+        const int cp = tid % (D / 2), rg = tid / (D / 2);
+        float pacc[G][2], lsum[G];
+  #pragma unroll
+        for (int h = 0; h < G; ++h) pacc[h][0] = pacc[h][1] = lsum[h] = 0.f;
+  #pragma unroll 4
+        for (int r = rg; r < nr; r += PVG) {
+          float v0, v1;
+          if constexpr (ESZ == 2) {
+            const float2 f = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(Vr + (size_t)r * RS)[cp]);
+            v0 = f.x;
+            v1 = f.y;
+          } else {
+            const float2 f = reinterpret_cast<const float2*>(Vr + (size_t)r * RS)[cp];
+            v0 = f.x;
+            v1 = f.y;
+          }
+  #pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float pr = lg[h * GB + r];
+            pacc[h][0] = fmaf(pr, v0, pacc[h][0]);
+            pacc[h][1] = fmaf(pr, v1, pacc[h][1]);
+            lsum[h] += pr;
+          }
+        }
+        float* red = reinterpret_cast<float*>(Kr);  // [PVG][G][D]
+  #pragma unroll
+        for (int h = 0; h < G; ++h)
+          reinterpret_cast<float2*>(red + ((size_t)rg * G + h) * D)[cp] = make_float2(pacc[h][0], pacc[h][1]);
+        if (cp == 0)
+  #pragma unroll
+          for (int h = 0; h < G; ++h) s_redl[rg * G + h] = lsum[h];
+        __syncthreads();
+  #pragma unroll
+        for (int q = 0; q < OPT; ++q) {
+          const int e = tid + q * kTThreads;
+          if (e < G * D) {
+            const int h = e / D, i = e % D;
+            const float m_old = s_m[h];
+            const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
+            const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+            float sum = 0.f;
+  #pragma unroll
+            for (int j = 0; j < PVG; ++j) sum += red[((size_t)j * G + h) * D + i];
+            oacc[q] = fmaf(oacc[q], alpha, sum);
+          }
+        }
+        __syncthreads();  // every thread has read the running maxima and the partial sums
+        if (tid < G) {
+          const int h = tid;
+          const float m_old = s_m[h];
+          const float mn = fmaxf(m_old, float_of_ord(s_bmax[h]));
+          const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - mn);
+          float ls = 0.f;
+  #pragma unroll
+          for (int j = 0; j < PVG; ++j) ls += s_redl[j * G + h];
+          s_l[h] = s_l[h] * alpha + ls;
+          s_m[h] = mn;
+          s_bmax[h] = ord_of(-INFINITY);
+        }
+      }
     }
   }
   __syncthreads();
+  if constexpr (ESZ == 2) {  // the accumulators' columns into oacc's layout, through the K rows' buffer
+    float* red = reinterpret_cast<float*>(Kr);  // [G][D]
+    if (gq < G) {
+      red[gq * D + 8 * warp + 2 * cq] = acc[0];
+      red[gq * D + 8 * warp + 2 * cq + 1] = acc[1];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < OPT; ++q) {
+      const int e = tid + q * kTThreads;
+      if (e < G * D) oacc[q] = red[e];
+    }
+    __syncthreads();
+  }
   if (tid < G) {  // this CTA's partial: running maximum and sum per head (oacc holds the weighted V sums)
     part[2 * tid] = s_m[tid];
     part[2 * tid + 1] = s_l[tid];
