@@ -119,8 +119,9 @@ typedef struct {
  * every exchange on chip) is used while the units are few.  The all-SM form (an
  * encode kernel, a scan kernel that spreads every unit's cache over all SMs, and
  * a tail kernel with one cluster per unit, chained by programmatic dependent
- * launch) is used for 64 or more units and for paged caches.  This flag selects
- * the all-SM form for any shape it covers. */
+ * launch) is used for 64 or more units, for 32 or more units that select at least
+ * 32768 rows in all (units x min(k, max_seq)), and for paged caches.  This flag
+ * selects the all-SM form for any shape it covers. */
 #define HATA_FLAG_ALL_SM_SCAN 4
 
 /* Bytes of workspace that every call below needs for these dims and budget k

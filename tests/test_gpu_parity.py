@@ -436,6 +436,9 @@ def test_kernel_count_reports_the_form(H):
     assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16"), 512) == 1
     assert H.hata_decode_step_kernel_count(H.dims_for(16, 32, 8, 128, 128, 65536, "bf16"), 1024) == 3
     assert H.hata_decode_step_kernel_count(H.dims_for(1, 32, 8, 128, 128, 131072, "bf16", 4), 512) == 3
+    # 32 units: the all-SM form once the selection is large (k = 2048), the cluster form for k = 512
+    assert H.hata_decode_step_kernel_count(H.dims_for(4, 32, 8, 128, 32, 65536, "bf16"), 2048) == 3
+    assert H.hata_decode_step_kernel_count(H.dims_for(4, 32, 8, 128, 32, 65536, "bf16"), 512) == 1
     assert H.hata_decode_step_kernel_count(H.dims_for(1, 6, 2, 128, 128, 3000, "bf16"), 100) == 6
 
 
