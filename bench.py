@@ -492,11 +492,15 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
 
     import torch
 
-    def capture(n):
+    def capture(n, events=None):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
+            if events:
+                events[0].record(stream)
             for i in range(n):
                 step(i)
+            if events:
+                events[1].record(stream)
         return g
 
     with torch.cuda.stream(stream):
@@ -504,7 +508,13 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
             step(i)
     torch.cuda.synchronize()
     chunk = min(steps, GRAPH_CHUNK)
-    g_chunk = capture(chunk)
+    # A run that fits one graph records its timing events inside it (event-record nodes), so
+    # they bracket exactly the timed steps on the device and not the host's submission of
+    # the graph; longer runs record them around the replays (the submission gap is then
+    # spread over GRAPH_CHUNK steps per graph).
+    ev0, ev1 = torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True)
+    inside = steps <= GRAPH_CHUNK
+    g_chunk = capture(chunk, (ev0, ev1) if inside else None)
     rem = steps % chunk
     g_rem = capture(rem) if rem else None
     g_warm = capture(warmup)
@@ -518,14 +528,15 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with (sampler or contextlib.nullcontext()), torch.cuda.stream(stream):
-        ev0.record(stream)
+        if not inside:
+            ev0.record(stream)
         for _ in range(steps // chunk):
             g_chunk.replay()
         if g_rem is not None:
             g_rem.replay()
-        ev1.record(stream)
+        if not inside:
+            ev1.record(stream)
         ev1.synchronize()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
@@ -570,9 +581,13 @@ class LayerSet:
             self.layers.append(lay)
         torch.cuda.synchronize()
 
-    def timing_note(self):
-        return {"layer_buffers": self.R, "mb_touched_per_rotation": round(self.R * self.step_bytes / 1e6),
+    def timing_note(self, steps=None):
+        note = {"layer_buffers": self.R, "mb_touched_per_rotation": round(self.R * self.step_bytes / 1e6),
                 "l2_mb": round(self.l2 / 1e6)}
+        if steps is not None:
+            note["events"] = ("recorded inside the one CUDA graph of the timed steps" if steps <= GRAPH_CHUNK else
+                              f"recorded around the replays of CUDA graphs of {GRAPH_CHUNK} steps")
+        return note
 
 
 def time_prefill_encode(H, ls, stream):
@@ -661,11 +676,14 @@ def run_gpu(args, wl):
     # copies its inputs (q and the new token's K and V rows) from pinned host memory in one
     # copy, appends the rows to the caches (hata_append_kv), runs hata_decode_step with the
     # output in pinned host memory, and waits for it
-    e2e_steps = min(args.steps, 2000)
+    # (at least 200 timed steps, after 20 untimed ones, so that a short run's figure is not one
+    # cold step's)
+    e2e_steps = max(200, min(args.steps, 2000))
     in_host, out_host = e2e_inputs(wl, layers[0], inp["seq_lens"])
     stages = [torch.empty_like(in_host, device=dev) for _ in layers]
     h2d = in_host.numel() * in_host.element_size()
     d2h = out_host.numel() * out_host.element_size()
+    run_e2e(H, dims, wl.k, 20, layers, stages, in_host, out_host, ws, stream)  # warm-up
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -732,7 +750,7 @@ def run_gpu(args, wl):
         paged = {"kernel": "hata_decode_step_paged (256-token blocks, random block table)", "steps": p_steps,
                  "us_per_step": p_ms * 1e3, "achieved_gbs": step_bytes / (p_ms * 1e-3) / 1e9,
                  "vs_unpaged": ms_per_step / p_ms}
-    timing = ls.timing_note()
+    timing = ls.timing_note(args.steps)
     del ls, layers
     torch.cuda.empty_cache()
 
@@ -761,7 +779,7 @@ def run_gpu(args, wl):
         gbs2 = ls2.step_bytes / (ms2 * 1e-3) / 1e9
         workloads[name] = {"steps": n2, "us_per_step": ms2 * 1e3, "steps_per_s": 1e3 / ms2,
                            "algorithmic_bytes_per_step": ls2.step_bytes, "achieved_gbs": gbs2,
-                           "frac": gbs2 / peak, **ls2.timing_note(),
+                           "frac": gbs2 / peak, **ls2.timing_note(n2),
                            "prefill_encode": time_prefill_encode(H, ls2, stream)}
         del ls2
         torch.cuda.empty_cache()
