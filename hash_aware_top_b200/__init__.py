@@ -27,6 +27,7 @@ __all__ = [
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_append_kv",
+    "hata_append_kv_paged",
     "hata_prefill_workspace_size",
     "hata_prefill_attention",
     "hata_encode_append",
@@ -60,6 +61,7 @@ EXPORTED_SYMBOLS = (
     "hata_workspace_size",
     "hata_workspace_init",
     "hata_append_kv",
+    "hata_append_kv_paged",
     "hata_prefill_workspace_size",
     "hata_prefill_attention",
     "hata_encode_append",
@@ -125,6 +127,7 @@ def _load():
         "hata_workspace_size": (I, [DP, I, ctypes.POINTER(S)]),
         "hata_workspace_init": (I, [P, S, P]),
         "hata_append_kv": (I, [DP, P, P, P, P, P, P]),
+        "hata_append_kv_paged": (I, [DP, P, P, P, P, P, I, I, P, P]),
         "hata_prefill_workspace_size": (I, [DP, ctypes.POINTER(S)]),
         "hata_prefill_attention": (I, [DP, P, P, P, P, P, P, F, P, P, S, P]),
         "hata_encode_append": (I, [DP, P, I, I, I, P, P, P, I, P, S, P]),
@@ -234,6 +237,24 @@ def hata_append_kv(dims: Dims, new_k, new_v, K, V, seq_lens, stream=None):
             _ptr(K, "K", cache, d.torch_dtype), _ptr(V, "V", cache, d.torch_dtype),
             _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), _stream(stream)),
         "hata_append_kv")
+
+
+def hata_append_kv_paged(dims: Dims, new_k, new_v, K_pool, V_pool, block_table, block_size, seq_lens,
+                         stream=None):
+    """Write the new token's rows new_k/new_v ([B][Hkv][d]) into the paged pools ([n_blocks][Hkv][bs][d])
+    at the slot the block table gives for position seq_lens[b] - 1."""
+    d = dims
+    row = (d.batch, d.n_kv_heads, d.head_dim)
+    n_blocks = K_pool.shape[0]
+    pool = (n_blocks, d.n_kv_heads, int(block_size), d.head_dim)
+    _check(
+        lib.hata_append_kv_paged(
+            ctypes.byref(d),
+            _ptr(new_k, "new_k", row, d.torch_dtype), _ptr(new_v, "new_v", row, d.torch_dtype),
+            _ptr(K_pool, "K_pool", pool, d.torch_dtype), _ptr(V_pool, "V_pool", pool, d.torch_dtype),
+            _ptr(block_table, "block_table", (d.batch, -(-d.max_seq // int(block_size))), torch.int32),
+            int(block_size), int(n_blocks), _ptr(seq_lens, "seq_lens", (d.batch,), torch.int32), _stream(stream)),
+        "hata_append_kv_paged")
 
 
 def hata_prefill_workspace_size(dims: Dims) -> int:

@@ -125,7 +125,27 @@ hata_status_t hata_append_kv(const hata_dims_t* dims, const void* new_k, const v
   if (s != HATA_OK) return s;
   if (!new_k || !new_v || !K || !V || !seq_lens) return HATA_ERR_INVALID_ARG;
   if (!aligned16(new_k) || !aligned16(new_v) || !aligned16(K) || !aligned16(V)) return HATA_ERR_INVALID_ARG;
-  return cuda_status(launch_append_kv(*dims, new_k, new_v, K, V, seq_lens, static_cast<cudaStream_t>(stream)));
+  return cuda_status(
+      launch_append_kv(*dims, new_k, new_v, K, V, seq_lens, nullptr, static_cast<cudaStream_t>(stream)));
+}
+
+hata_status_t hata_append_kv_paged(const hata_dims_t* dims, const void* new_k, const void* new_v, void* K_pool,
+                                   void* V_pool, const int32_t* block_table, int block_size, int n_blocks,
+                                   const int32_t* seq_lens, void* stream) {
+  hata_status_t s = check_dims(dims);
+  if (s != HATA_OK) return s;
+  if (!new_k || !new_v || !K_pool || !V_pool || !block_table || !seq_lens) return HATA_ERR_INVALID_ARG;
+  if (!aligned16(new_k) || !aligned16(new_v) || !aligned16(K_pool) || !aligned16(V_pool)) return HATA_ERR_INVALID_ARG;
+  if (block_size < 16 || block_size > 65536 || (block_size & (block_size - 1)) || n_blocks < 1)
+    return HATA_ERR_INVALID_ARG;
+  PagedCache pg;
+  pg.block_table = block_table;
+  pg.block_shift = 0;
+  while ((1 << pg.block_shift) < block_size) ++pg.block_shift;
+  pg.n_blocks = n_blocks;
+  pg.max_blocks = (dims->max_seq + block_size - 1) / block_size;
+  return cuda_status(
+      launch_append_kv(*dims, new_k, new_v, K_pool, V_pool, seq_lens, &pg, static_cast<cudaStream_t>(stream)));
 }
 
 hata_status_t hata_hamming_scores(const hata_dims_t* dims, const uint32_t* qcode, const uint32_t* codes,

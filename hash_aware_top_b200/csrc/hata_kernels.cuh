@@ -15,8 +15,6 @@ size_t prefill_ws_bytes(const hata_dims_t& d);
 cudaError_t launch_prefill(const hata_dims_t& d, const void* q, const void* K, const void* V, const float* W,
                            void* codes, const int32_t* seq_lens, float scale, void* out, char* ws,
                            cudaStream_t stream);
-cudaError_t launch_append_kv(const hata_dims_t& d, const void* new_k, const void* new_v, void* K, void* V,
-                             const int32_t* seq_lens, cudaStream_t stream);
 cudaError_t launch_hamming(const hata_dims_t& d, const uint32_t* qcode, const uint32_t* codes,
                            const int32_t* seq_lens, int32_t* scores, cudaStream_t stream);
 
@@ -48,6 +46,10 @@ struct PagedCache {
   const int32_t* block_table;
   int block_shift, n_blocks, max_blocks;
 };
+
+// pg: paged pools (the layout of the paged step), or null for [B][Hkv][max_seq][d] caches
+cudaError_t launch_append_kv(const hata_dims_t& d, const void* new_k, const void* new_v, void* K, void* V,
+                             const int32_t* seq_lens, const PagedCache* pg, cudaStream_t stream);
 
 // Wk: separate key encoder, or equal to W (one encoder for queries and keys).
 // pg: paged cache, or null for [B][Hkv][max_seq][...] slabs.

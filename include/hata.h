@@ -149,6 +149,18 @@ HATA_API hata_status_t hata_append_kv(const hata_dims_t* dims, const void* new_k
                              const int32_t* seq_lens, void* stream);
 
 /*
+ * The same cache update for the paged pools of hata_decode_step_paged: the new
+ * rows go to slot (L_b - 1) mod bs of pool block block_table[b][(L_b - 1) / bs]
+ * of K_pool / V_pool ([n_blocks][Hkv][bs][d], dims->dtype, 16-byte aligned).
+ * block_table is device [B][ceil(max_seq / bs)] int32; block_size bs is a power
+ * of two in [16, 65536].  Batches with L_b outside [1, max_seq], or whose block
+ * number lies outside [0, n_blocks), are left unchanged.  No workspace.
+ */
+HATA_API hata_status_t hata_append_kv_paged(const hata_dims_t* dims, const void* new_k, const void* new_v, void* K_pool,
+                                   void* V_pool, const int32_t* block_table, int block_size, int n_blocks,
+                                   const int32_t* seq_lens, void* stream);
+
+/*
  * HashEncode + cache update (Decode 阶段算法, first two steps; 硬件高效优化,
  * fused projection -> sign -> bitpack -> cache update).  For every batch b,
  * head h < x_heads and token t in [end_b - n_tok, end_b) that also lies in

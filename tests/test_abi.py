@@ -100,6 +100,11 @@ def test_calls_reject_bad_arguments_before_launch(H):
     assert lib.hata_append_kv(ctypes.byref(d), fake, fake, fake, fake, null, null) == 1
     assert lib.hata_append_kv(ctypes.byref(d), null, fake, fake, fake, fake, null) == 1
     assert lib.hata_append_kv(ctypes.byref(d), fake, fake, P(0x1008), fake, fake, null) == 1
+    # the paged cache update: pointers, alignment, a power-of-two block size in [16, 65536], a pool
+    assert lib.hata_append_kv_paged(ctypes.byref(d), fake, fake, fake, fake, null, 64, 4, fake, null) == 1
+    assert lib.hata_append_kv_paged(ctypes.byref(d), fake, fake, fake, fake, fake, 48, 4, fake, null) == 1
+    assert lib.hata_append_kv_paged(ctypes.byref(d), fake, fake, fake, fake, fake, 64, 0, fake, null) == 1
+    assert lib.hata_append_kv_paged(ctypes.byref(d), fake, P(0x1004), fake, fake, fake, 64, 4, fake, null) == 1
     # k < 1
     assert lib.hata_topk(ctypes.byref(d), fake, fake, 0, fake, null, fake, 1 << 20, null) == 1
     # workspace too small / missing

@@ -148,3 +148,34 @@ def test_paged_growing_cache_multi_step(H):
         check_against_oracle(wl, q, inp["K"], inp["V"], W, W, codes, lens, codes_after, out, qcode, idx)
         codes = codes_after  # the cache as the GPU left it (codes inside the exemption band included)
     assert H.hata_read_device_status(ws) == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_append_kv_paged(H, dtype):
+    """The paged cache update writes each new row to the slot the block table gives for
+    position L_b - 1 (compared on the dense view with oracle.append_kv), and nothing else;
+    lengths 0 and max_seq + 1 and a block number outside the pool write nothing."""
+    B, Hkv, Lmax, bs = 5, 2, 300, 64
+    rng = np.random.default_rng(41)
+    K0 = rng.standard_normal((B, Hkv, Lmax, 128)).astype(np.float32)
+    V0 = rng.standard_normal((B, Hkv, Lmax, 128)).astype(np.float32)
+    nk = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    nv = rng.standard_normal((B, Hkv, 128)).astype(np.float32)
+    lens = np.array([1, 300, 0, 301, 130], dtype=np.int32)
+    max_blocks = (Lmax + bs - 1) // bs
+    bt, n_blocks = block_table_for(B, max_blocks, 2, seed=43)
+    bt_dev = bt.copy()
+    bt_dev[4, 129 // bs] = n_blocks + 5  # batch 4's page of position 129: outside the pool
+    d = H.dims_for(B, 2 * Hkv, Hkv, 128, 128, Lmax, dtype)
+    rnd = lambda a: dev_float(a, dtype).float().cpu().numpy()  # noqa: E731  (the device's rounding)
+    K0, V0, nk, nv = rnd(K0), rnd(V0), rnd(nk), rnd(nv)
+    Kp = dev_float(to_pool(K0, bt, n_blocks, bs, 0.0), dtype)
+    Vp = dev_float(to_pool(V0, bt, n_blocks, bs, 0.0), dtype)
+    H.hata_append_kv_paged(d, dev_float(nk, dtype), dev_float(nv, dtype), Kp, Vp, torch.from_numpy(bt_dev).cuda(), bs,
+                           torch.from_numpy(lens).cuda())
+    torch.cuda.synchronize()
+    want_lens = lens.copy()
+    want_lens[4] = 0  # its block number is outside the pool: nothing written
+    K2, V2 = oracle.append_kv(K0, V0, nk, nv, want_lens)
+    assert np.array_equal(from_pool(Kp.float().cpu().numpy(), bt, Lmax), K2)
+    assert np.array_equal(from_pool(Vp.float().cpu().numpy(), bt, Lmax), V2)
