@@ -128,16 +128,6 @@ __device__ __forceinline__ void mask_after_row(uint32_t (&va)[32], uint32_t (&vb
   }
 }
 
-__device__ __forceinline__ float tree_max64(uint32_t (&va)[32], const uint32_t (&vb)[32]) {
-#pragma unroll
-  for (int e = 0; e < 32; ++e) va[e] = __float_as_uint(fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
-#pragma unroll
-  for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-    for (int e = 0; e < w; ++e) va[e] = __float_as_uint(fmaxf(__uint_as_float(va[e]), __uint_as_float(va[e + w])));
-  return __uint_as_float(va[0]);
-}
-
 // sum of 64 values by a tree of additions (consumes va)
 __device__ __forceinline__ float tree_sum64(uint32_t (&va)[32], const uint32_t (&vb)[32]) {
 #pragma unroll
@@ -160,7 +150,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                    const __grid_constant__ CUtensorMap vmap, const PfParams p) {
   extern __shared__ __align__(1024) unsigned char pf_smem[];
   __shared__ __align__(8) uint64_t q_full, k_full[kPfKStages], k_free[kPfKStages], v_full[kPfVStages],
-      v_free[kPfVStages], s_full[kPfSBufs], s_free[kPfSBufs], p_full, pv_done, w_full, y_done, drain, never;
+      v_free[kPfVStages], s_full[kPfSBufs], s_free[kPfSBufs], p_full, pv_done, w_full, y_done, drain, never,
+      mx_bar[2];
   __shared__ uint32_t tmem_s;
   __shared__ volatile int abort_s;
   __shared__ int k_issued_s, v_issued_s, w_issued_s;
@@ -203,6 +194,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc::mbar_init(&y_done, 1);
     tc::mbar_init(&drain, 1);
     tc::mbar_init(&never, 1);
+    tc::mbar_init(&mx_bar[0], kPfSoftmax);
+    tc::mbar_init(&mx_bar[1], kPfSoftmax);
     tc::mbar_init_fence();
     abort_s = 0;
     k_issued_s = 0;
@@ -366,19 +359,31 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc::fence_after();
       const uint32_t sa = lane_base + (uint32_t)((j % kPfSBufs) * kPfTile);
       const bool diag = j == i;
-      // pass 1: the row maximum over the visible keys (scale > 0, so of the raw scores); two
-      // 32-column loads at a time, a tree of maxima (short dependency chains), the diagonal
-      // tile's keys after the row set to -inf first
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; cc += 2) {
-        uint32_t va[32], vb[32];
-        tc::ld32_nowait(sa + 32 * cc, va);
-        tc::ld32_nowait(sa + 32 * cc + 32, vb);
-        tc::ld_wait();
-        if (diag) mask_after_row(va, vb, 32 * cc, m);
-        mx = fmaxf(mx, tree_max64(va, vb));
-      }
+      // pass 1 (this warpgroup's 64 keys, kept in registers for pass 2): the maximum over its
+      // visible keys (scale > 0, so of the raw scores; the diagonal tile's keys after the row
+      // set to -inf first), then the other warpgroup's half.  The halves meet in TMEM: column
+      // 64 w + 32 of this score buffer (read already; P only takes the first 32 of each half)
+      // on the row's lane, ordered by mx_bar; two barrier slots suffice, since a warpgroup
+      // reaches tile j + 2 only after both have finished tile j.
+      const int cc = 2 * wg;
+      uint32_t va[32], vb[32];
+      tc::ld32_nowait(sa + 32 * cc, va);
+      tc::ld32_nowait(sa + 32 * cc + 32, vb);
+      tc::ld_wait();
+      if (diag) mask_after_row(va, vb, 32 * cc, m);
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e]));
+#pragma unroll
+      for (int e = 8; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], fmaxf(__uint_as_float(va[e]), __uint_as_float(vb[e])));
+      const float mown = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      tc::st1(sa + 64 * wg + 32, __float_as_uint(mown));
+      tc::st_wait();
+      tc::fence_before();
+      tc::mbar_arrive(&mx_bar[j & 1]);
+      if (!(ok = wait_warp(&mx_bar[j & 1], (uint32_t)((j >> 1) & 1)))) break;
+      tc::fence_after();
+      const float mx = fmaxf(mown, __uint_as_float(tc::ld1(sa + 64 * (wg ^ 1) + 32)));
       const float m_tile = mx * c;
       if (j == 0) {
         m_used = m_tile;
@@ -400,17 +405,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         l *= alpha;
         m_used = m_new;
       }
-      // pass 2 (this warpgroup's 64 keys): p = 2^(s c - m_used) (0 for masked keys), packed as
-      // bf16 pairs over the first half of the scores it just read (columns 64 w .. 64 w + 31
-      // of this buffer), and its part of the row sum
+      // pass 2 (this warpgroup's 64 keys, from pass 1's registers): p = 2^(s c - m_used) (0 for
+      // masked keys), packed as bf16 pairs over the first half of the scores it read (columns
+      // 64 w .. 64 w + 31 of this buffer), and its part of the row sum
       float sum = 0.f;
       {
-        const int cc = 2 * wg;
-        uint32_t va[32], vb[32];
-        tc::ld32_nowait(sa + 32 * cc, va);
-        tc::ld32_nowait(sa + 32 * cc + 32, vb);
-        tc::ld_wait();
-        if (diag) mask_after_row(va, vb, 32 * cc, m);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           va[e] = __float_as_uint(ex2(fmaf(__uint_as_float(va[e]), c, -m_used)));
