@@ -17,10 +17,11 @@
 //     TMEM output accumulator, with P_j read from TMEM and V as an MN-major operand
 //     (no transpose);
 //   * warps 0-7 are two softmax warpgroups over the same 128 query rows (TMEM lane =
-//     row).  Both find the row maximum over all 128 scores of S_j (identical
-//     arithmetic, so the same m); warpgroup w then computes p = 2^(s * scale * log2 e
-//     - m) for keys 64 w .. 64 w + 63, stores it as bf16 pairs over the first half of
-//     the scores it just read (the A operand of PV_j), and sums it.  A buffer is
+//     row).  Warpgroup w reads keys 64 w .. 64 w + 63 of S_j, finds their maximum and
+//     exchanges it with the other warpgroup through a TMEM column (both then hold the
+//     same row maximum m), computes p = 2^(s * scale * log2 e - m) for its keys,
+//     stores it as bf16 pairs over the first half of the scores it read (the A operand
+//     of PV_j), and sums it.  A buffer is
 //     reused three tiles later, after PV_j has read it, so the softmax of tile j
 //     never waits for PV_{j-1}.  The running maximum m used for O moves only when a
 //     row's maximum exceeds it by more than 2^8; then each warpgroup rescales its half
