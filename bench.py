@@ -484,10 +484,20 @@ def graph_upload(g, stream):
         return False
 
 
-def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
-    """Milliseconds for `steps` calls of step(i) replayed from CUDA graphs, after `warmup`
-    replayed steps: CUDA events on the launching stream, a synchronize (and a barrier
-    across ranks) on both sides."""
+WARM_MIN_S = 0.05  # the warm-up runs for at least this long (whole rotations of the layer buffers)
+
+
+def graph_time(step, steps, warmup, stream, dist=None, sampler=None, rotation=1):
+    """Milliseconds for `steps` calls of step(i) replayed from CUDA graphs, after the
+    warm-up: CUDA events on the launching stream, a synchronize (and a barrier across
+    ranks) on both sides.
+
+    The warm-up is at least `warmup` steps, in whole rotations over the `rotation` layer
+    buffers that step(i) cycles through, replayed until WARM_MIN_S has passed, so that the
+    timed steps start from the steady state of a running decode loop that keeps cycling
+    over all its layers (a cold rotation measured 20.4 us/step over 20 steps at 128K,
+    against 19.3 after this warm-up and 18.9 over 2000 steps).  The number of warm-up
+    steps run is left in graph_time.last_warmup_steps."""
     import contextlib
 
     import torch
@@ -517,13 +527,32 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None):
     g_chunk = capture(chunk, (ev0, ev1) if inside else None)
     rem = steps % chunk
     g_rem = capture(rem) if rem else None
-    g_warm = capture(warmup)
+    rotation = max(1, rotation)
+    n_warm = -(-max(warmup, 1) // rotation) * rotation
+    g_warm = capture(n_warm)
     for g in (g_chunk, g_rem, g_warm):
         if g is not None:
             graph_upload(g, stream)
     torch.cuda.synchronize()
+    reps = 0
+    t0 = time.perf_counter()
     with torch.cuda.stream(stream):  # graph replays go to torch's current stream: the timed one
-        g_warm.replay()
+        while True:
+            g_warm.replay()
+            torch.cuda.synchronize()
+            reps += 1
+            if time.perf_counter() - t0 >= WARM_MIN_S:
+                break
+    if dist:  # every rank replays the same number of times (the slowest rank's count)
+        import torch.distributed as tdist
+
+        r = torch.tensor([reps], dtype=torch.int64, device=torch.device("cuda", torch.cuda.current_device()))
+        tdist.all_reduce(r, op=tdist.ReduceOp.MAX)
+        with torch.cuda.stream(stream):
+            for _ in range(int(r.item()) - reps):
+                g_warm.replay()
+        reps = int(r.item())
+    graph_time.last_warmup_steps = reps * n_warm
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -663,7 +692,8 @@ def run_gpu(args, wl):
                            None, ws, stream)
 
     sampler = ClockSampler(local)
-    ms = graph_time(step, args.steps, args.warmup, stream, dist, sampler)
+    ms = graph_time(step, args.steps, args.warmup, stream, dist, sampler, rotation=R)
+    warm_run = graph_time.last_warmup_steps
     ms = max_over_ranks(ms, dist, dev)
     if dist:
         dist.barrier()
@@ -701,7 +731,7 @@ def run_gpu(args, wl):
             H.hata_dense_decode(dims, L["q"], L["K"], L["V"], L["lens"], 0.0, L["out"], dws, stream)
 
         d_steps = min(args.steps, 2000)
-        d_ms = graph_time(dense_step, d_steps, args.warmup, stream) / d_steps
+        d_ms = graph_time(dense_step, d_steps, args.warmup, stream, rotation=R) / d_steps
         d_bytes = sum(2 * int(Lb) * wl.n_kv_heads * wl.head_dim * 2 for Lb in inp["seq_lens"]) + \
             2 * wl.batch * wl.n_q_heads * wl.head_dim * 2
         dense = {"kernel": "hata_dense_decode (dense flash-decode, bf16 tensor-core tiles)", "steps": d_steps,
@@ -746,11 +776,12 @@ def run_gpu(args, wl):
                                      0.0, L["out"], None, None, ws, stream)
 
         p_steps = min(args.steps, 2000)
-        p_ms = graph_time(paged_step, p_steps, args.warmup, stream) / p_steps
+        p_ms = graph_time(paged_step, p_steps, args.warmup, stream, rotation=R) / p_steps
         paged = {"kernel": "hata_decode_step_paged (256-token blocks, random block table)", "steps": p_steps,
                  "us_per_step": p_ms * 1e3, "achieved_gbs": step_bytes / (p_ms * 1e-3) / 1e9,
                  "vs_unpaged": ms_per_step / p_ms}
     timing = ls.timing_note(args.steps)
+    timing["warmup_steps_run"] = warm_run  # >= args.warmup: whole rotations for at least WARM_MIN_S
     del ls, layers
     torch.cuda.empty_cache()
 
@@ -773,7 +804,7 @@ def run_gpu(args, wl):
                                L["out"], None, None, ls2.ws, stream)
 
         n2 = min(args.steps, 2000)
-        ms2 = graph_time(step2, n2, args.warmup, stream) / n2
+        ms2 = graph_time(step2, n2, args.warmup, stream, rotation=ls2.R) / n2
         if H.hata_read_device_status(ls2.ws) != 0:
             raise RuntimeError(f"device status set on workload {name}")
         gbs2 = ls2.step_bytes / (ms2 * 1e-3) / 1e9
