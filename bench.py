@@ -706,14 +706,17 @@ def run_gpu(args, wl):
     # copies its inputs (q and the new token's K and V rows) from pinned host memory in one
     # copy, appends the rows to the caches (hata_append_kv), runs hata_decode_step with the
     # output in pinned host memory, and waits for it
-    # (at least 200 timed steps, after 20 untimed ones, so that a short run's figure is not one
-    # cold step's)
-    e2e_steps = max(200, min(args.steps, 2000))
+    # (at least 1000 timed steps, after untimed loop calls for at least WARM_MIN_S, so that a
+    # short run's figure is the running loop's and not its cold start's)
+    e2e_steps = max(1000, min(args.steps, 2000))
     in_host, out_host = e2e_inputs(wl, layers[0], inp["seq_lens"])
     stages = [torch.empty_like(in_host, device=dev) for _ in layers]
     h2d = in_host.numel() * in_host.element_size()
     d2h = out_host.numel() * out_host.element_size()
-    run_e2e(H, dims, wl.k, 20, layers, stages, in_host, out_host, ws, stream)  # warm-up
+    e2e_warm, t_w = 0, time.perf_counter()
+    while e2e_warm == 0 or time.perf_counter() - t_w < WARM_MIN_S:  # warm-up
+        run_e2e(H, dims, wl.k, 100, layers, stages, in_host, out_host, ws, stream)
+        e2e_warm += 100
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -846,7 +849,7 @@ def run_gpu(args, wl):
             "algorithmic_bytes_per_step": step_bytes,
         },
         "e2e": {"value": e2e_value, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps, "host_wall_ms": e2e_host_ms,
+                "steps": e2e_steps, "warmup_steps_run": e2e_warm, "host_wall_ms": e2e_host_ms,
                 "loop": "native loop over the C ABI, every step: one H2D of q and the new K/V rows, "
                         "hata_append_kv, hata_decode_step writing its output into mapped pinned host memory "
                         "(the D2H bytes), stream synchronize"},
