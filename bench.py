@@ -543,16 +543,7 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None, rotation=1)
             reps += 1
             if time.perf_counter() - t0 >= WARM_MIN_S:
                 break
-    if dist:  # every rank replays the same number of times (the slowest rank's count)
-        import torch.distributed as tdist
-
-        r = torch.tensor([reps], dtype=torch.int64, device=torch.device("cuda", torch.cuda.current_device()))
-        tdist.all_reduce(r, op=tdist.ReduceOp.MAX)
-        with torch.cuda.stream(stream):
-            for _ in range(int(r.item()) - reps):
-                g_warm.replay()
-        reps = int(r.item())
-    graph_time.last_warmup_steps = reps * n_warm
+    graph_time.last_warmup_steps = reps * n_warm  # this rank's; the barrier below aligns the ranks
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
