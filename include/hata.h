@@ -341,8 +341,10 @@ HATA_API hata_status_t hata_prefill_attention(const hata_dims_t* dims, const voi
 HATA_API hata_status_t hata_topk_noalloc(const hata_dims_t* dims, const int32_t* scores, const int32_t* seq_lens,
                                          int k, int32_t* idx, int32_t* n_sel, void* stream);
 
-/* Number of kernels one hata_decode_step call with these dims and k enqueues
- * (1 when the fused persistent kernel applies), or -1 for invalid dims. */
+/* Number of kernels one hata_decode_step call with these dims and k enqueues:
+ * 1 for the cluster form, 3 for the all-SM form (see HATA_FLAG_ALL_SM_SCAN), 6
+ * for the granular chain (r = 16, or shapes neither fused form covers), or -1
+ * for invalid dims. */
 HATA_API int hata_decode_step_kernel_count(const hata_dims_t* dims, int k);
 
 /* Wait for `stream`, then return the workspace's device status word (a
