@@ -487,6 +487,13 @@ def graph_upload(g, stream):
 WARM_MIN_S = 0.05  # the warm-up runs for at least this long (whole rotations of the layer buffers)
 
 
+def warmup_pass_steps(warmup, rotation):
+    """Steps in one replay of the warm-up graph: at least `warmup` (and at least one), rounded
+    up to whole rotations over the `rotation` layer buffers."""
+    rotation = max(1, rotation)
+    return -(-max(warmup, 1) // rotation) * rotation
+
+
 def graph_time(step, steps, warmup, stream, dist=None, sampler=None, rotation=1):
     """Milliseconds for `steps` calls of step(i) replayed from CUDA graphs, after the
     warm-up: CUDA events on the launching stream, a synchronize (and a barrier across
@@ -527,8 +534,7 @@ def graph_time(step, steps, warmup, stream, dist=None, sampler=None, rotation=1)
     g_chunk = capture(chunk, (ev0, ev1) if inside else None)
     rem = steps % chunk
     g_rem = capture(rem) if rem else None
-    rotation = max(1, rotation)
-    n_warm = -(-max(warmup, 1) // rotation) * rotation
+    n_warm = warmup_pass_steps(warmup, rotation)
     g_warm = capture(n_warm)
     for g in (g_chunk, g_rem, g_warm):
         if g is not None:
