@@ -18,6 +18,8 @@
 // Partials (max, sum, weighted V) go to the workspace; the last CTA of each
 // (batch, KV head) to arrive merges them (log-sum-exp) and resets the counter.
 #include <algorithm>
+#include <map>
+#include <mutex>
 
 #include "hata_kernels.cuh"
 
@@ -267,10 +269,29 @@ __global__ void __launch_bounds__(kDnThreads, 2) dense_decode_kernel(const Dense
   if (tid == 0) p.count[u] = 0u;
 }
 
+// Per device: the shared-memory attribute of dense_decode_kernel<G>, set once under a
+// mutex; a failed attribute call is returned on every later launch on that device.
+template <int G>
+cudaError_t dense_attr_g() {
+  static std::mutex mu;
+  static std::map<int, cudaError_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = done.find(dev);
+  if (it == done.end()) {
+    e = cudaFuncSetAttribute(dense_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(2 * kDnStageB + 8 * kDnTile * 6));
+    if (e != cudaSuccess) (void)cudaGetLastError();
+    it = done.emplace(dev, e).first;
+  }
+  return it->second;
+}
+
 template <int G>
 cudaError_t launch_dense_g(const DenseParams& prm, int units, size_t smem, cudaStream_t st) {
-  static cudaError_t attr = cudaFuncSetAttribute(dense_decode_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(2 * kDnStageB + 8 * kDnTile * 6));
+  const cudaError_t attr = dense_attr_g<G>();
   if (attr != cudaSuccess) return attr;
   dense_decode_kernel<G><<<dim3((unsigned)prm.nsplit, (unsigned)units), kDnThreads, smem, st>>>(prm);
   return cudaGetLastError();
@@ -280,20 +301,36 @@ cudaError_t launch_dense_g(const DenseParams& prm, int units, size_t smem, cudaS
 
 // Tokens per CTA: the splits of all units fill the CTAs that fit on the device
 // at once (one wave), rounded to whole tiles.
-int dense_split(const hata_dims_t& d) {
-  static int slots = 0;
-  if (!slots) {
-    int dev = 0, sms = 0, per_sm = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+// CTAs of one wave on the current device (SMs x resident CTAs), found once per device
+// under a mutex.
+int dense_slots() {
+  static std::mutex mu;
+  static std::map<int, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    dev = -1;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    int sms = 0, per_sm = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 1;
     const size_t smem = 2 * kDnStageB + (size_t)8 * kDnTile * 6;
-    cudaFuncSetAttribute(dense_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dense_decode_kernel<8>, kDnThreads, smem) !=
-        cudaSuccess)
+    if (dev < 0 ||
+        cudaFuncSetAttribute(dense_decode_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dense_decode_kernel<8>, kDnThreads, smem) !=
+            cudaSuccess)
       per_sm = 1;
     (void)cudaGetLastError();
-    slots = std::max(1, sms * std::max(1, per_sm));
+    it = cache.emplace(dev, std::max(1, std::max(1, sms) * std::max(1, per_sm))).first;
   }
+  return it->second;
+}
+
+int dense_split(const hata_dims_t& d) {
+  const int slots = dense_slots();
   const long long units = (long long)d.batch * d.n_kv_heads;
   const long long per_unit = std::max(1LL, slots / units);
   const long long split = (d.max_seq + per_unit - 1) / per_unit;

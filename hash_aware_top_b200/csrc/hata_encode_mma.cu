@@ -21,6 +21,9 @@
 // columns) pair are gathered with four ballots and written as one u16, and the
 // tile's codes leave as whole words.  CTAs are persistent per (batch, head).
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "hata_kernels.cuh"
 
@@ -176,15 +179,29 @@ cudaError_t launch_encode_mma(const hata_dims_t& d, const void* x, int x_heads, 
                               const int32_t* seq_end, const float* W, uint32_t* codes, int codes_len,
                               cudaStream_t st) {
   if (d.dtype != HATA_BF16 || d.hash_bits > 128 || d.hash_bits < 32) return cudaErrorNotSupported;
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms < 1) sms = 1;
-    cudaFuncSetAttribute(encode_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
-    cudaFuncSetAttribute(encode_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
-    cudaFuncSetAttribute(encode_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+  // Per device, once under a mutex: the SM count and the shared-memory attributes of the
+  // three instantiations.  A failed attribute call makes this form unavailable on that
+  // device (cudaErrorNotSupported: the caller uses the SIMT encode).
+  static std::mutex mu;
+  static std::map<int, std::pair<bool, int>> setup;
+  int dev = 0;
+  const cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess) return de;
+  int sms = 1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = setup.find(dev);
+    if (it == setup.end()) {
+      int n = 0;
+      cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_mma_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_mma_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(encode_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmSmem);
+      if (e != cudaSuccess) (void)cudaGetLastError();
+      it = setup.emplace(dev, std::make_pair(e == cudaSuccess, std::max(n, 1))).first;
+    }
+    if (!it->second.first) return cudaErrorNotSupported;
+    sms = it->second.second;
   }
   const int hpg = x_heads / d.n_kv_heads;
   const long long heads = (long long)d.batch * x_heads;
